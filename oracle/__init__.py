@@ -1,0 +1,19 @@
+"""CPU oracle for GQE prefill (test infrastructure, not product code).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The library under
+``moe_routed_grouped_b200`` never calls it and shares no code with it.
+"""
+from .gqe_oracle import (  # noqa: F401
+    bf16_to_f64,
+    router_logits,
+    route,
+    topk_exact_order,
+    bucket,
+    causal_attention,
+    gqe_prefill,
+    gqe_prefill_rows,
+    dense_gqa,
+    dense_gqa_repeat,
+    kv_cache_bytes,
+)

@@ -1,0 +1,329 @@
+"""Plain, slow CPU oracle for causal GQE prefill (float64).
+
+TEST INFRASTRUCTURE ONLY.  Imported by ``tests/``, ``__graft_entry__.smoke()``
+and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py``; never by
+the library.  It shares no code with the CUDA path: the only thing both sides
+use is the seeded input generator in ``synth``, which holds none of the
+method's arithmetic.
+
+Sources (web pages; cited by title and section):
+
+* [GQE review] "论文综述：分组查询专家——在 GQA 自注意力上引入混合专家"
+  (review of *Grouped Query Experts*), §二 核心方法与创新: sub-sections
+  "整体设计" (N heads, G groups, M = N/G experts), "路由器" (softmax then
+  top-k), "输出怎么拼起来：三个关键部件" (hard-selected slots, renormalised
+  weighted-sum slot, always-on shared head, concat feeding W_O).
+* [GQE abstract] "Grouped Query Experts: Mixture-of-Experts on GQA
+  Self-Attention" (1kpapers summary page), "01 In brief": 9 of 16 query
+  attentions active.
+* [GQA article] "AI 大模型之 GQA": §4.1 (KV bytes 2·L·G·d·S·b), §4.2 (the
+  512 MiB / 2048 MiB worked value), "技术深化 分组查询的张量映射与权重转换"
+  (head i reads KV head floor(i/(H/G)); explicit map vs logical repeat), and
+  "工程实操 非方形因果遮罩与头分片检查" (causal mask on absolute positions).
+* [MQA/GQA explainer] "MQA、GQA、稀疏/滑动窗口注意力及混合范式": the MQA and
+  GQA numeric examples and the KV-cache byte examples.
+
+Readings where the pages are silent (also listed in the design doc):
+
+* r_g is linear, ``l = x · W_r[g]`` (+ an optional per-(g, m) bias).
+* Top-k is decided on the EXACT real-valued logits (softmax is strictly
+  monotone, so this is the same as exact p); ties go to the lower expert
+  index; the k selected experts are stored in rank order (slot j = rank).
+* The weighted-sum slot is per group: ō_{i,g} = Σ_j w_{i,g,j} o_{i,g,j}.
+* The shared head's query is the given Qs; it attends over KV head 0.
+* Scale 1/sqrt(d), causal: key position <= query position (diagonal kept).
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, the pages' worked values, brute force, invariants).
+"""
+from __future__ import annotations
+
+import functools
+import math
+from typing import Optional, Tuple
+
+import numpy as np
+
+_U = 2.0 ** -53  # unit roundoff of float64
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of bf16 bit patterns as float64."""
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# small helpers kept separate so the pin tests can plant mistakes in them
+# ---------------------------------------------------------------------------
+
+def _kv_head_of(h: int, N: int, G: int) -> int:
+    """[GQA article] 技术深化: query head i reads KV head floor(i / (H/G))."""
+    return h // (N // G)
+
+
+def _expert_head(g: int, m, M: int):
+    """[GQE review] 整体设计: expert m of group g is query head g*M + m."""
+    return g * M + m
+
+
+def _scale(d: int) -> float:
+    """[GQA article] 最小参考实现: scores are divided by sqrt(d)."""
+    return 1.0 / math.sqrt(d)
+
+
+def _visible(key_pos: np.ndarray, query_pos: np.ndarray) -> np.ndarray:
+    """[GQA article] 工程实操 step 1: a key is visible iff key pos <= query pos."""
+    return key_pos[None, :] <= query_pos[:, None]
+
+
+# ---------------------------------------------------------------------------
+# router
+# ---------------------------------------------------------------------------
+
+def router_logits(x: np.ndarray, Wr: np.ndarray, bias: Optional[np.ndarray]
+                  ) -> Tuple[np.ndarray, np.ndarray]:
+    """Router logits l[t, g, m] = sum_j x[t, j] W_r[g, j, m] (+ bias[g, m]).
+
+    [GQE review] 路由器: p_{i,g} = softmax(r_g(x_i)); r_g read as linear.
+    Returns the float64 logits and a rigorous bound on their rounding error:
+    every bf16*bf16 product is exact in float64, so a d_model-term sum plus the
+    bias carries at most (d_model + 1) roundings of relative size 2^-53 of
+    sum |x_j w_jm| + |bias| (any summation order).  The bound is doubled for
+    the rounding of that magnitude itself.
+    """
+    T, dm = x.shape
+    G, dm2, M = Wr.shape
+    assert dm == dm2
+    W2 = np.ascontiguousarray(Wr.transpose(1, 0, 2).reshape(dm, G * M))
+    L = (x @ W2).reshape(T, G, M)
+    A = (np.abs(x) @ np.abs(W2)).reshape(T, G, M)
+    if bias is not None:
+        b = np.asarray(bias, dtype=np.float64).reshape(1, G, M)
+        L = L + b
+        A = A + np.abs(b)
+    err = 2.0 * (dm + 2) * _U * A
+    return L, err
+
+
+def topk_exact_order(x_row: np.ndarray, W_g: np.ndarray, bias_g: Optional[np.ndarray]
+                     ) -> list:
+    """All M experts of one (token, group) ordered by EXACT logit, desc.
+
+    Exact ties are broken towards the lower expert index.  The sign of
+    l_a - l_b is taken from ``math.fsum`` over the exact float64 products
+    (x_j * w_ja, -x_j * w_jb, bias_a, -bias_b): fsum returns the correctly
+    rounded exact sum, so its sign is the sign of the exact difference.
+    """
+    M = W_g.shape[1]
+    bias_g = np.zeros(M) if bias_g is None else np.asarray(bias_g, dtype=np.float64)
+    prods = [(x_row * W_g[:, m]).tolist() for m in range(M)]
+
+    def before(a: int, b: int) -> int:
+        s = math.fsum(prods[a] + [-v for v in prods[b]] + [float(bias_g[a]), -float(bias_g[b])])
+        if s > 0 or (s == 0 and a < b):
+            return -1
+        return 1
+
+    return sorted(range(M), key=functools.cmp_to_key(before))
+
+
+def route(x_bits: np.ndarray, Wr_bits: np.ndarray, bias: Optional[np.ndarray], k: int):
+    """GQE router: logits -> softmax over the group's M experts -> top-k -> w.
+
+    [GQE review] 路由器 and 三个关键部件 (renormalised weights
+    w = p / sum_{m' in K_g} p).  x_bits [B,S,dm] and Wr_bits [G,dm,M] are bf16
+    bit patterns.  Returns (topk_idx int32 [B,S,G,k] in rank order,
+    p float64 [B,S,G,M], w float64 [B,S,G,k], n_exact) where n_exact counts
+    the (token, group) pairs decided by the exact comparison.
+    """
+    B, S, dm = x_bits.shape
+    G, _, M = Wr_bits.shape
+    if not 1 <= k <= M:
+        raise ValueError("need 1 <= k <= M")
+    x = bf16_to_f64(x_bits).reshape(B * S, dm)
+    Wr = bf16_to_f64(Wr_bits)
+    L, err = router_logits(x, Wr, bias)
+
+    # candidate order from the float64 estimate (stable: lower index first)
+    order = np.argsort(-L, axis=-1, kind="stable")
+    Ls = np.take_along_axis(L, order, axis=-1)
+    Es = np.take_along_axis(err, order, axis=-1)
+    lo = Ls - Es
+    hi = Ls + Es
+    certain = np.ones(L.shape[:2], dtype=bool)
+    for r in range(min(k, M - 1)):
+        # rank r must be certainly above every later rank
+        rest_hi = hi[..., r + 1:].max(axis=-1)
+        certain &= lo[..., r] > rest_hi
+    idx = order[..., :k].copy()
+
+    unsure = np.argwhere(~certain)
+    for t, g in unsure:
+        ordr = topk_exact_order(x[t], Wr[g], None if bias is None else bias[g])
+        idx[t, g] = ordr[:k]
+
+    # p = softmax over the group's M experts (float64)
+    mx = L.max(axis=-1, keepdims=True)
+    e = np.exp(L - mx)
+    p = e / e.sum(axis=-1, keepdims=True)
+    psel = np.take_along_axis(p, idx, axis=-1)
+    den = np.zeros(psel.shape[:-1])
+    for j in range(k):  # ascending slot order
+        den = den + psel[..., j]
+    w = psel / den[..., None]
+    return (idx.reshape(B, S, G, k).astype(np.int32), p.reshape(B, S, G, M),
+            w.reshape(B, S, G, k), int(len(unsure)))
+
+
+# ---------------------------------------------------------------------------
+# bucketing
+# ---------------------------------------------------------------------------
+
+def bucket(topk_idx: np.ndarray, M: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Stable per-(batch, group, expert) lists of token positions.
+
+    For b, g, m in that order: the tokens i (ascending) whose selected set
+    K_g(x_i) contains m ([GQE review] 路由器: only selected heads compute).
+    Returns (bucket_off int64 [B*G*M+1] exclusive scan, bucket_tok int32).
+    """
+    B, S, G, k = topk_idx.shape
+    off = [0]
+    toks = []
+    for b in range(B):
+        for g in range(G):
+            sel = topk_idx[b, :, g, :]
+            for m in range(M):
+                members = np.nonzero((sel == m).any(axis=-1))[0]
+                toks.append(members.astype(np.int32))
+                off.append(off[-1] + len(members))
+    return np.asarray(off, dtype=np.int64), (np.concatenate(toks) if toks else
+                                             np.zeros(0, np.int32))
+
+
+# ---------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------
+
+def causal_attention(q: np.ndarray, pos: np.ndarray, K: np.ndarray, V: np.ndarray,
+                     dtype=np.float64, row_chunk: int = 512) -> np.ndarray:
+    """Softmax attention of query rows at absolute positions ``pos``.
+
+    o_r = sum_{t <= pos_r} softmax_t(q_r . K_t / sqrt(d)) V_t.
+    [GQA article] 最小参考实现 (scaled dot product, softmax, times V) and
+    工程实操 (mask by absolute position, not by a top-left triangle).
+    Rows are independent; they are processed in chunks only to bound memory.
+    """
+    q = np.asarray(q, dtype=dtype)
+    K = np.asarray(K, dtype=dtype)
+    V = np.asarray(V, dtype=dtype)
+    pos = np.asarray(pos, dtype=np.int64)
+    R, d = q.shape
+    out = np.empty((R, V.shape[1]), dtype=dtype)
+    sc = dtype(_scale(d))
+    for s in range(0, R, row_chunk):
+        e = min(R, s + row_chunk)
+        pm = int(pos[s:e].max())
+        keys = np.arange(pm + 1)
+        sco = (q[s:e] @ K[: pm + 1].T) * sc
+        sco = np.where(_visible(keys, pos[s:e]), sco, -np.inf)
+        mx = sco.max(axis=1, keepdims=True)
+        p = np.exp(sco - mx)
+        out[s:e] = (p @ V[: pm + 1]) / p.sum(axis=1, keepdims=True)
+    return out
+
+
+def gqe_prefill(Q_bits, Qs_bits, K_bits, V_bits, topk_idx, w, dtype=np.float64):
+    """Routed GQE causal prefill: selected heads, weighted-sum slot, shared head.
+
+    [GQE review] 三个关键部件: O_i are the selected heads' outputs (slot j =
+    rank j of the selection), ō_{i,g} = sum_j w_{i,g,j} o_{i,g,j}, and the
+    always-on shared head s(x_i); the three are concatenated before W_O.
+    Q [B,S,N,d], Qs [B,S,d], K/V [B,S,G,d] as bf16 bits.  Returns
+    (O_sel [B,S,G,k,d], o_bar [B,S,G,d], s [B,S,d]).
+    """
+    B, S = Q_bits.shape[:2]
+    O_sel, o_bar, s_out = gqe_prefill_rows(Q_bits, Qs_bits, K_bits, V_bits, topk_idx, w,
+                                           rows=[np.arange(S)] * B, dtype=dtype)
+    return np.stack(O_sel), np.stack(o_bar), np.stack(s_out)
+
+
+def gqe_prefill_rows(Q_bits, Qs_bits, K_bits, V_bits, topk_idx, w, rows, dtype=np.float64):
+    """Like :func:`gqe_prefill` but only for token positions ``rows[b]``.
+
+    Returns three lists over b of arrays indexed by the requested rows.
+    """
+    B, S, N, d = Q_bits.shape
+    G = K_bits.shape[2]
+    M = N // G
+    k = topk_idx.shape[-1]
+    O_sel, o_bar, s_out = [], [], []
+    for b in range(B):
+        r = np.asarray(rows[b], dtype=np.int64)
+        Kb = bf16_to_f64(K_bits[b])
+        Vb = bf16_to_f64(V_bits[b])
+        Ob = np.zeros((len(r), G, k, d), dtype=dtype)
+        for g in range(G):
+            for j in range(k):
+                heads = _expert_head(g, topk_idx[b, r, g, j].astype(np.int64), M)
+                q = bf16_to_f64(Q_bits[b, r, heads])
+                Ob[:, g, j] = causal_attention(q, r, Kb[:, g], Vb[:, g], dtype=dtype)
+        wb = np.asarray(w[b, r], dtype=dtype)
+        ob = np.zeros((len(r), G, d), dtype=dtype)
+        for j in range(k):  # ascending slot order
+            ob = ob + wb[:, :, j, None] * Ob[:, :, j]
+        sb = causal_attention(bf16_to_f64(Qs_bits[b, r]), r, Kb[:, 0], Vb[:, 0], dtype=dtype)
+        O_sel.append(Ob)
+        o_bar.append(ob)
+        s_out.append(sb)
+    return O_sel, o_bar, s_out
+
+
+def dense_gqa(Q_bits, K_bits, V_bits, dtype=np.float64, rows=None):
+    """Dense GQA (every query head active), explicit head -> KV-head map.
+
+    [GQA article] 最小参考实现 (first form: loop over heads, g = i // (H/G));
+    [GQE review] §四: the all-active GQA baseline.  Returns O [B,S,N,d]
+    (or [B][rows] lists when ``rows`` is given).
+    """
+    B, S, N, d = Q_bits.shape
+    G = K_bits.shape[2]
+    outs = []
+    for b in range(B):
+        r = np.arange(S) if rows is None else np.asarray(rows[b], dtype=np.int64)
+        Kb = bf16_to_f64(K_bits[b])
+        Vb = bf16_to_f64(V_bits[b])
+        Ob = np.zeros((len(r), N, d), dtype=dtype)
+        for h in range(N):
+            g = _kv_head_of(h, N, G)
+            Ob[:, h] = causal_attention(bf16_to_f64(Q_bits[b, r, h]), r, Kb[:, g], Vb[:, g],
+                                        dtype=dtype)
+        outs.append(Ob)
+    return np.stack(outs) if rows is None else outs
+
+
+def dense_gqa_repeat(Q_bits, K_bits, V_bits, dtype=np.float64):
+    """Dense GQA by logical repeat of the KV heads (the second form).
+
+    [GQA article] 最小参考实现: K and V repeated H/G times along the head axis,
+    then one batched causal attention over all heads.  Only for small inputs.
+    """
+    B, S, N, d = Q_bits.shape
+    G = K_bits.shape[2]
+    Q = bf16_to_f64(Q_bits).astype(dtype)
+    Kr = np.repeat(bf16_to_f64(K_bits), N // G, axis=2).astype(dtype)
+    Vr = np.repeat(bf16_to_f64(V_bits), N // G, axis=2).astype(dtype)
+    q = Q.transpose(0, 2, 1, 3)    # [B,N,S,d]
+    kk = Kr.transpose(0, 2, 3, 1)  # [B,N,d,S]
+    vv = Vr.transpose(0, 2, 1, 3)  # [B,N,S,d]
+    sco = (q @ kk) * dtype(_scale(d))
+    pos = np.arange(S)
+    sco = np.where(_visible(pos, pos)[None, None], sco, -np.inf)
+    p = np.exp(sco - sco.max(axis=-1, keepdims=True))
+    o = (p @ vv) / p.sum(axis=-1, keepdims=True)
+    return o.transpose(0, 2, 1, 3)
+
+
+def kv_cache_bytes(L: int, G: int, S: int, d: int, b: int, B: int = 1) -> int:
+    """[GQA article] §4.1: KV bytes per sequence = 2 * L * G * d * S * b (times B)."""
+    return 2 * L * G * d * S * b * B

@@ -1,0 +1,492 @@
+"""Pins for the CPU oracle: facts fixed by the pages or by mathematics.
+
+Each ``check_*`` function raises AssertionError when the oracle is wrong.  The
+``test_*`` functions run them; ``test_planted_*`` plant a plausible mistake in
+one oracle helper (on the CPU) and require that some pin catches it.
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.gqe_oracle as og
+from synth import f32_to_bf16_bits, normal_bf16, bf16_bits_to_f32
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bits(a):
+    return f32_to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------
+# KV-cache bytes (GQA article §4.1/§4.2; MQA/GQA explainer 数值示例)
+# --------------------------------------------------------------------------
+
+def check_kv_bytes():
+    for c in _gold("kv_cache_bytes.json")["cases"]:
+        got = oracle.kv_cache_bytes(c["L"], c["G"], c["S"], c["d"], c["b"])
+        if "bytes" in c:
+            assert got == c["bytes"], (c["cite"], got)
+        if "MiB" in c:
+            assert got == c["MiB"] * 2 ** 20, (c["cite"], got)
+
+
+def test_kv_cache_bytes_pages():
+    check_kv_bytes()
+
+
+# --------------------------------------------------------------------------
+# worked GQA / MQA examples (MQA/GQA explainer)
+# --------------------------------------------------------------------------
+
+def _example_tensors(ex):
+    h, G, d = ex["h"], ex["G"], ex["d"]
+    Q = np.asarray(ex["Q"], dtype=np.float32).reshape(1, 1, h, d)
+    K = np.asarray(ex["K"], dtype=np.float32).reshape(1, 1, G, d)
+    V = np.asarray(ex["V"], dtype=np.float32).reshape(1, 1, G, d)
+    return _bits(Q), _bits(K), _bits(V)
+
+
+def check_worked_examples():
+    g = _gold("gqa_examples.json")
+    for key in ("gqa", "mqa"):
+        ex = g[key]
+        Q, K, V = _example_tensors(ex)
+        out = oracle.dense_gqa(Q, K, V)
+        assert out.reshape(-1).tolist() == ex["expect_concat"], (ex["cite"], out.reshape(-1))
+        # the scaled score of head 0 against its own KV head
+        q0 = np.asarray(ex["Q"][0], float)
+        k0 = np.asarray(ex["K"][0], float)
+        s = float(q0 @ k0) * og._scale(ex["d"])
+        assert abs(s - ex["expect_scaled_score"]) < 5e-5, (ex["cite"], s)
+
+
+def test_worked_gqa_mqa_examples():
+    check_worked_examples()
+
+
+def check_worked_example_routed():
+    """The GQA example through the routed path with k = M (every head selected)."""
+    ex = _gold("gqa_examples.json")["gqa"]
+    Q, K, V = _example_tensors(ex)
+    M = ex["h"] // ex["G"]
+    idx = np.tile(np.arange(M, dtype=np.int32), (1, 1, ex["G"], 1))  # [1,1,G,M]
+    w = np.full((1, 1, ex["G"], M), 1.0 / M)
+    Qs = _bits(np.zeros((1, 1, ex["d"])))
+    O_sel, _, _ = oracle.gqe_prefill(Q, Qs, K, V, idx, w)
+    assert O_sel.reshape(-1).tolist() == ex["expect_concat"]
+
+
+def test_worked_example_routed():
+    check_worked_example_routed()
+
+
+def test_active_head_count():
+    a = _gold("gqa_examples.json")["active_heads"]
+    from synth import WORKLOADS
+    w = WORKLOADS["layer250m"]
+    assert (w.N, w.G, w.k) == (a["N"], a["G"], a["k"])
+    assert w.G * w.k + 1 == a["active"]
+    assert math.isclose(w.useful_flop_routed() / w.useful_flop_dense(), a["active"] / a["N"])
+
+
+# --------------------------------------------------------------------------
+# causal attention closed forms
+# --------------------------------------------------------------------------
+
+def check_geometric_scores():
+    """Scores s_t = t (after the 1/sqrt(d) scale) and one-hot V give the
+    softmax itself, whose closed form is a geometric series:
+    o_t = e^t (e - 1) / (e^(P+1) - 1) for t <= P."""
+    S, d = 12, 4
+    q = np.zeros((S, d)); q[:, 0] = 2.0          # q . K_t = 2t, / sqrt(4) = t
+    K = np.zeros((S, d)); K[:, 0] = np.arange(S)
+    V = np.eye(S)
+    pos = np.arange(S)
+    o = oracle.causal_attention(q, pos, K, V)
+    e = math.e
+    for P in range(S):
+        for t in range(S):
+            want = (e ** t) * (e - 1) / (e ** (P + 1) - 1) if t <= P else 0.0
+            assert abs(o[P, t] - want) < 1e-12, (P, t, o[P, t], want)
+
+
+def test_geometric_closed_form():
+    check_geometric_scores()
+
+
+def check_nonsquare_positions():
+    """Queries at absolute positions 5 and 6 over keys 0..6 see 6 and 7 keys."""
+    c = _gold("gqa_examples.json")["nonsquare_causal"]
+    n = c["n_keys"]
+    q = np.ones((2, 8))
+    K = np.ones((n, 8))        # identical keys: uniform weights over visible keys
+    V = np.eye(n)
+    o = oracle.causal_attention(q, np.asarray(c["query_pos"]), K, V)
+    for r, nv in enumerate(c["visible"]):
+        want = np.array([1.0 / nv] * nv + [0.0] * (n - nv))
+        assert np.allclose(o[r], want, atol=1e-15, rtol=0), (r, o[r])
+
+
+def test_nonsquare_causal_positions():
+    check_nonsquare_positions()
+
+
+def check_head_to_kv_map():
+    """8 query heads, 2 KV heads: heads 0-3 read KV 0, heads 4-7 read KV 1.
+    KV heads are made numerically distinct (GQA article: make KV heads differ
+    so a mapping bug shows); identical K rows make each output the prefix
+    mean of its KV head's V."""
+    c = _gold("gqa_examples.json")["nonsquare_causal"]
+    H, G, S, d = c["H"], c["G"], 6, 4
+    Q = np.ones((1, S, H, d), np.float32)
+    K = np.ones((1, S, G, d), np.float32)
+    V = np.zeros((1, S, G, d), np.float32)
+    for g in range(G):
+        V[0, :, g, :] = (np.arange(S)[:, None] + 1) * (10.0 ** g)
+    out = oracle.dense_gqa(_bits(Q), _bits(K), _bits(V))
+    for h in range(H):
+        g = c["kv_of_head"][h]
+        for i in range(S):
+            want = np.mean(np.arange(1, i + 2)) * (10.0 ** g)
+            assert np.allclose(out[0, i, h], want, rtol=1e-14), (h, i, out[0, i, h], want)
+
+
+def test_head_to_kv_map():
+    check_head_to_kv_map()
+
+
+def check_row0_and_hull():
+    rng = np.random.default_rng(0)
+    S, d = 40, 16
+    q = rng.standard_normal((S, d)); K = rng.standard_normal((S, d)); V = rng.standard_normal((S, d))
+    o = oracle.causal_attention(q, np.arange(S), K, V)
+    assert np.array_equal(o[0], V[0])            # row 0 sees only key 0
+    for i in range(S):                           # convex combination of visible V
+        assert np.all(o[i] <= V[: i + 1].max(0) + 1e-12)
+        assert np.all(o[i] >= V[: i + 1].min(0) - 1e-12)
+    Vc = np.tile(rng.standard_normal((1, d)), (S, 1))   # constant V -> constant output
+    oc = oracle.causal_attention(q, np.arange(S), K, Vc)
+    assert np.allclose(oc, Vc, rtol=0, atol=1e-14)
+
+
+def test_row0_hull_constant_v():
+    check_row0_and_hull()
+
+
+def check_explicit_equals_repeat():
+    """GQA article 最小参考实现: explicit head map and logical repeat agree
+    (the page reports max_abs_error 0.0); KV heads are offset so they differ."""
+    B, S, N, G, d = 2, 33, 8, 2, 16
+    Q = normal_bf16((B, S, N, d), 11)
+    K = bf16_bits_to_f32(normal_bf16((B, S, G, d), 12))
+    V = bf16_bits_to_f32(normal_bf16((B, S, G, d), 13))
+    for g in range(G):
+        K[:, :, g] += 3.0 * g
+        V[:, :, g] += 5.0 * g
+    Kb, Vb = _bits(K), _bits(V)
+    a = oracle.dense_gqa(Q, Kb, Vb)
+    b = oracle.dense_gqa_repeat(Q, Kb, Vb)
+    assert np.max(np.abs(a - b)) <= 1e-12, np.max(np.abs(a - b))
+
+
+def test_explicit_equals_repeat():
+    check_explicit_equals_repeat()
+
+
+def test_fp32_variant_close_to_fp64():
+    rng_bits = normal_bf16((1, 128, 16, 64), 21)
+    K = normal_bf16((1, 128, 8, 64), 22)
+    V = normal_bf16((1, 128, 8, 64), 23)
+    a = oracle.dense_gqa(rng_bits, K, V, dtype=np.float64)
+    b = oracle.dense_gqa(rng_bits, K, V, dtype=np.float32)
+    rel = np.linalg.norm(a - b) / np.linalg.norm(a)
+    assert rel < 1e-5, rel
+
+
+# --------------------------------------------------------------------------
+# router
+# --------------------------------------------------------------------------
+
+def _exact_logits(xb, Wb, bias):
+    """Exact rational logits of bf16 inputs (independent of math.fsum)."""
+    x = bf16_bits_to_f32(xb).astype(np.float64)
+    W = bf16_bits_to_f32(Wb).astype(np.float64)
+    B, S, dm = x.shape
+    G, _, M = W.shape
+    out = {}
+    for b in range(B):
+        for i in range(S):
+            xs = [Fraction(float(v)) for v in x[b, i]]
+            for g in range(G):
+                for m in range(M):
+                    v = sum((xs[j] * Fraction(float(W[g, j, m])) for j in range(dm)), Fraction(0))
+                    if bias is not None:
+                        v += Fraction(float(bias[g, m]))
+                    out[(b, i, g, m)] = v
+    return out
+
+
+def check_topk_bruteforce(xb, Wb, bias, k):
+    B, S, dm = xb.shape
+    G, _, M = Wb.shape
+    idx, p, w, _ = oracle.route(xb, Wb, bias, k)
+    ex = _exact_logits(xb, Wb, bias)
+
+    def beats(a, b, key):
+        la, lb = ex[key + (a,)], ex[key + (b,)]
+        return la > lb or (la == lb and a < b)
+
+    for b in range(B):
+        for i in range(S):
+            for g in range(G):
+                key = (b, i, g)
+                valid = [set(c) for c in itertools.combinations(range(M), k)
+                         if all(beats(a, o, key) for a in c for o in range(M) if o not in c)]
+                assert len(valid) == 1, (key, valid)
+                got = list(idx[b, i, g])
+                assert set(got) == valid[0], (key, got, valid)
+                for j in range(k - 1):      # slots in rank order
+                    assert beats(got[j], got[j + 1], key), (key, got)
+    return idx, p, w
+
+
+def test_topk_bruteforce_random():
+    dm, G, M = 16, 3, 4
+    xb = normal_bf16((2, 9, dm), 31)
+    Wb = normal_bf16((G, dm, M), 32, std=0.25)
+    for k in (1, 2, 3, 4):
+        check_topk_bruteforce(xb, Wb, None, k)
+
+
+def test_topk_bruteforce_ties():
+    """Duplicated W_r columns force exact ties; the lower index must win."""
+    dm, G, M = 8, 2, 4
+    vals = np.array([-2, -1, -0.5, 0, 0.5, 1, 2], np.float32)
+    rng = np.random.default_rng(5)
+    x = vals[rng.integers(0, len(vals), (1, 20, dm))]
+    W = vals[rng.integers(0, len(vals), (G, dm, M))]
+    W[:, :, 2] = W[:, :, 0]          # expert 2 ties expert 0 on every token
+    W[1, :, 3] = W[1, :, 1]
+    xb, Wb = _bits(x), _bits(W)
+    for k in (1, 2, 3):
+        idx, _, _ = check_topk_bruteforce(xb, Wb, None, k)
+        # expert 2 can never rank above expert 0
+        for t in range(20):
+            got = list(idx[0, t, 0])
+            if 2 in got:
+                assert 0 in got and got.index(0) < got.index(2)
+
+
+def test_topk_ties_with_bias_and_exact_path_used():
+    dm, G, M = 8, 2, 2
+    x = np.ones((1, 6, dm), np.float32)
+    W = np.zeros((G, dm, M), np.float32)
+    W[:, :, 0] = 0.25
+    W[:, :, 1] = 0.125
+    bias = np.array([[0.0, 1.0], [0.0, 1.5]], np.float32)  # group 0 exact tie, group 1 expert 1 wins
+    idx, p, w, n_exact = oracle.route(_bits(x), _bits(W), bias, 1)
+    assert (idx[0, :, 0, 0] == 0).all()      # tie -> lower index
+    assert (idx[0, :, 1, 0] == 1).all()
+    assert n_exact >= 6                      # the tie went through the exact comparison
+    check_topk_bruteforce(_bits(x), _bits(W), bias, 1)
+
+
+def check_router_sums():
+    xb = normal_bf16((1, 64, 32), 41)
+    Wb = normal_bf16((4, 32, 4), 42, std=0.2)
+    for k in (1, 2, 4):
+        idx, p, w, _ = oracle.route(xb, Wb, None, k)
+        assert np.allclose(p.sum(-1), 1.0, rtol=0, atol=1e-14)
+        assert np.allclose(w.sum(-1), 1.0, rtol=0, atol=1e-14)
+        if k == 1:
+            assert (w == 1.0).all()
+        # top-1 is the arg-max of p
+        assert (np.take_along_axis(p, idx[..., :1].astype(np.int64), -1)[..., 0]
+                >= p.max(-1) - 1e-15).all()
+
+
+def test_router_sums():
+    check_router_sums()
+
+
+# --------------------------------------------------------------------------
+# buckets
+# --------------------------------------------------------------------------
+
+def check_buckets(idx, M):
+    B, S, G, k = idx.shape
+    off, tok = oracle.bucket(idx, M)
+    assert off[0] == 0 and off[-1] == B * G * S * k == len(tok)
+    # brute force: walk tokens in order and append
+    lists = {(b, g, m): [] for b in range(B) for g in range(G) for m in range(M)}
+    for b in range(B):
+        for i in range(S):
+            for g in range(G):
+                for j in range(k):
+                    lists[(b, g, int(idx[b, i, g, j]))].append(i)
+    n = 0
+    for b in range(B):
+        for g in range(G):
+            for m in range(M):
+                bi = (b * G + g) * M + m
+                seg = tok[off[bi]:off[bi + 1]].tolist()
+                assert seg == lists[(b, g, m)], (b, g, m)
+                assert all(seg[a] < seg[a + 1] for a in range(len(seg) - 1))
+                n += len(seg)
+    assert n == B * G * S * k
+
+
+def test_bucket_bruteforce():
+    xb = normal_bf16((3, 50, 16), 51)
+    Wb = normal_bf16((4, 16, 4), 52, std=0.3)
+    for k in (1, 2, 4):
+        idx, _, _, _ = oracle.route(xb, Wb, None, k)
+        check_buckets(idx, 4)
+
+
+def test_bucket_empty_expert():
+    idx = np.zeros((1, 10, 2, 1), np.int32)   # expert 1 never chosen
+    off, tok = oracle.bucket(idx, 2)
+    assert off.tolist() == [0, 10, 10, 20, 20]
+    check_buckets(idx, 2)
+
+
+# --------------------------------------------------------------------------
+# routed prefill
+# --------------------------------------------------------------------------
+
+def _small_problem(B=2, S=40, N=8, G=4, d=16, dm=16, seed=60):
+    return dict(
+        x=normal_bf16((B, S, dm), seed), Wr=normal_bf16((G, dm, N // G), seed + 1, std=0.25),
+        Q=normal_bf16((B, S, N, d), seed + 2), Qs=normal_bf16((B, S, d), seed + 3),
+        K=normal_bf16((B, S, G, d), seed + 4), V=normal_bf16((B, S, G, d), seed + 5))
+
+
+def check_routed_kM_equals_dense():
+    P = _small_problem()
+    N, G = P["Q"].shape[2], P["K"].shape[2]
+    M = N // G
+    idx, p, w, _ = oracle.route(P["x"], P["Wr"], None, M)
+    O_sel, _, s = oracle.gqe_prefill(P["Q"], P["Qs"], P["K"], P["V"], idx, w)
+    dense = oracle.dense_gqa(P["Q"], P["K"], P["V"])
+    B, S = P["Q"].shape[:2]
+    for b in range(B):
+        for i in range(S):
+            for g in range(G):
+                for j in range(M):
+                    h = g * M + int(idx[b, i, g, j])
+                    assert np.array_equal(O_sel[b, i, g, j], dense[b, i, h]), (b, i, g, j)
+
+
+def test_routed_kM_equals_dense():
+    check_routed_kM_equals_dense()
+
+
+def check_shared_head_is_dense_head_on_kv0():
+    P = _small_problem(seed=70)
+    idx, p, w, _ = oracle.route(P["x"], P["Wr"], None, 1)
+    _, _, s = oracle.gqe_prefill(P["Q"], P["Qs"], P["K"], P["V"], idx, w)
+    B, S, d = P["Qs"].shape
+    # a single-head, single-KV-head dense GQA over (Qs, K[:, :, 0], V[:, :, 0])
+    ref = oracle.dense_gqa(P["Qs"].reshape(B, S, 1, d), P["K"][:, :, :1], P["V"][:, :, :1])
+    assert np.array_equal(s, ref[:, :, 0])
+
+
+def test_shared_head_kv0():
+    check_shared_head_is_dense_head_on_kv0()
+
+
+def check_k1_obar():
+    P = _small_problem(seed=80)
+    idx, p, w, _ = oracle.route(P["x"], P["Wr"], None, 1)
+    assert (w == 1.0).all()
+    O_sel, o_bar, _ = oracle.gqe_prefill(P["Q"], P["Qs"], P["K"], P["V"], idx, w)
+    assert np.array_equal(o_bar, O_sel[:, :, :, 0])
+
+
+def test_k1_weights_and_obar():
+    check_k1_obar()
+
+
+def check_obar_weighted_sum_k2():
+    """ō with k=2 is the w-weighted sum of the two selected heads, each of
+    which equals the dense output of that head."""
+    P = _small_problem(seed=90)
+    idx, p, w, _ = oracle.route(P["x"], P["Wr"], None, 2)
+    O_sel, o_bar, _ = oracle.gqe_prefill(P["Q"], P["Qs"], P["K"], P["V"], idx, w)
+    dense = oracle.dense_gqa(P["Q"], P["K"], P["V"])
+    M = P["Q"].shape[2] // P["K"].shape[2]
+    b, i, g = 1, 17, 2
+    want = sum(w[b, i, g, j] * dense[b, i, g * M + idx[b, i, g, j]] for j in range(2))
+    assert np.allclose(o_bar[b, i, g], want, rtol=1e-14, atol=1e-15)
+    # w is p restricted to the selection, renormalised
+    ps = p[b, i, g, idx[b, i, g]]
+    assert np.allclose(w[b, i, g], ps / ps.sum(), rtol=1e-15)
+
+
+def test_obar_weighted_sum_k2():
+    check_obar_weighted_sum_k2()
+
+
+def test_rows_subset_matches_full():
+    P = _small_problem(seed=100)
+    idx, p, w, _ = oracle.route(P["x"], P["Wr"], None, 2)
+    full = oracle.gqe_prefill(P["Q"], P["Qs"], P["K"], P["V"], idx, w)
+    rows = [np.array([0, 5, 39]), np.array([3, 38])]
+    sub = oracle.gqe_prefill_rows(P["Q"], P["Qs"], P["K"], P["V"], idx, w, rows)
+    for t in range(3):
+        for b in range(2):
+            assert np.allclose(sub[t][b], full[t][b][rows[b]], rtol=0, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: each must be caught by at least one pin
+# --------------------------------------------------------------------------
+
+ALL_CHECKS = [check_kv_bytes, check_worked_examples, check_worked_example_routed,
+              check_geometric_scores, check_nonsquare_positions, check_head_to_kv_map,
+              check_row0_and_hull, check_explicit_equals_repeat, check_router_sums,
+              check_routed_kM_equals_dense, check_shared_head_is_dense_head_on_kv0,
+              check_k1_obar, check_obar_weighted_sum_k2]
+
+
+def _caught(monkeypatch, name, fn):
+    monkeypatch.setattr(og, name, fn)
+    failed = []
+    for c in ALL_CHECKS:
+        try:
+            c()
+        except AssertionError:
+            failed.append(c.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name,fn", [
+    ("_visible", lambda k, q: k[None, :] < q[:, None]),             # diagonal dropped
+    ("_visible", lambda k, q: k[None, :] <= q[:, None] + 1),        # one key of the future
+    ("_scale", lambda d: 1.0),                                      # scale dropped
+    ("_scale", lambda d: 1.0 / d),                                  # wrong scale
+    ("_kv_head_of", lambda h, N, G: h % G),                         # interleaved map
+    ("_expert_head", lambda g, m, M: m * M + g),                    # transposed roles
+])
+def test_planted_mistakes_are_caught(monkeypatch, name, fn):
+    failed = _caught(monkeypatch, name, fn)
+    assert failed, f"planted mistake in {name} went unnoticed"
+
+
+def test_planted_kv_bytes_mistake(monkeypatch):
+    monkeypatch.setattr(oracle, "kv_cache_bytes", lambda L, G, S, d, b, B=1: L * G * d * S * b * B)
+    with pytest.raises(AssertionError):
+        check_kv_bytes()
