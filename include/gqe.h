@@ -1,0 +1,171 @@
+/*
+ * gqe.h - C ABI of the GQE (Grouped Query Experts) causal-prefill library.
+ *
+ * Grouped Query Experts puts a per-group router on grouped-query attention:
+ * N query heads form G groups of M = N/G "query-head experts" that share one
+ * KV head.  For every token i and group g the router scores the group's M
+ * experts, p_{i,g} = softmax(r_g(x_i)), keeps the top k, and only those query
+ * heads attend (against the group's dense, never repeated, KV head).  The
+ * layer output feeds W_O with Concat(O_i, o_bar_i, s(x_i)): the selected
+ * heads' outputs, their renormalised weighted sum, and an always-on shared
+ * head.  Sources: the review "论文综述：分组查询专家——在 GQA 自注意力上引入
+ * 混合专家" §二 (路由器; 输出怎么拼起来：三个关键部件) and the summary page
+ * "Grouped Query Experts: Mixture-of-Experts on GQA Self-Attention" (01 In
+ * brief).  GQA head mapping and the causal rule follow "AI 大模型之 GQA"
+ * (技术深化 分组查询的张量映射; 工程实操 非方形因果遮罩).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - Pointers marked "device" are CUDA device pointers owned by the caller;
+ *    the library never allocates, frees or retains them.  All work is queued
+ *    asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
+ *  - Every device pointer must be 16-byte aligned.  Tensors are dense,
+ *    row-major, in the layouts stated per argument (B batch, S tokens).
+ *  - `ws` is a caller-owned device workspace of at least
+ *    gqe_workspace_size(dims) bytes, zero-filled once before its first use
+ *    (it holds a latched device status word; the library keeps the rest
+ *    consistent itself).  Calls that share one workspace must be ordered
+ *    (same stream or explicit events).
+ *  - Arguments are validated before anything is launched; on any error the
+ *    call returns a non-zero gqe_status and launches nothing.  Unsupported
+ *    shapes are rejected, never silently remapped ("AI 大模型之 GQA",
+ *    工程实操: unsupported H/G combinations must be refused explicitly).
+ *  - Errors found on the device (a bounded wait that ran out, an expert index
+ *    out of range, non-finite router logits, V outside the fp16 range) are
+ *    latched into the workspace status word; read them with
+ *    gqe_get_device_status().  Nothing is thrown across the ABI.
+ *
+ * Supported shapes: N % G == 0, M = N/G <= 32, 1 <= k <= M,
+ * d in {64, 128}, G*M in {4, 8, 16, 32} for the router, d_model % 8 == 0,
+ * B*S*G*max(k,M) < 2^31.
+ */
+#ifndef GQE_H
+#define GQE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gqe_status {
+  GQE_OK = 0,
+  GQE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, k > M ... */
+  GQE_ERR_UNSUPPORTED = 2,  /* a valid GQE shape this build does not run   */
+  GQE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed         */
+  GQE_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out           */
+  GQE_ERR_WORKSPACE = 5,    /* workspace missing or smaller than required   */
+  GQE_ERR_BAD_INDEX = 6,    /* a top-k index outside [0, M) reached a kernel */
+  GQE_ERR_NONFINITE = 7     /* non-finite logit, or |V| above the fp16 range */
+} gqe_status;
+
+/* Problem size.  M = N / G is derived.  `out_fp32` selects the element type
+ * of every output written by the attention calls: 1 = float32, 0 = bf16. */
+typedef struct gqe_dims {
+  int32_t B, S, N, G, k, d, d_model;
+  int32_t out_fp32;
+} gqe_dims;
+
+/* Bytes of workspace the calls below need for `dims` (0 if dims invalid). */
+size_t gqe_workspace_size(const gqe_dims* dims);
+
+/*
+ * gqe_route - the per-group router.
+ * Review §二 路由器: p_{i,g} = softmax(r_g(x_i)) over the group's M experts,
+ * K_g(x_i) = TopK_m(p_{i,g,m}, k); 三个关键部件: w = p / sum_{m' in K_g} p.
+ * r_g is linear: l_{i,g,m} = x_i . W_r[g,:,m] (+ bias[g,m]).
+ *
+ *  x        device bf16 [B, S, d_model]
+ *  W_r      device bf16 [G, d_model, M]
+ *  bias     device fp32 [G, M] or NULL (an additive logit offset)
+ *  topk_idx device int32 [B, S, G, k]  out: expert indices in rank order
+ *  p        device fp32  [B, S, G, M]  out: router probabilities
+ *  w        device fp32  [B, S, G, k]  out: renormalised weights (k=1 -> 1)
+ *
+ * Selection is decided on the exact real-valued logits; exact ties go to the
+ * lower expert index.  The fast path certifies each decision with a rigorous
+ * float32 error bound; undecided (token, group) pairs are recomputed with an
+ * exact fixed-point dot product, so topk_idx is deterministic and exact.
+ */
+gqe_status gqe_route(const gqe_dims* dims, const void* x, const void* W_r, const float* bias,
+                     int32_t* topk_idx, float* p, float* w, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/*
+ * gqe_bucket - stable per-(batch, group, expert) token lists.
+ * For b, g, m in that order, the tokens i (ascending) with m in K_g(x_i).
+ *  topk_idx   device int32 [B, S, G, k]   (as written by gqe_route)
+ *  bucket_off device int32 [B*G*M + 1]    out: exclusive scan of bucket sizes;
+ *             bucket (b,g,m) occupies [off[(b*G+g)*M+m], off[...+1]) and the
+ *             (b,g) block starts at (b*G+g)*S*k.
+ *  bucket_tok device int32 [B*G*S*k]      out: token positions
+ * gqe_attention_prefill runs the same bucketing internally (into `ws`); this
+ * entry exists so callers and tests can inspect it.
+ */
+gqe_status gqe_bucket(const gqe_dims* dims, const int32_t* topk_idx, int32_t* bucket_off,
+                      int32_t* bucket_tok, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * gqe_attention_prefill - routed causal attention, shared head and combine.
+ * Review §二 三个关键部件: only the selected heads attend; each selected head
+ * h = g*M + m uses query Q[:, :, h] against KV head g with scale 1/sqrt(d) and
+ * the causal rule key position <= query position.
+ *
+ *  Q        device bf16 [B, S, N, d]
+ *  Qs       device bf16 [B, S, d]      query of the always-on shared head
+ *  K, V     device bf16 [B, S, G, d]   one KV head per group, not repeated
+ *  topk_idx device int32 [B, S, G, k]; w device fp32 [B, S, G, k] (gqe_route)
+ *  O_sel    out: row (b,i) + (g*k + j)*d -> output of the head in slot j
+ *  o_bar    out: row (b,i) + g*d         -> sum_j w_j * O_sel[g, j]
+ *  s_out    out: row (b,i)               -> shared-head output (attends KV 0)
+ *  out_row_stride  elements between consecutive tokens (b,i) in all three
+ *           outputs (multiple of 8).  With one concat buffer of row length
+ *           (G*k + G + 1)*d, pass O_sel = buf, o_bar = buf + G*k*d,
+ *           s_out = buf + (G*k + G)*d and stride (G*k + G + 1)*d.
+ * Output element type: float32 if dims->out_fp32 else bf16.
+ * The shared head's KV source is not given by the sources; this library
+ * fixes it to KV head 0.
+ */
+gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void* Qs,
+                                 const void* K, const void* V, const int32_t* topk_idx,
+                                 const float* w, void* O_sel, void* o_bar, void* s_out,
+                                 int64_t out_row_stride, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/*
+ * gqe_dense_gqa_prefill - the all-active GQA baseline ("16 heads all
+ * active", review §四): every query head h attends KV head floor(h/M).
+ *  Q device bf16 [B, S, N, d]; K, V device bf16 [B, S, G, d]
+ *  O device [B, S, N, d], float32 if dims->out_fp32 else bf16.
+ * dims->k is ignored.
+ */
+gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void* K,
+                                 const void* V, void* O, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* Synchronises `stream`, then returns the status word latched in `ws`
+ * (GQE_OK if no device-side error was recorded).  If `clear` is non-zero the
+ * word is reset to GQE_OK afterwards. */
+gqe_status gqe_get_device_status(void* ws, int32_t clear, void* stream);
+
+/* "AI 大模型之 GQA" §4.1: KV-cache bytes = 2 * L * G * d * S * b, times B
+ * sequences (L layers, G KV heads, b bytes per element).  Host-only. */
+uint64_t gqe_kv_cache_bytes(int32_t L, int32_t G, int64_t S, int32_t d,
+                            int32_t bytes_per_elem, int32_t B);
+
+/* Static, human-readable name of a status code. */
+const char* gqe_status_string(gqe_status s);
+
+/* Failure-detection self test: launches one kernel whose mbarrier wait can
+ * never complete, bounded by `limit_us` microseconds; the kernel gives up,
+ * latches GQE_ERR_TIMEOUT into `ws` and exits cleanly.  Returns the launch
+ * status (the latched code is read with gqe_get_device_status). */
+gqe_status gqe_selftest_bounded_wait(void* ws, size_t ws_bytes, int32_t limit_us,
+                                     void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQE_H */

@@ -1,0 +1,130 @@
+"""ctypes binding of libgqe.so (argument marshalling only).
+
+Every function here has the name and argument order of the C entry point in
+``include/gqe.h``; tensors are passed as raw device pointers.  Nothing is
+computed in Python: if the library cannot be loaded, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgqe.so")
+
+EXPORTS = (
+    "gqe_workspace_size", "gqe_route", "gqe_bucket", "gqe_attention_prefill",
+    "gqe_dense_gqa_prefill", "gqe_get_device_status", "gqe_kv_cache_bytes",
+    "gqe_status_string", "gqe_selftest_bounded_wait",
+)
+
+STATUS = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED", 3: "GQE_ERR_CUDA",
+          4: "GQE_ERR_TIMEOUT", 5: "GQE_ERR_WORKSPACE", 6: "GQE_ERR_BAD_INDEX",
+          7: "GQE_ERR_NONFINITE"}
+
+
+class GqeDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("S", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("G", ctypes.c_int32), ("k", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("d_model", ctypes.c_int32), ("out_fp32", ctypes.c_int32)]
+
+
+class GqeError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libgqe.so not built ({LIB_PATH}); run moe_routed_grouped_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, S, I32, I64, SZ = ctypes.c_void_p, ctypes.POINTER(GqeDims), ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "gqe_workspace_size": (SZ, [S]),
+        "gqe_route": (I32, [S, P, P, P, P, P, P, P, SZ, P]),
+        "gqe_bucket": (I32, [S, P, P, P, P, SZ, P]),
+        "gqe_attention_prefill": (I32, [S, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
+        "gqe_dense_gqa_prefill": (I32, [S, P, P, P, P, P, SZ, P]),
+        "gqe_get_device_status": (I32, [P, I32, P]),
+        "gqe_kv_cache_bytes": (ctypes.c_uint64, [I32, I32, I64, I32, I32, I32]),
+        "gqe_status_string": (ctypes.c_char_p, [I32]),
+        "gqe_selftest_bounded_wait": (I32, [P, SZ, I32, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    return ctypes.c_void_p(stream if isinstance(stream, int) else
+                           (0 if stream is None else stream.cuda_stream))
+
+
+def _check(code: int, where: str) -> int:
+    if code != 0:
+        raise GqeError(code, where)
+    return code
+
+
+def dims(B, S, N, G, k, d, d_model=8, out_fp32=1) -> GqeDims:
+    return GqeDims(B, S, N, G, k, d, d_model, out_fp32)
+
+
+def gqe_workspace_size(dm: GqeDims) -> int:
+    return LIB.gqe_workspace_size(ctypes.byref(dm))
+
+
+def gqe_route(dm, x, W_r, bias, topk_idx, p, w, ws, stream=None, check=True):
+    r = LIB.gqe_route(ctypes.byref(dm), _ptr(x), _ptr(W_r), _ptr(bias), _ptr(topk_idx), _ptr(p),
+                      _ptr(w), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_route") if check else r
+
+
+def gqe_bucket(dm, topk_idx, bucket_off, bucket_tok, ws, stream=None, check=True):
+    r = LIB.gqe_bucket(ctypes.byref(dm), _ptr(topk_idx), _ptr(bucket_off), _ptr(bucket_tok),
+                       _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_bucket") if check else r
+
+
+def gqe_attention_prefill(dm, Q, Qs, K, V, topk_idx, w, O_sel, o_bar, s_out, out_row_stride,
+                          ws, stream=None, check=True):
+    r = LIB.gqe_attention_prefill(ctypes.byref(dm), _ptr(Q), _ptr(Qs), _ptr(K), _ptr(V),
+                                  _ptr(topk_idx), _ptr(w), _ptr(O_sel), _ptr(o_bar), _ptr(s_out),
+                                  int(out_row_stride), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream))
+    return _check(r, "gqe_attention_prefill") if check else r
+
+
+def gqe_dense_gqa_prefill(dm, Q, K, V, O, ws, stream=None, check=True):
+    r = LIB.gqe_dense_gqa_prefill(ctypes.byref(dm), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_dense_gqa_prefill") if check else r
+
+
+def gqe_get_device_status(ws, clear=1, stream=None) -> int:
+    return LIB.gqe_get_device_status(_ptr(ws), int(clear), _stream(stream))
+
+
+def gqe_kv_cache_bytes(L, G, S, d, bytes_per_elem, B=1) -> int:
+    return LIB.gqe_kv_cache_bytes(L, G, S, d, bytes_per_elem, B)
+
+
+def gqe_status_string(code: int) -> str:
+    return LIB.gqe_status_string(code).decode()
+
+
+def gqe_selftest_bounded_wait(ws, limit_us, stream=None, check=True):
+    r = LIB.gqe_selftest_bounded_wait(_ptr(ws), ws.numel() * ws.element_size(), int(limit_us),
+                                      _stream(stream))
+    return _check(r, "gqe_selftest_bounded_wait") if check else r

@@ -1,0 +1,324 @@
+// C-ABI entry points of the GQE prefill library (declared in include/gqe.h).
+// Argument validation happens here, before any launch; the kernels live in
+// gqe_route.cu, gqe_bucket.cu and gqe_attn.cu.
+#include <cmath>
+#include <cstring>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "gqe_internal.h"
+
+using namespace gqe;
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Tiled map over a row-major tensor; dims innermost first, strides in bytes
+// for dims 1..rank-1; box of 64 elements (128 B, the swizzle span) x rows.
+bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
+                const uint64_t* dims, const uint64_t* strides, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
+  return fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gd, gs, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [B, S, H, d] (H heads) -> 4-D map with a {64, 1, 128, 1} box
+bool map_bshd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, int S, int H,
+              int d) {
+  const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(H),
+                            static_cast<uint64_t>(S), static_cast<uint64_t>(B)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(H) * d * 2,
+                               static_cast<uint64_t>(S) * H * d * 2};
+  const uint32_t box[4] = {64, 1, static_cast<uint32_t>(kTileM), 1};
+  return encode_map(m, dt, 4, base, dims, strides, box);
+}
+
+// [B, S, d] -> 3-D map with a {64, 128, 1} box
+bool map_bsd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, int S, int d) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(S),
+                            static_cast<uint64_t>(B)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(S) * d * 2};
+  const uint32_t box[3] = {64, static_cast<uint32_t>(kTileM), 1};
+  return encode_map(m, dt, 3, base, dims, strides, box);
+}
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by all entry points.  Unsupported combinations are
+// refused explicitly (never silently remapped).
+gqe_status check_dims(const gqe_dims* d, bool router) {
+  if (!d) return GQE_ERR_INVALID_ARG;
+  if (d->B < 1 || d->S < 1 || d->N < 1 || d->G < 1 || d->k < 1 || d->d < 1)
+    return GQE_ERR_INVALID_ARG;
+  if (d->N % d->G != 0) return GQE_ERR_INVALID_ARG;
+  const int64_t M = d->N / d->G;
+  if (d->k > M) return GQE_ERR_INVALID_ARG;
+  if (d->out_fp32 != 0 && d->out_fp32 != 1) return GQE_ERR_INVALID_ARG;
+  if (M > kMaxM) return GQE_ERR_UNSUPPORTED;
+  if (d->d != 64 && d->d != 128) return GQE_ERR_UNSUPPORTED;
+  const int64_t B = d->B, S = d->S, G = d->G, k = d->k;
+  const int64_t wide = k > M ? k : M;
+  if (B * S * G * wide >= (int64_t(1) << 31)) return GQE_ERR_UNSUPPORTED;
+  if (B * S * d->N >= (int64_t(1) << 31)) return GQE_ERR_UNSUPPORTED;
+  if (B * G * M >= (int64_t(1) << 24) || B >= (int64_t(1) << 24)) return GQE_ERR_UNSUPPORTED;
+  const int64_t nq = (S + kTileM - 1) / kTileM;
+  if ((nq + 2) * 4 > 200 * 1024) return GQE_ERR_UNSUPPORTED;  // scheduler histogram
+  if (router) {
+    if (d->d_model < 8 || d->d_model % 8 != 0) return GQE_ERR_UNSUPPORTED;
+    const int64_t gm = G * M;
+    if (gm != 4 && gm != 8 && gm != 16 && gm != 32) return GQE_ERR_UNSUPPORTED;
+  }
+  return GQE_OK;
+}
+
+gqe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t gqe_workspace_size(const gqe_dims* dims) {
+  if (check_dims(dims, false) != GQE_OK) return 0;
+  return make_ws_layout(*dims).total;
+}
+
+gqe_status gqe_route(const gqe_dims* dims, const void* x, const void* W_r, const float* bias,
+                     int32_t* topk_idx, float* p, float* w, void* ws, size_t ws_bytes,
+                     void* stream) {
+  gqe_status st = check_dims(dims, true);
+  if (st != GQE_OK) return st;
+  if (!aligned16(x) || !aligned16(W_r) || !aligned16(topk_idx) || !aligned16(p) ||
+      !aligned16(w) || (bias && !aligned16(bias)))
+    return GQE_ERR_INVALID_ARG;
+  const WsLayout L = make_ws_layout(*dims);
+  if (!aligned16(ws) || ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  if (cudaMemsetAsync(wb + L.counters, 0, 256, s) != cudaSuccess) return GQE_ERR_CUDA;
+  RouteArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.Wr = static_cast<const uint16_t*>(W_r);
+  a.bias = bias;
+  a.topk_idx = topk_idx;
+  a.p = p;
+  a.w = w;
+  a.fix_list = reinterpret_cast<int32_t*>(wb + L.fix_list);
+  a.fix_count = reinterpret_cast<int32_t*>(wb + L.counters);
+  a.status = reinterpret_cast<int*>(wb + L.status);
+  a.T = dims->B * dims->S;
+  a.dm = dims->d_model;
+  a.G = dims->G;
+  a.M = dims->N / dims->G;
+  a.k = dims->k;
+  return from_cuda(launch_route(a, s));
+}
+
+static BucketArgs bucket_args(const gqe_dims* dims, const int32_t* topk_idx, int32_t* off,
+                              int32_t* tok, uint8_t* wb, const WsLayout& L) {
+  BucketArgs a{};
+  a.topk_idx = topk_idx;
+  a.bucket_off = off;
+  a.bucket_tok = tok;
+  a.tiles_raw = reinterpret_cast<TileDesc*>(wb + L.tiles_raw);
+  a.tiles = reinterpret_cast<TileDesc*>(wb + L.tiles);
+  a.tile_count = reinterpret_cast<int32_t*>(wb + L.counters) + 1;
+  a.status = reinterpret_cast<int*>(wb + L.status);
+  a.B = dims->B;
+  a.S = dims->S;
+  a.G = dims->G;
+  a.M = dims->N / dims->G;
+  a.k = dims->k;
+  a.cap_bg = L.cap_bg;
+  a.n_raw_tiles = L.n_raw_tiles;
+  return a;
+}
+
+gqe_status gqe_bucket(const gqe_dims* dims, const int32_t* topk_idx, int32_t* bucket_off,
+                      int32_t* bucket_tok, void* ws, size_t ws_bytes, void* stream) {
+  gqe_status st = check_dims(dims, false);
+  if (st != GQE_OK) return st;
+  if (!aligned16(topk_idx) || !aligned16(bucket_off) || !aligned16(bucket_tok))
+    return GQE_ERR_INVALID_ARG;
+  const WsLayout L = make_ws_layout(*dims);
+  if (!aligned16(ws) || ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  const BucketArgs a = bucket_args(dims, topk_idx, bucket_off, bucket_tok, wb, L);
+  return from_cuda(launch_bucket(a, false, static_cast<cudaStream_t>(stream)));
+}
+
+static AttnArgs attn_common(const gqe_dims* dims, uint8_t* wb, const WsLayout& L) {
+  AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.status = reinterpret_cast<int*>(wb + L.status);
+  a.B = dims->B;
+  a.S = dims->S;
+  a.N = dims->N;
+  a.G = dims->G;
+  a.M = dims->N / dims->G;
+  a.k = dims->k;
+  a.d = dims->d;
+  a.out_fp32 = dims->out_fp32;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dims->d)));
+  a.wait_limit_ns = kWaitLimitNs;
+  return a;
+}
+
+gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void* Qs,
+                                 const void* K, const void* V, const int32_t* topk_idx,
+                                 const float* w, void* O_sel, void* o_bar, void* s_out,
+                                 int64_t out_row_stride, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  gqe_status st = check_dims(dims, false);
+  if (st != GQE_OK) return st;
+  if (!aligned16(Q) || !aligned16(Qs) || !aligned16(K) || !aligned16(V) ||
+      !aligned16(topk_idx) || !aligned16(w) || !aligned16(O_sel) || !aligned16(o_bar) ||
+      !aligned16(s_out))
+    return GQE_ERR_INVALID_ARG;
+  if (out_row_stride < dims->d || out_row_stride % 8 != 0) return GQE_ERR_INVALID_ARG;
+  const WsLayout L = make_ws_layout(*dims);
+  if (!aligned16(ws) || ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  const int64_t B = dims->B, S = dims->S, G = dims->G, d = dims->d;
+
+  ConvertArgs cv{static_cast<const uint16_t*>(V), reinterpret_cast<uint16_t*>(wb + L.v16),
+                 B * S * G * d, reinterpret_cast<int*>(wb + L.status)};
+  cudaError_t e = launch_convert_v(cv, s);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+
+  const BucketArgs ba = bucket_args(dims, topk_idx, reinterpret_cast<int32_t*>(wb + L.bucket_off),
+                                    reinterpret_cast<int32_t*>(wb + L.bucket_tok), wb, L);
+  e = launch_bucket(ba, true, s);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+
+  AttnArgs a = attn_common(dims, wb, L);
+  if (!map_bshd(&a.tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, dims->B, dims->S, dims->G, dims->d) ||
+      !map_bshd(&a.tmV, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wb + L.v16, dims->B, dims->S, dims->G,
+                dims->d) ||
+      !map_bshd(&a.tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, dims->B, dims->S, dims->N, dims->d) ||
+      !map_bsd(&a.tmQs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Qs, dims->B, dims->S, dims->d))
+    return GQE_ERR_CUDA;
+  a.Q = static_cast<const uint16_t*>(Q);
+  a.bucket_off = reinterpret_cast<const int32_t*>(wb + L.bucket_off);
+  a.bucket_tok = reinterpret_cast<const int32_t*>(wb + L.bucket_tok);
+  a.topk_idx = topk_idx;
+  a.tiles = reinterpret_cast<const TileDesc*>(wb + L.tiles);
+  a.tile_count = reinterpret_cast<const int32_t*>(wb + L.counters) + 1;
+  a.O_sel = O_sel;
+  a.o_bar = o_bar;
+  a.s_out = s_out;
+  a.out_row_stride = out_row_stride;
+  a.dense = 0;
+  e = launch_attention(a, L.n_raw_tiles, s);
+  if (e != cudaSuccess) return GQE_ERR_CUDA;
+
+  if (dims->k > 1) {
+    CombineArgs c{O_sel, o_bar, w, out_row_stride, dims->B * dims->S, dims->G, dims->k, dims->d,
+                  dims->out_fp32};
+    e = launch_combine(c, s);
+    if (e != cudaSuccess) return GQE_ERR_CUDA;
+  }
+  return GQE_OK;
+}
+
+gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void* K,
+                                 const void* V, void* O, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  gqe_status st = check_dims(dims, false);
+  if (st != GQE_OK) return st;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return GQE_ERR_INVALID_ARG;
+  const WsLayout L = make_ws_layout(*dims);
+  if (!aligned16(ws) || ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  const int64_t B = dims->B, S = dims->S, G = dims->G, d = dims->d;
+  ConvertArgs cv{static_cast<const uint16_t*>(V), reinterpret_cast<uint16_t*>(wb + L.v16),
+                 B * S * G * d, reinterpret_cast<int*>(wb + L.status)};
+  if (launch_convert_v(cv, s) != cudaSuccess) return GQE_ERR_CUDA;
+  AttnArgs a = attn_common(dims, wb, L);
+  if (!map_bshd(&a.tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, dims->B, dims->S, dims->G, dims->d) ||
+      !map_bshd(&a.tmV, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wb + L.v16, dims->B, dims->S, dims->G,
+                dims->d) ||
+      !map_bshd(&a.tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, dims->B, dims->S, dims->N, dims->d))
+    return GQE_ERR_CUDA;
+  a.tmQs = a.tmQ;  // unused by dense tiles
+  a.Q = static_cast<const uint16_t*>(Q);
+  a.O_dense = O;
+  a.dense = 1;
+  const int64_t nq = (S + kTileM - 1) / kTileM;
+  return from_cuda(launch_attention(a, B * dims->N * nq, s));
+}
+
+gqe_status gqe_get_device_status(void* ws, int32_t clear, void* stream) {
+  if (!aligned16(ws)) return GQE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GQE_ERR_CUDA;
+  int32_t code = 0;
+  if (cudaMemcpy(&code, ws, sizeof(code), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GQE_ERR_CUDA;
+  if (clear && cudaMemset(ws, 0, sizeof(int32_t)) != cudaSuccess) return GQE_ERR_CUDA;
+  if (code < GQE_OK || code > GQE_ERR_NONFINITE) return GQE_ERR_CUDA;
+  return static_cast<gqe_status>(code);
+}
+
+uint64_t gqe_kv_cache_bytes(int32_t L, int32_t G, int64_t S, int32_t d, int32_t bytes_per_elem,
+                            int32_t B) {
+  if (L < 0 || G < 0 || S < 0 || d < 0 || bytes_per_elem < 0 || B < 0) return 0;
+  return 2ull * static_cast<uint64_t>(L) * static_cast<uint64_t>(G) * static_cast<uint64_t>(d) *
+         static_cast<uint64_t>(S) * static_cast<uint64_t>(bytes_per_elem) *
+         static_cast<uint64_t>(B);
+}
+
+const char* gqe_status_string(gqe_status s) {
+  switch (s) {
+    case GQE_OK: return "ok";
+    case GQE_ERR_INVALID_ARG: return "invalid argument";
+    case GQE_ERR_UNSUPPORTED: return "unsupported shape";
+    case GQE_ERR_CUDA: return "CUDA error";
+    case GQE_ERR_TIMEOUT: return "device wait timed out";
+    case GQE_ERR_WORKSPACE: return "workspace missing or too small";
+    case GQE_ERR_BAD_INDEX: return "expert index out of range";
+    case GQE_ERR_NONFINITE: return "non-finite value or value outside the fp16 range";
+  }
+  return "unknown status";
+}
+
+gqe_status gqe_selftest_bounded_wait(void* ws, size_t ws_bytes, int32_t limit_us, void* stream) {
+  if (!aligned16(ws) || ws_bytes < 256) return GQE_ERR_WORKSPACE;
+  if (limit_us < 1 || limit_us > 10000000) return GQE_ERR_INVALID_ARG;
+  return from_cuda(launch_selftest_wait(static_cast<int*>(ws),
+                                        static_cast<uint64_t>(limit_us) * 1000ull,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

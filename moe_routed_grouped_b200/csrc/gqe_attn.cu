@@ -1,0 +1,462 @@
+// Causal flash attention on the sm_100a tensor cores for GQE prefill.
+//
+// One CTA computes one work item: 128 query rows against every KV tile they
+// can see.  Three kinds of rows share the kernel:
+//   routed  - the rows of one (batch, group, expert) bucket: the tokens whose
+//             router picked query head h = g*M + m ("论文综述：分组查询专家"
+//             §二 路由器), gathered by token index; they attend KV head g;
+//   shared  - 128 consecutive tokens of the always-on shared head (§二 三个
+//             关键部件), KV head 0;
+//   dense   - 128 consecutive tokens of one query head h, KV head
+//             floor(h / M) ("AI 大模型之 GQA", 技术深化: the explicit head map).
+// K and V are read straight from the group's KV head; nothing is repeated.
+// The causal rule is applied on absolute token positions (key <= query,
+// "AI 大模型之 GQA" 工程实操), so gathered rows mask correctly and KV tiles past
+// the last row's position are never visited.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax + epilogue; thread r owns query row r (TMEM lane r)
+//   warp 4     producer: Q gather (cp.async) or TMA tile load; K/V via TMA
+//   warp 5     TMEM owner and single-thread tcgen05.mma issuer
+// TMEM: S = Q.K^T (128 fp32 columns), P (fp16, 64 columns), O (d columns).
+// Per KV tile j: S_j = Q K_j^T (UMMA, smem x smem) -> softmax warps read S_j,
+// release it, exponentiate, write P_j to TMEM -> O += P_j V_j (UMMA, A from
+// TMEM).  Q.K^T of tile j+1 runs while the softmax of tile j is computed.
+// The running max is only moved when it grows by more than 2^8, so O is
+// rescaled rarely; the final division by the row sum makes this exact.
+#include "gqe_device.cuh"
+
+namespace gqe {
+namespace {
+
+template <int D>
+struct Cfg {
+  static constexpr int kStages = 2;
+  static constexpr int kAtom = kTileM * 128;          // 128 rows x 128 B (64 elements)
+  static constexpr int kQBytes = kTileM * D * 2;
+  static constexpr int kKVBytes = kTileN * D * 2;
+  static constexpr int kSmemQ = 0;
+  static constexpr int kSmemK = kQBytes;
+  static constexpr int kSmemV = kSmemK + kStages * kKVBytes;
+  static constexpr int kSmemBar = kSmemV + kStages * kKVBytes;
+  static constexpr int kSmemBytes = kSmemBar + 256 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t kTmemS = 0, kTmemP = 128, kTmemO = (D == 64 ? 192 : 256);
+  static constexpr uint32_t kTmemCols = (D == 64 ? 256 : 512);
+  static constexpr int kMinBlocks = (D == 64 ? 2 : 1);
+  static constexpr uint32_t kIdescQK = make_idesc_f16(kTileM, kTileN, /*bf16*/ 1, 0, 0);
+  static constexpr uint32_t kIdescPV = make_idesc_f16(kTileM, D, /*f16*/ 0, 0, /*MN*/ 1);
+};
+
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+
+// barrier slots
+enum {
+  kBarQFull = 0,
+  kBarKFull = 1,   // +stage
+  kBarKEmpty = 3,  // +stage
+  kBarVFull = 5,   // +stage
+  kBarVEmpty = 7,  // +stage
+  kBarSFull = 9,
+  kBarSFree = 10,
+  kBarPFull = 11,
+  kBarODone = 12,
+  kBarSpare = 13,
+  kNumBars = 14
+};
+
+struct Waiter {
+  volatile int* abort;
+  int* status;
+  uint64_t limit;
+  __device__ bool operator()(uint64_t* bar, uint32_t parity) const {
+    return mbar_wait(bar, parity, abort, status, limit);
+  }
+};
+
+__device__ __forceinline__ void store_row32(void* dst, const uint32_t (&v)[32], float scale,
+                                            bool fp32) {
+  if (fp32) {
+    float4* o = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      o[q] = make_float4(__uint_as_float(v[4 * q]) * scale, __uint_as_float(v[4 * q + 1]) * scale,
+                         __uint_as_float(v[4 * q + 2]) * scale,
+                         __uint_as_float(v[4 * q + 3]) * scale);
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]) * scale,
+                                                 __uint_as_float(v[8 * q + 2 * e + 1]) * scale);
+        w[e] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      o[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
+    attn_kernel(const __grid_constant__ AttnArgs a) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.S, N = a.N, G = a.G, M = a.M;
+
+  // ---------------------------------------------------------- work item
+  int kind, b, h = 0, g = 0, m = 0, row0, nrows, nkv, bstart = 0;
+  if (a.dense) {
+    const int nq = (S + kTileM - 1) / kTileM;
+    const int64_t bn = static_cast<int64_t>(a.B) * N;
+    const int64_t t = blockIdx.x;
+    const int qt = nq - 1 - static_cast<int>(t / bn);
+    const int bh = static_cast<int>(t % bn);
+    kind = kDense;
+    b = bh / N;
+    h = bh % N;
+    g = h / M;
+    row0 = qt * kTileM;
+    nrows = min(kTileM, S - row0);
+    nkv = qt + 1;
+  } else {
+    if (static_cast<int>(blockIdx.x) >= *a.tile_count) return;
+    const TileDesc td = a.tiles[blockIdx.x];
+    kind = td.code >> 24;
+    const int id = td.code & 0xFFFFFF;
+    if (kind == kRouted) {
+      b = id / (G * M);
+      g = (id / M) % G;
+      m = id % M;
+      h = g * M + m;
+      bstart = a.bucket_off[id];
+    } else {
+      b = id;
+      g = 0;  // the shared head reads KV head 0
+    }
+    row0 = td.row0;
+    nrows = td.nrows;
+    nkv = td.nkv;
+  }
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kNumBars + 1);
+  const Waiter wait{abort_flag, a.status, a.wait_limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kBarQFull], 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&bars[kBarKFull + s], 1);
+      mbar_init(&bars[kBarKEmpty + s], 1);
+      mbar_init(&bars[kBarVFull + s], 1);
+      mbar_init(&bars[kBarVEmpty + s], 1);
+    }
+    mbar_init(&bars[kBarSFull], 1);
+    mbar_init(&bars[kBarSFree], 4);
+    mbar_init(&bars[kBarPFull], 4);
+    mbar_init(&bars[kBarODone], 1);
+    mbar_init(&bars[kBarSpare], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&a.tmK);
+    tma_prefetch_desc(&a.tmV);
+    tma_prefetch_desc(kind == kDense ? &a.tmQ : &a.tmQs);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------ producer
+    uint8_t* sQ = smem + C::kSmemQ;
+    if (kind == kRouted) {
+      // gather the bucket's query rows, writing the 128-byte swizzle that
+      // the UMMA descriptor expects (16-byte chunk c of row r at c ^ (r & 7))
+      for (int rr = 0; rr < kTileM / 32; ++rr) {
+        const int r = lane + 32 * rr;
+        const bool ok = r < nrows;
+        const int tok = ok ? a.bucket_tok[bstart + row0 + r] : 0;
+        const uint16_t* src = a.Q + ((static_cast<int64_t>(b) * S + tok) * N + h) * D;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const int atom = c >> 3, ch = c & 7;
+          uint8_t* dst = sQ + atom * C::kAtom + r * 128 + ((ch ^ (r & 7)) << 4);
+          cp_async_16(dst, src + c * 8, ok ? 16u : 0u);
+        }
+      }
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarQFull]);
+    } else if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[kBarQFull], C::kQBytes);
+#pragma unroll
+      for (int atom = 0; atom < D / 64; ++atom) {
+        if (kind == kDense)
+          tma_load_4d(sQ + atom * C::kAtom, &a.tmQ, &bars[kBarQFull], atom * 64, h, row0, b);
+        else
+          tma_load_3d(sQ + atom * C::kAtom, &a.tmQs, &bars[kBarQFull], atom * 64, row0, b);
+      }
+    }
+    if (lane == 0) {
+      int issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j & 1;
+        const uint32_t round = static_cast<uint32_t>(j >> 1);
+        if (round > 0 && !wait(&bars[kBarKEmpty + s], (round - 1) & 1)) break;
+        mbar_arrive_expect_tx(&bars[kBarKFull + s], C::kKVBytes);
+#pragma unroll
+        for (int atom = 0; atom < D / 64; ++atom)
+          tma_load_4d(smem + C::kSmemK + s * C::kKVBytes + atom * C::kAtom, &a.tmK,
+                      &bars[kBarKFull + s], atom * 64, g, j * kTileN, b);
+        if (round > 0 && !wait(&bars[kBarVEmpty + s], (round - 1) & 1)) {
+          issued = 2 * j + 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&bars[kBarVFull + s], C::kKVBytes);
+#pragma unroll
+        for (int atom = 0; atom < D / 64; ++atom)
+          tma_load_4d(smem + C::kSmemV + s * C::kKVBytes + atom * C::kAtom, &a.tmV,
+                      &bars[kBarVFull + s], atom * 64, g, j * kTileN, b);
+        issued = 2 * j + 2;
+      }
+      if (*abort_flag) {
+        // let the copies already in flight land before the CTA exits
+        const int nk = (issued + 1) / 2, nv = issued / 2;
+        for (int q = max(0, nk - 2); q < nk; ++q)
+          mbar_wait(&bars[kBarKFull + (q & 1)], (q >> 1) & 1, nullptr, a.status, a.wait_limit_ns);
+        for (int q = max(0, nv - 2); q < nv; ++q)
+          mbar_wait(&bars[kBarVFull + (q & 1)], (q >> 1) & 1, nullptr, a.status, a.wait_limit_ns);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t tS = tbase + C::kTmemS, tP = tbase + C::kTmemP, tO = tbase + C::kTmemO;
+      const uint32_t qaddr = smem_u32(smem + C::kSmemQ);
+      auto issue_pv = [&](int jj) -> bool {
+        const int s = jj & 1;
+        if (!wait(&bars[kBarPFull], jj & 1)) return false;
+        if (!wait(&bars[kBarVFull + s], (jj >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t vaddr = smem_u32(smem + C::kSmemV + s * C::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk)
+          umma_ts(tO, tP + kk * 8, make_sdesc_sw128(vaddr + kk * 2048, C::kAtom, 1024),
+                  C::kIdescPV, (jj > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&bars[kBarODone]);
+        tc_commit(&bars[kBarVEmpty + s]);
+        return true;
+      };
+      bool ok = wait(&bars[kBarQFull], 0);
+      tc_fence_after();
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j & 1;
+        if (!wait(&bars[kBarKFull + s], (j >> 1) & 1)) { ok = false; break; }
+        if (j > 0 && !wait(&bars[kBarSFree], (j - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(smem + C::kSmemK + s * C::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kAtom + (kk & 3) * 32;
+          umma_ss(tS, make_sdesc_sw128(qaddr + off, 16, 1024),
+                  make_sdesc_sw128(kaddr + off, 16, 1024), C::kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars[kBarSFull]);
+        tc_commit(&bars[kBarKEmpty + s]);
+        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) ok = issue_pv(nkv - 1);
+      if (!ok) {
+        // drain whatever was issued before giving up
+        tc_commit(&bars[kBarSpare]);
+        mbar_wait(&bars[kBarSpare], 0, nullptr, a.status, a.wait_limit_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ softmax warps
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int rv = min(r, nrows - 1);
+    int pos, pos_first;
+    if (kind == kRouted) {
+      pos = a.bucket_tok[bstart + row0 + rv];
+      pos_first = a.bucket_tok[bstart + row0];
+    } else {
+      pos = row0 + rv;
+      pos_first = row0;
+    }
+    const float sl2 = a.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      if (!wait(&bars[kBarSFull], j & 1)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tbase + lane_off + C::kTmemS + 32 * c, sv[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarSFree]);
+
+      const int kbase = j * kTileN;
+      if (kbase + kTileN - 1 > pos_first) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (kbase + 32 * c + e > pos) sv[c][e] = __float_as_uint(-INFINITY);
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[c][e]));
+      const float mnew = fmaxf(m_used, mx * sl2);
+      float factor = 1.f;
+      if (mnew - m_used > 8.f) {
+        factor = ex2_approx(m_used - mnew);
+        m_used = mnew;
+      }
+      l *= factor;
+      uint32_t pk[2][32];
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c][e]), sl2, -m_used));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c][e + 1]), sl2, -m_used));
+          rs += p0 + p1;
+          pk[c >> 1][(c & 1) * 16 + e / 2] = pack_half2(p0, p1);
+        }
+      l += rs;
+      if (j > 0) {
+        if (!wait(&bars[kBarODone], (j - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xFFFFFFFFu, factor != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tbase + lane_off + C::kTmemO + 32 * c, ov);
+            tmem_ld_wait(ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+            tmem_st32(tbase + lane_off + C::kTmemO + 32 * c, ov);
+          }
+        }
+      }
+      tmem_st32(tbase + lane_off + C::kTmemP, pk[0]);
+      tmem_st32(tbase + lane_off + C::kTmemP + 32, pk[1]);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarPFull]);
+    }
+    if (ok) ok = wait(&bars[kBarODone], (nkv - 1) & 1);
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const bool fp32 = a.out_fp32 != 0;
+      const size_t esz = fp32 ? 4 : 2;
+      uint8_t* dst = nullptr;
+      uint8_t* dst2 = nullptr;
+      if (r < nrows) {
+        const int64_t tokrow = static_cast<int64_t>(b) * S + pos;
+        if (kind == kDense) {
+          dst = static_cast<uint8_t*>(a.O_dense) + ((tokrow * N + h) * D) * esz;
+        } else if (kind == kShared) {
+          dst = static_cast<uint8_t*>(a.s_out) + (tokrow * a.out_row_stride) * esz;
+        } else {
+          const int32_t* sel = a.topk_idx + (tokrow * G + g) * a.k;
+          int slot = 0;
+          for (int q = 0; q < a.k; ++q)
+            if (sel[q] == m) slot = q;
+          dst = static_cast<uint8_t*>(a.O_sel) +
+                (tokrow * a.out_row_stride + static_cast<int64_t>(g * a.k + slot) * D) * esz;
+          if (a.k == 1)
+            dst2 = static_cast<uint8_t*>(a.o_bar) +
+                   (tokrow * a.out_row_stride + static_cast<int64_t>(g) * D) * esz;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tbase + lane_off + C::kTmemO + 32 * c, ov);
+        tmem_ld_wait(ov);
+        if (dst) store_row32(dst + 32 * c * esz, ov, inv, fp32);
+        if (dst2) store_row32(dst2 + 32 * c * esz, ov, inv, fp32);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::kTmemCols);
+  }
+}
+
+__global__ void selftest_wait_kernel(int* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the wait must give up by itself
+  mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+}
+
+template <int D>
+cudaError_t launch_d(const AttnArgs& a, int64_t grid, cudaStream_t st) {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (configured_device != dev) {
+    e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg<D>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  attn_kernel<D><<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmemBytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnArgs& a, int64_t grid, cudaStream_t st) {
+  if (grid <= 0) return cudaSuccess;
+  if (a.d == 64) return launch_d<64>(a, grid, st);
+  if (a.d == 128) return launch_d<128>(a, grid, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_selftest_wait(int* status, uint64_t limit_ns, cudaStream_t st) {
+  selftest_wait_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace gqe

@@ -1,0 +1,268 @@
+// Bucketing, work-list scheduling, V conversion and the k>1 combine.
+//
+// bucket_kernel: one CTA per (batch, group).  Each token appears once in each
+// of the k buckets its router picked ("论文综述：分组查询专家" §二 路由器:
+// only the selected heads compute), so the (b, g) block of the token list has
+// the fixed size S*k and starts at (b*G + g)*S*k; the per-expert offsets are
+// a scan local to the CTA.  The scatter is a stable counting sort built from
+// warp ballots, so each bucket lists its tokens in ascending position, which
+// the attention kernel needs for causal tile skipping ("AI 大模型之 GQA",
+// 工程实操: the mask is decided on absolute positions).
+#include "gqe_device.cuh"
+
+namespace gqe {
+namespace {
+
+constexpr int kBucketThreads = 1024;
+constexpr int kBucketWarps = kBucketThreads / 32;
+
+__global__ void __launch_bounds__(kBucketThreads) bucket_kernel(const BucketArgs a) {
+  __shared__ int cnt[kMaxM];
+  __shared__ int start[kMaxM];
+  __shared__ int running[kMaxM];
+  __shared__ int wcnt[kMaxM][kBucketWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bg = blockIdx.x, b = bg / a.G, g = bg % a.G;
+  const int S = a.S, G = a.G, M = a.M, k = a.k;
+  const int64_t base = static_cast<int64_t>(bg) * S * k;
+  if (tid < kMaxM) {
+    cnt[tid] = 0;
+    running[tid] = 0;
+  }
+  __syncthreads();
+
+  // phase 1: bucket sizes (warp-aggregated counts)
+  bool bad = false;
+  for (int i0 = 0; i0 < S; i0 += kBucketThreads) {
+    const int i = i0 + tid;
+    uint32_t mine = 0;
+    if (i < S) {
+      const int32_t* row = a.topk_idx + ((static_cast<int64_t>(b) * S + i) * G + g) * k;
+      for (int j = 0; j < k; ++j) {
+        const int m = row[j];
+        if (m < 0 || m >= M) bad = true;
+        else mine |= 1u << m;
+      }
+    }
+    for (int m = 0; m < M; ++m) {
+      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, (mine >> m) & 1u);
+      if (lane == 0 && bal) atomicAdd(&cnt[m], __popc(bal));
+    }
+  }
+  if (bad) latch_status(a.status, GQE_ERR_BAD_INDEX);
+  __syncthreads();
+  if (tid == 0) {
+    int s = 0;
+    for (int m = 0; m < M; ++m) {
+      start[m] = s;
+      s += cnt[m];
+    }
+  }
+  __syncthreads();
+  if (tid < M) a.bucket_off[bg * M + tid] = static_cast<int32_t>(base + start[tid]);
+  if (bg == a.B * a.G - 1 && tid == 0)
+    a.bucket_off[a.B * a.G * M] = static_cast<int32_t>(static_cast<int64_t>(a.B) * G * S * k);
+
+  // phase 2: stable scatter, one chunk of 1024 tokens at a time
+  for (int i0 = 0; i0 < S; i0 += kBucketThreads) {
+    const int i = i0 + tid;
+    uint32_t mine = 0;  // bit m set if this token picked expert m
+    if (i < S) {
+      const int32_t* row = a.topk_idx + ((static_cast<int64_t>(b) * S + i) * G + g) * k;
+      for (int j = 0; j < k; ++j) {
+        const int m = row[j];
+        if (m >= 0 && m < M) mine |= 1u << m;
+      }
+    }
+    for (int m = 0; m < M; ++m) {
+      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, (mine >> m) & 1u);
+      if (lane == 0) wcnt[m][warp] = __popc(bal);
+    }
+    __syncthreads();
+    if (tid < M) {
+      int s = running[tid];
+      for (int w = 0; w < kBucketWarps; ++w) {
+        const int c = wcnt[tid][w];
+        wcnt[tid][w] = s;
+        s += c;
+      }
+      running[tid] = s;
+    }
+    __syncthreads();
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int m = 0; m < M; ++m) {
+      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, (mine >> m) & 1u);
+      if ((mine >> m) & 1u) {
+        const int r = wcnt[m][warp] + __popc(bal & lt);
+        a.bucket_tok[base + start[m] + r] = i;
+      }
+    }
+    __syncthreads();
+  }
+
+  // routed work items: ceil(cnt/128) tiles per expert; unused slots get nkv 0
+  TileDesc* slots = a.tiles_raw + static_cast<int64_t>(bg) * a.cap_bg;
+  int first = 0;
+  for (int m = 0; m < M; ++m) {
+    const int nt = (cnt[m] + kTileM - 1) / kTileM;
+    for (int t = tid; t < nt; t += kBucketThreads) {
+      const int row0 = t * kTileM;
+      const int nrows = min(kTileM, cnt[m] - row0);
+      const int last = a.bucket_tok[base + start[m] + row0 + nrows - 1];
+      TileDesc d;
+      d.code = (kRouted << 24) | (bg * M + m);
+      d.row0 = row0;
+      d.nrows = nrows;
+      d.nkv = last / kTileN + 1;
+      slots[first + t] = d;
+    }
+    first += nt;
+  }
+  for (int t = first + tid; t < a.cap_bg; t += kBucketThreads) slots[t] = TileDesc{0, 0, 0, 0};
+}
+
+// One CTA: shared-head tiles are appended, then every work item is sorted by
+// its KV-tile count, longest first (so the heaviest tiles start first and the
+// grid's tail is short).  Counting sort on nkv in [1, ceil(S/128)].
+constexpr int kSchedThreads = 1024;
+
+__global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const BucketArgs a) {
+  extern __shared__ int hist[];  // nq + 2 bins
+  const int tid = threadIdx.x;
+  const int nq = (a.S + kTileM - 1) / kTileM;
+  const int64_t n_routed = static_cast<int64_t>(a.B) * a.G * a.cap_bg;
+  TileDesc* shared_tiles = a.tiles_raw + n_routed;
+  for (int v = tid; v < nq + 2; v += kSchedThreads) hist[v] = 0;
+  // the shared head's tiles: every token, KV head 0
+  for (int64_t t = tid; t < static_cast<int64_t>(a.B) * nq; t += kSchedThreads) {
+    const int b = static_cast<int>(t / nq), q = static_cast<int>(t % nq);
+    TileDesc d;
+    d.code = (kShared << 24) | b;
+    d.row0 = q * kTileM;
+    d.nrows = min(kTileM, a.S - q * kTileM);
+    d.nkv = q + 1;
+    shared_tiles[t] = d;
+  }
+  __syncthreads();
+  for (int64_t t = tid; t < a.n_raw_tiles; t += kSchedThreads) {
+    const int v = a.tiles_raw[t].nkv;
+    if (v > 0) atomicAdd(&hist[v], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {  // exclusive scan from the largest nkv down
+    int s = 0;
+    for (int v = nq; v >= 1; --v) {
+      const int c = hist[v];
+      hist[v] = s;
+      s += c;
+    }
+    *a.tile_count = s;
+  }
+  __syncthreads();
+  for (int64_t t = tid; t < a.n_raw_tiles; t += kSchedThreads) {
+    const TileDesc d = a.tiles_raw[t];
+    if (d.nkv > 0) a.tiles[atomicAdd(&hist[d.nkv], 1)] = d;
+  }
+}
+
+// V (bf16) -> fp16 for the P.V product; P is rounded to fp16 (11-bit
+// significand), which is what keeps the output within 1e-3 relative L2.
+__global__ void convert_v_kernel(const ConvertArgs a) {
+  const int64_t n8 = a.n / 8;
+  bool bad = false;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(a.V)[i];
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = __uint_as_float(in[q] << 16);
+      const float hi = __uint_as_float(in[q] & 0xFFFF0000u);
+      bad |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+      out[q] = pack_half2(lo, hi);
+    }
+    reinterpret_cast<uint4*>(a.V16)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+  if (bad) latch_status(a.status, GQE_ERR_NONFINITE);
+}
+
+// o_bar[t, g] = sum_j w[t, g, j] * O_sel[t, g, j] in slot order
+// (review §二 三个关键部件, the renormalised weighted-sum slot); k > 1 only.
+__global__ void combine_kernel(const CombineArgs a) {
+  const int lanes_per_row = a.d / 4;  // 4 elements per thread
+  const int64_t rows = static_cast<int64_t>(a.T) * a.G;
+  const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t q = tid; q < rows * lanes_per_row; q += nthreads) {
+    const int64_t row = q / lanes_per_row;
+    const int c = static_cast<int>(q % lanes_per_row) * 4;
+    const int64_t t = row / a.G;
+    const int g = static_cast<int>(row % a.G);
+    const float* wr = a.w + row * a.k;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < a.k; ++j) {
+      const int64_t off = t * a.out_row_stride + static_cast<int64_t>(g * a.k + j) * a.d + c;
+      float v[4];
+      if (a.out_fp32) {
+        const float4 f = *reinterpret_cast<const float4*>(static_cast<const float*>(a.O_sel) + off);
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+      } else {
+        const uint2 h = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(a.O_sel) + off);
+        v[0] = __uint_as_float(h.x << 16); v[1] = __uint_as_float(h.x & 0xFFFF0000u);
+        v[2] = __uint_as_float(h.y << 16); v[3] = __uint_as_float(h.y & 0xFFFF0000u);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = fmaf(wr[j], v[e], acc[e]);
+    }
+    const int64_t off = t * a.out_row_stride + static_cast<int64_t>(g) * a.d + c;
+    if (a.out_fp32) {
+      *reinterpret_cast<float4*>(static_cast<float*>(a.o_bar) + off) =
+          make_float4(acc[0], acc[1], acc[2], acc[3]);
+    } else {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
+      uint2 h;
+      h.x = *reinterpret_cast<uint32_t*>(&lo);
+      h.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.o_bar) + off) = h;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bucket(const BucketArgs& a, bool with_schedule, cudaStream_t st) {
+  bucket_kernel<<<a.B * a.G, kBucketThreads, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !with_schedule) return e;
+  const int nq = (a.S + kTileM - 1) / kTileM;
+  const size_t smem = sizeof(int) * (nq + 2);
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  schedule_kernel<<<1, kSchedThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_convert_v(const ConvertArgs& a, cudaStream_t st) {
+  const int64_t n8 = a.n / 8;
+  int64_t blocks = (n8 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  convert_v_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
+  const int64_t work = static_cast<int64_t>(a.T) * a.G * (a.d / 4);
+  int64_t blocks = (work + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  combine_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace gqe

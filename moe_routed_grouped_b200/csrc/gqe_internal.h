@@ -1,0 +1,138 @@
+// Internal declarations shared by the GQE kernels and the C-ABI layer.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/gqe.h"
+
+namespace gqe {
+
+constexpr int kTileM = 128;      // query rows per attention tile (UMMA M)
+constexpr int kTileN = 128;      // keys per KV tile (UMMA N of Q.K^T)
+constexpr int kMaxM = 32;        // experts per group supported
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s per bounded wait
+
+// Tile kinds of the attention work list.
+enum TileKind : int { kRouted = 0, kShared = 1, kDense = 2 };
+
+// One attention work item: 128 query rows against the keys they can see.
+//   code  = (kind << 24) | id   (routed: bucket (b*G+g)*M+m; shared: b)
+//   row0  = first row inside the bucket (routed) or first token (shared)
+//   nrows = valid rows (1..128); nkv = KV tiles to visit (0 = empty slot)
+struct TileDesc {
+  int32_t code, row0, nrows, nkv;
+};
+
+// Byte offsets of the regions inside the caller's workspace.
+struct WsLayout {
+  size_t status;      // int32 status word (latched errors)
+  size_t counters;    // int32[16]: [0] router fixup count, [1] tile count
+  size_t fix_list;    // int32[B*S*G]: (token*G + g) pairs needing exact routing
+  size_t v16;         // fp16 [B,S,G,d]: V converted for the P.V product
+  size_t bucket_off;  // int32[B*G*M + 1]
+  size_t bucket_tok;  // int32[B*G*S*k]
+  size_t tiles_raw;   // TileDesc[n_raw_tiles]
+  size_t tiles;       // TileDesc[n_raw_tiles] sorted by nkv, descending
+  size_t total;
+  int64_t cap_bg;       // routed tile slots per (b, g)
+  int64_t n_raw_tiles;  // B*G*cap_bg + B*nq (routed + shared)
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WsLayout make_ws_layout(const gqe_dims& d) {
+  WsLayout L{};
+  const int64_t B = d.B, S = d.S, G = d.G, M = d.N / d.G, k = d.k, hd = d.d;
+  const int64_t nq = (S + kTileM - 1) / kTileM;
+  L.cap_bg = (S * k + kTileM - 1) / kTileM + M;
+  L.n_raw_tiles = B * G * L.cap_bg + B * nq;
+  size_t off = 0;
+  L.status = off;     off += 256;
+  L.counters = off;   off += 256;
+  L.fix_list = off;   off = align_up(off + sizeof(int32_t) * B * S * G, 256);
+  L.v16 = off;        off = align_up(off + sizeof(uint16_t) * B * S * G * hd, 256);
+  L.bucket_off = off; off = align_up(off + sizeof(int32_t) * (B * G * M + 1), 256);
+  L.bucket_tok = off; off = align_up(off + sizeof(int32_t) * B * G * S * k, 256);
+  L.tiles_raw = off;  off = align_up(off + sizeof(TileDesc) * L.n_raw_tiles, 256);
+  L.tiles = off;      off = align_up(off + sizeof(TileDesc) * L.n_raw_tiles, 256);
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------ launchers
+struct RouteArgs {
+  const uint16_t* x;    // bf16 [T, dm]
+  const uint16_t* Wr;   // bf16 [G, dm, M]
+  const float* bias;    // [G*M] or null
+  int32_t* topk_idx;    // [T, G, k]
+  float* p;             // [T, G, M]
+  float* w;             // [T, G, k]
+  int32_t* fix_list;
+  int32_t* fix_count;
+  int* status;
+  int T, dm, G, M, k;
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+
+struct BucketArgs {
+  const int32_t* topk_idx;  // [B,S,G,k]
+  int32_t* bucket_off;      // [B*G*M+1]
+  int32_t* bucket_tok;      // [B*G*S*k]
+  TileDesc* tiles_raw;      // routed slots then shared-head tiles
+  TileDesc* tiles;          // sorted output
+  int32_t* tile_count;
+  int* status;
+  int B, S, G, M, k;
+  int64_t cap_bg;
+  int64_t n_raw_tiles;
+};
+cudaError_t launch_bucket(const BucketArgs& a, bool with_schedule, cudaStream_t st);
+
+struct ConvertArgs {
+  const uint16_t* V;  // bf16
+  uint16_t* V16;      // fp16
+  int64_t n;          // elements (multiple of 8)
+  int* status;
+};
+cudaError_t launch_convert_v(const ConvertArgs& a, cudaStream_t st);
+
+struct AttnArgs {
+  CUtensorMap tmK;    // bf16 K  [B,S,G,d]   box {64,1,128,1}
+  CUtensorMap tmV;    // fp16 V  [B,S,G,d]   box {64,1,128,1}
+  CUtensorMap tmQ;    // bf16 Q  [B,S,N,d]   box {64,1,128,1}   (dense tiles)
+  CUtensorMap tmQs;   // bf16 Qs [B,S,d]     box {64,128,1}     (shared tiles)
+  const uint16_t* Q;  // for the routed row gather
+  const int32_t* bucket_off;
+  const int32_t* bucket_tok;
+  const int32_t* topk_idx;
+  const TileDesc* tiles;
+  const int32_t* tile_count;
+  void* O_sel;
+  void* o_bar;
+  void* s_out;
+  void* O_dense;
+  int64_t out_row_stride;
+  int* status;
+  int B, S, N, G, M, k, d;
+  int out_fp32;
+  int dense;          // 1: dense GQA tiles from blockIdx; 0: routed/shared list
+  float scale_log2;   // log2(e) / sqrt(d)
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_attention(const AttnArgs& a, int64_t grid, cudaStream_t st);
+
+struct CombineArgs {
+  const void* O_sel;
+  void* o_bar;
+  const float* w;
+  int64_t out_row_stride;
+  int T, G, k, d, out_fp32;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
+
+cudaError_t launch_selftest_wait(int* status, uint64_t limit_ns, cudaStream_t st);
+
+}  // namespace gqe

@@ -1,0 +1,98 @@
+"""CPU checks of the C-ABI library: it loads, exports every entry point the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import moe_routed_grouped_b200 as gqe
+from moe_routed_grouped_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "gqe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gqe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_symbols_exported():
+    names = _declared()
+    assert len(names) >= 9
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_lib.EXPORTS)
+
+
+def test_kv_cache_bytes_matches_pages():
+    # "AI 大模型之 GQA" §4.2 and the MQA/GQA explainer's 数值示例
+    assert gqe.gqe_kv_cache_bytes(32, 8, 4096, 128, 2, 1) == 512 * 2 ** 20
+    assert gqe.gqe_kv_cache_bytes(32, 32, 4096, 128, 2, 1) == 2048 * 2 ** 20
+    assert gqe.gqe_kv_cache_bytes(1, 32, 1024, 128, 2, 1) == 16777216
+    assert gqe.gqe_kv_cache_bytes(1, 8, 1024, 128, 2, 1) == 4194304
+    assert gqe.gqe_kv_cache_bytes(1, 1, 1024, 128, 2, 1) == 524288
+    assert gqe.gqe_kv_cache_bytes(1, 8, 1024, 128, 2, 3) == 3 * 4194304
+
+
+def test_status_strings():
+    for code in range(8):
+        assert gqe.gqe_status_string(code)
+    assert gqe.gqe_status_string(99) == "unknown status"
+
+
+FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced
+
+
+def _route(dm, ws_bytes=1 << 40, x=FAKE, ws=FAKE):
+    return _lib.LIB.gqe_route(ctypes.byref(dm), x, FAKE, None, FAKE, FAKE, FAKE, ws, ws_bytes,
+                              None)
+
+
+@pytest.mark.parametrize("args,code", [
+    ((1, 16, 16, 6, 1, 64, 256), 1),    # N % G != 0 is rejected, not remapped
+    ((1, 16, 16, 8, 3, 64, 256), 1),    # k > M
+    ((0, 16, 16, 8, 1, 64, 256), 1),    # empty batch
+    ((1, 0, 16, 8, 1, 64, 256), 1),     # empty sequence
+    ((1, 16, 16, 8, 1, 96, 256), 2),    # head dim outside {64, 128}
+    ((1, 16, 16, 8, 1, 64, 250), 2),    # d_model not a multiple of 8
+    ((1, 16, 48, 8, 1, 64, 256), 2),    # G*M = 48 not supported by the router
+    ((1, 16, 264, 4, 1, 64, 256), 2),   # M = 66 > 32
+])
+def test_route_rejects_bad_dims(args, code):
+    dm = _lib.dims(*args)
+    assert _route(dm) == code
+    if code == 1:
+        assert _lib.gqe_workspace_size(dm) == 0
+
+
+def test_route_rejects_pointers_and_workspace():
+    dm = _lib.dims(1, 16, 16, 8, 1, 64, 256)
+    assert _route(dm, x=None) == 1
+    assert _route(dm, x=ctypes.c_void_p(0x10008)) == 1            # misaligned
+    need = _lib.gqe_workspace_size(dm)
+    assert need > 0
+    assert _route(dm, ws_bytes=need - 1) == 5
+    assert _route(dm, ws=None) == 5
+
+
+def test_attention_rejects_bad_stride_and_workspace():
+    dm = _lib.dims(1, 16, 16, 8, 1, 64, 256)
+    L = _lib.LIB
+    def call(stride, ws_bytes=1 << 40):
+        return L.gqe_attention_prefill(ctypes.byref(dm), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                       FAKE, FAKE, stride, FAKE, ws_bytes, None)
+    assert call(60) == 1      # not a multiple of 8
+    assert call(8) == 1       # shorter than d
+    assert call(17 * 64, ws_bytes=10) == 5
+    assert L.gqe_dense_gqa_prefill(ctypes.byref(dm), FAKE, FAKE, None, FAKE, FAKE, 1 << 40,
+                                   None) == 1
+
+
+def test_workspace_grows_with_shape():
+    a = _lib.gqe_workspace_size(_lib.dims(1, 128, 16, 8, 1, 64, 256))
+    b = _lib.gqe_workspace_size(_lib.dims(8, 2048, 16, 8, 1, 64, 1024))
+    c = _lib.gqe_workspace_size(_lib.dims(1, 131072, 32, 8, 2, 128, 4096))
+    assert 0 < a < b < c
