@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""GQE causal-prefill benchmark.
+
+One step = the whole routed hot path on one batch of synthetic input that is
+already resident in HBM: gqe_route (router, softmax, exact top-k, weights)
+then gqe_attention_prefill (V conversion, bucketing, scheduling, routed +
+shared-head attention, combine).  The dense-GQA baseline from the same
+library is timed the same way for the routed/dense speedup.
+
+Prints ONE JSON line on rank 0.  Under torchrun every rank runs its own
+replica on its own GPU (weak scaling; batches are independent, so there is no
+collective on the data path); ranks only meet for barriers and the max-over-
+ranks of the device time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--sweep] [--impl ours|reference] [--no-cpu-baseline]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "GQE prefill tokens/s & useful TFLOP/s (% bf16 TC peak), S=2k–1M, vs dense GQA"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every ~2 ms."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, torch_dev):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = None
+            try:
+                import torch
+                pr = torch.cuda.get_device_properties(torch_dev)
+                bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(int(torch_dev))
+            self.nv, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that, do not guess
+            self.err = str(e)
+
+    def _reasons(self):
+        nv = self.nv
+        try:
+            return nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(),
+                                     self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM),
+                                     int(self._reasons())))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvml unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if len(inside) < 3:
+            inside = self.samples
+            window = "warm-up + timed region (timed region shorter than the sampling period)"
+        mhz = [s[1] for s in inside]
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = sorted(v for k, v in self.REASONS.items() if bits & k and k != 0x1)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+# ----------------------------------------------------------------- helpers
+def dev_bf16(torch, bits, device):
+    a = np.ascontiguousarray(bits, dtype=np.uint16)
+    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def gpu_inputs(torch, w, device, rank, host_gen):
+    """bf16 inputs on the device.  host_gen: the seeded synth generator (same
+    bits the oracle sees); otherwise torch's generator with the same
+    distributions (used for the very large sweep workloads)."""
+    if host_gen:
+        inp = make_inputs(w, seed_base=1000 * w.cid + 100 * rank)
+        out = {k: dev_bf16(torch, v, device) for k, v in inp.items() if k != "bias"}
+        out["bias"] = torch.from_numpy(inp["bias"]).to(device) if "bias" in inp else None
+        return out, inp
+    g = torch.Generator(device=device)
+    g.manual_seed(1000 * w.cid + 100 * rank)
+    def rn(*shape, std=1.0):
+        t = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        t.normal_(0.0, std, generator=g)
+        return t
+    out = dict(x=rn(w.B, w.S, w.d_model), W_r=rn(w.G, w.d_model, w.M, std=w.wr_std),
+               Q=rn(w.B, w.S, w.N, w.d), Qs=rn(w.B, w.S, w.d), K=rn(w.B, w.S, w.G, w.d),
+               V=rn(w.B, w.S, w.G, w.d))
+    out["bias"] = None
+    if w.bias0:
+        b = torch.zeros(w.G, w.M, dtype=torch.float32, device=device)
+        b[:, 0] = w.bias0
+        out["bias"] = b
+    return out, None
+
+
+def timed_loop(torch, fn, steps, warmup, flush, attn_events=False):
+    """Per-step device times (ms) with CUDA events on the launching stream.
+    The L2 flush before each step is outside the events."""
+    import moe_routed_grouped_b200 as gqe
+    for _ in range(warmup):
+        flush()
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    aev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)] if attn_events else []
+    for a, b in aev:  # create the event handles before handing them to the library
+        a.record(); b.record()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(steps):
+        flush()
+        if attn_events:
+            gqe.gqe_set_profile_events(*aev[i])
+        ev[i][0].record()
+        fn()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    if attn_events:
+        gqe.gqe_set_profile_events(None, None)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    attn_ms = [a.elapsed_time(b) for a, b in aev]
+    return step_ms, attn_ms, t0, t1
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(w, inp, budget_s=12.0, rows_per_seq=None):
+    """Time the CPU oracle (router + routed attention of all G*k + 1 heads)
+    on whole sequences of the workload until ~budget_s of CPU work."""
+    import oracle
+    done_tokens, t_total, seqs = 0, 0.0, 0
+    for b in range(w.B):
+        rows = np.arange(w.S) if rows_per_seq is None else \
+            np.unique(np.linspace(0, w.S - 1, rows_per_seq).astype(np.int64))
+        t0 = time.perf_counter()
+        xb = inp["x"][b:b + 1, rows]
+        idx, p, wts, _ = oracle.route(xb, inp["W_r"], inp.get("bias"), w.k)
+        full_idx = np.zeros((1, w.S, w.G, w.k), np.int32)
+        full_w = np.zeros((1, w.S, w.G, w.k))
+        full_idx[0, rows] = idx[0]
+        full_w[0, rows] = wts[0]
+        oracle.gqe_prefill_rows(inp["Q"][b:b + 1], inp["Qs"][b:b + 1], inp["K"][b:b + 1],
+                                inp["V"][b:b + 1], full_idx, full_w, [rows])
+        t_total += time.perf_counter() - t0
+        done_tokens += len(rows)
+        seqs += 1
+        if t_total >= budget_s:
+            break
+    return done_tokens, t_total, seqs
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    # each step: the oracle on an evenly spaced sample of one sequence's rows
+    rows_per_step = max(64, min(w.S, 512))
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, budget_s=0.0, rows_per_seq=min(rows_per_step, 64))
+    toks, secs = 0, 0.0
+    for _ in range(args.steps):
+        n, t, _ = oracle_sample(w, inp, budget_s=0.0, rows_per_seq=rows_per_step)
+        toks += n
+        secs += t
+    val = toks / secs
+    sample = (f"{args.steps} steps; each step routes and attends (all {w.G * w.k + 1} active "
+              f"heads) {rows_per_step} evenly spaced token positions of sequence 0")
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, world),
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, world):
+    return {"workload": w.name, "B": w.B, "S": w.S, "N": w.N, "G": w.G, "M": w.M, "k": w.k,
+            "d": w.d, "d_model": w.d_model, "router_bias_expert0": w.bias0,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "output": "float32 concat buffer (W_O input)",
+            "l2": "256 MiB buffer written between steps; the write is outside the step time"}
+
+
+# ----------------------------------------------------------------- our arm
+def measure_workload(torch, w, device, rank, steps, warmup, flush, host_gen, with_attn_events):
+    from moe_routed_grouped_b200.layer import GqePrefill
+    dev, host = gpu_inputs(torch, w, device, rank, host_gen)
+    L = GqePrefill(w.B, w.S, w.N, w.G, w.k, w.d, w.d_model, out_fp32=True, device=device)
+
+    def routed():
+        L.route(dev["x"], dev["W_r"], dev["bias"])
+        L.attention(dev["Q"], dev["Qs"], dev["K"], dev["V"])
+
+    def dense():
+        L.dense(dev["Q"], dev["K"], dev["V"])
+
+    r_ms, r_attn, t0, t1 = timed_loop(torch, routed, steps, warmup, flush, with_attn_events)
+    d_ms, d_attn, _, _ = timed_loop(torch, dense, steps, max(1, warmup // 2), flush,
+                                    with_attn_events)
+    status = L.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after {w.name}")
+    return dict(L=L, dev=dev, host=host, routed_ms=r_ms, routed_attn_ms=r_attn, dense_ms=d_ms,
+                dense_attn_ms=d_attn, t0=t0, t1=t1)
+
+
+def e2e_measure(torch, w, L, dev, steps):
+    """Through the public API with host buffers: pinned H2D of every input,
+    route + attention, D2H of the concat output and the top-k indices."""
+    host_in = {k: v.to("cpu").pin_memory() for k, v in dev.items() if v is not None}
+    out_h = torch.empty_like(L.concat, device="cpu").pin_memory()
+    idx_h = torch.empty_like(L.topk_idx, device="cpu").pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = out_h.numel() * out_h.element_size() + idx_h.numel() * idx_h.element_size()
+
+    def step():
+        for k, v in host_in.items():
+            dev[k].copy_(v, non_blocking=True)
+        L.route(dev["x"], dev["W_r"], dev["bias"])
+        L.attention(dev["Q"], dev["Qs"], dev["K"], dev["V"])
+        out_h.copy_(L.concat, non_blocking=True)
+        idx_h.copy_(L.topk_idx, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    return ms, h2d, d2h
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="layer250m", choices=sorted(WORKLOADS))
+    ap.add_argument("--sweep", action="store_true",
+                    help="also time the S=32k, 131k and 1M workloads (routed and dense)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    import torch
+    import moe_routed_grouped_b200  # noqa: F401  (fails loudly if libgqe.so is missing)
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    peaks, peak_src = load_peaks()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = lambda: flush_buf.zero_()  # noqa: E731
+
+    w = WORKLOADS[args.workload]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    res = measure_workload(torch, w, device, rank, args.steps, args.warmup, flush, True, True)
+    barrier()
+    clocks.stop()
+
+    tot_ms = sum(res["routed_ms"])
+    dense_tot_ms = sum(res["dense_ms"])
+    attn_ms = statistics.mean(res["routed_attn_ms"])
+    dense_attn_ms = statistics.mean(res["dense_attn_ms"])
+    if dist is not None:
+        t = torch.tensor([tot_ms, dense_tot_ms, attn_ms, dense_attn_ms], device=device,
+                         dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms, dense_tot_ms, attn_ms, dense_attn_ms = t.tolist()
+
+    tokens = w.B * w.S
+    value = world * tokens * args.steps / (tot_ms / 1e3)
+    dense_value = world * tokens * args.steps / (dense_tot_ms / 1e3)
+    ms_step = tot_ms / args.steps
+    fl_r, fl_d = w.useful_flop_routed(), w.useful_flop_dense()
+    useful_tf = fl_r / (ms_step / 1e3) / 1e12
+    dense_tf = fl_d / (dense_tot_ms / args.steps / 1e3) / 1e12
+    peak_tf = peaks["bf16_tflops"]
+    attn_tf = fl_r / (attn_ms / 1e3) / 1e12
+    dense_attn_tf = fl_d / (dense_attn_ms / 1e3) / 1e12
+
+    e2e_ms, h2d, d2h = e2e_measure(torch, w, res["L"], res["dev"], max(3, args.steps // 5))
+    e2e_val = world * tokens / (e2e_ms / 1e3)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 inputs; random-init router)",
+        "config": config_of(w, world),
+        "useful_tflops_per_gpu": useful_tf,
+        "useful_frac_of_peak": useful_tf / peak_tf,
+        "dense_gqa": {"value": dense_value, "unit": "tokens/s",
+                      "ms_per_step": dense_tot_ms / args.steps,
+                      "useful_tflops_per_gpu": dense_tf, "attention_kernel_ms": dense_attn_ms,
+                      "attention_kernel_tflops": dense_attn_tf},
+        "routed_over_dense": dense_tot_ms / tot_ms,
+        "roofline": {"kernel": "attn_kernel<%d> (routed + shared head)" % w.d, "bound": "tensor",
+                     "achieved": attn_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": attn_tf / peak_tf, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "attention_kernel_ms": attn_ms,
+                     "per_launch_flop": fl_r,
+                     "flop_definition": "4*d per visible (query, key) pair, (G*k+1)*B*S*(S+1)/2 pairs"},
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * (6 + (1 if w.k > 1 else 0)),
+        "clocks": clocks.summary(res["t0"], res["t1"]),
+    }
+
+    if args.sweep:
+        del res
+        torch.cuda.empty_cache()
+        sweep = []
+        for name in ("imbalanced32k", "wide131k", "million"):
+            ws = WORKLOADS[name]
+            k_steps = 3 if ws.S >= 1 << 20 else 5
+            r = measure_workload(torch, ws, device, rank, k_steps, 3, flush, False, True)
+            rm = sum(r["routed_ms"]) / k_steps
+            dm = sum(r["dense_ms"]) / k_steps
+            sweep.append({
+                "workload": name, "S": ws.S, "routed_ms": rm, "dense_ms": dm,
+                "routed_tokens_per_s": ws.B * ws.S / (rm / 1e3),
+                "routed_useful_tflops": ws.useful_flop_routed() / (rm / 1e3) / 1e12,
+                "dense_useful_tflops": ws.useful_flop_dense() / (dm / 1e3) / 1e12,
+                "routed_attention_kernel_tflops":
+                    ws.useful_flop_routed() / (statistics.mean(r["routed_attn_ms"]) / 1e3) / 1e12,
+                "routed_over_dense": dm / rm,
+                "inputs": "torch generator, same distributions as the synth recipe"})
+            del r
+            torch.cuda.empty_cache()
+        line["sweep"] = sweep
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = make_inputs(w)
+        n, secs, seqs = oracle_sample(w, host)
+        line["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{seqs} whole sequence(s) of {w.S} tokens: router + "
+                                          f"all {w.G * w.k + 1} active heads, float64 numpy"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

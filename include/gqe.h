@@ -36,7 +36,7 @@
  *    gqe_get_device_status().  Nothing is thrown across the ABI.
  *
  * Supported shapes: N % G == 0, M = N/G <= 32, 1 <= k <= M,
- * d in {64, 128}, G*M in {4, 8, 16, 32} for the router, d_model % 8 == 0,
+ * d in {64, 128}; for the router G*M in {4, 8, 16, 32} and d_model % 8 == 0;
  * B*S*G*max(k,M) < 2^31.
  */
 #ifndef GQE_H
@@ -163,6 +163,14 @@ const char* gqe_status_string(gqe_status s);
  * status (the latched code is read with gqe_get_device_status). */
 gqe_status gqe_selftest_bounded_wait(void* ws, size_t ws_bytes, int32_t limit_us,
                                      void* stream);
+
+/* Profiling hook.  When both handles are non-NULL, every later
+ * gqe_attention_prefill / gqe_dense_gqa_prefill call records `begin`
+ * (a cudaEvent_t) on its stream immediately before its attention kernel and
+ * `end` immediately after it, so the caller can time that kernel alone with
+ * cudaEventElapsedTime.  Pass NULLs to switch it off.  Process-wide setting,
+ * not thread-safe: meant for benchmarks. */
+void gqe_set_profile_events(void* begin, void* end);
 
 #ifdef __cplusplus
 }

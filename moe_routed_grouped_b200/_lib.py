@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libgqe.so")
 EXPORTS = (
     "gqe_workspace_size", "gqe_route", "gqe_bucket", "gqe_attention_prefill",
     "gqe_dense_gqa_prefill", "gqe_get_device_status", "gqe_kv_cache_bytes",
-    "gqe_status_string", "gqe_selftest_bounded_wait",
+    "gqe_status_string", "gqe_selftest_bounded_wait", "gqe_set_profile_events",
 )
 
 STATUS = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED", 3: "GQE_ERR_CUDA",
@@ -51,6 +51,7 @@ def _load() -> ctypes.CDLL:
         "gqe_kv_cache_bytes": (ctypes.c_uint64, [I32, I32, I64, I32, I32, I32]),
         "gqe_status_string": (ctypes.c_char_p, [I32]),
         "gqe_selftest_bounded_wait": (I32, [P, SZ, I32, P]),
+        "gqe_set_profile_events": (None, [P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -128,3 +129,10 @@ def gqe_selftest_bounded_wait(ws, limit_us, stream=None, check=True):
     r = LIB.gqe_selftest_bounded_wait(_ptr(ws), ws.numel() * ws.element_size(), int(limit_us),
                                       _stream(stream))
     return _check(r, "gqe_selftest_bounded_wait") if check else r
+
+
+def gqe_set_profile_events(begin=None, end=None):
+    """begin/end: torch.cuda.Event (already recorded once) or None."""
+    b = None if begin is None else ctypes.c_void_p(begin.cuda_event)
+    e = None if end is None else ctypes.c_void_p(end.cuda_event)
+    LIB.gqe_set_profile_events(b, e)

@@ -102,6 +102,16 @@ gqe_status check_dims(const gqe_dims* d, bool router) {
 
 gqe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
 
+cudaEvent_t g_prof_begin = nullptr, g_prof_end = nullptr;
+
+cudaError_t timed_attention(const AttnArgs& a, int64_t grid, cudaStream_t s) {
+  const bool prof = g_prof_begin && g_prof_end;
+  if (prof && cudaEventRecord(g_prof_begin, s) != cudaSuccess) return cudaErrorUnknown;
+  cudaError_t e = launch_attention(a, grid, s);
+  if (e == cudaSuccess && prof) e = cudaEventRecord(g_prof_end, s);
+  return e;
+}
+
 }  // namespace
 
 extern "C" {
@@ -123,7 +133,6 @@ gqe_status gqe_route(const gqe_dims* dims, const void* x, const void* W_r, const
   if (!aligned16(ws) || ws_bytes < L.total) return GQE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* wb = static_cast<uint8_t*>(ws);
-  if (cudaMemsetAsync(wb + L.counters, 0, 256, s) != cudaSuccess) return GQE_ERR_CUDA;
   RouteArgs a{};
   a.x = static_cast<const uint16_t*>(x);
   a.Wr = static_cast<const uint16_t*>(W_r);
@@ -132,6 +141,8 @@ gqe_status gqe_route(const gqe_dims* dims, const void* x, const void* W_r, const
   a.p = p;
   a.w = w;
   a.fix_list = reinterpret_cast<int32_t*>(wb + L.fix_list);
+  a.wt = reinterpret_cast<float*>(wb + L.wt);
+  a.wsq = reinterpret_cast<float*>(wb + L.wsq);
   a.fix_count = reinterpret_cast<int32_t*>(wb + L.counters);
   a.status = reinterpret_cast<int*>(wb + L.status);
   a.T = dims->B * dims->S;
@@ -151,6 +162,7 @@ static BucketArgs bucket_args(const gqe_dims* dims, const int32_t* topk_idx, int
   a.tiles_raw = reinterpret_cast<TileDesc*>(wb + L.tiles_raw);
   a.tiles = reinterpret_cast<TileDesc*>(wb + L.tiles);
   a.tile_count = reinterpret_cast<int32_t*>(wb + L.counters) + 1;
+  a.done = reinterpret_cast<int32_t*>(wb + L.counters) + 2;
   a.status = reinterpret_cast<int*>(wb + L.status);
   a.B = dims->B;
   a.S = dims->S;
@@ -172,7 +184,7 @@ gqe_status gqe_bucket(const gqe_dims* dims, const int32_t* topk_idx, int32_t* bu
   if (!aligned16(ws) || ws_bytes < L.total) return GQE_ERR_WORKSPACE;
   uint8_t* wb = static_cast<uint8_t*>(ws);
   const BucketArgs a = bucket_args(dims, topk_idx, bucket_off, bucket_tok, wb, L);
-  return from_cuda(launch_bucket(a, false, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_prep(a, nullptr, false, static_cast<cudaStream_t>(stream)));
 }
 
 static AttnArgs attn_common(const gqe_dims* dims, uint8_t* wb, const WsLayout& L) {
@@ -212,12 +224,9 @@ gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void
 
   ConvertArgs cv{static_cast<const uint16_t*>(V), reinterpret_cast<uint16_t*>(wb + L.v16),
                  B * S * G * d, reinterpret_cast<int*>(wb + L.status)};
-  cudaError_t e = launch_convert_v(cv, s);
-  if (e != cudaSuccess) return GQE_ERR_CUDA;
-
   const BucketArgs ba = bucket_args(dims, topk_idx, reinterpret_cast<int32_t*>(wb + L.bucket_off),
                                     reinterpret_cast<int32_t*>(wb + L.bucket_tok), wb, L);
-  e = launch_bucket(ba, true, s);
+  cudaError_t e = launch_prep(ba, &cv, true, s);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
 
   AttnArgs a = attn_common(dims, wb, L);
@@ -238,7 +247,7 @@ gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void
   a.s_out = s_out;
   a.out_row_stride = out_row_stride;
   a.dense = 0;
-  e = launch_attention(a, L.n_raw_tiles, s);
+  e = timed_attention(a, L.n_raw_tiles, s);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
 
   if (dims->k > 1) {
@@ -276,7 +285,7 @@ gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void
   a.O_dense = O;
   a.dense = 1;
   const int64_t nq = (S + kTileM - 1) / kTileM;
-  return from_cuda(launch_attention(a, B * dims->N * nq, s));
+  return from_cuda(timed_attention(a, B * dims->N * nq, s));
 }
 
 gqe_status gqe_get_device_status(void* ws, int32_t clear, void* stream) {
@@ -311,6 +320,11 @@ const char* gqe_status_string(gqe_status s) {
     case GQE_ERR_NONFINITE: return "non-finite value or value outside the fp16 range";
   }
   return "unknown status";
+}
+
+void gqe_set_profile_events(void* begin, void* end) {
+  g_prof_begin = static_cast<cudaEvent_t>(begin);
+  g_prof_end = static_cast<cudaEvent_t>(end);
 }
 
 gqe_status gqe_selftest_bounded_wait(void* ws, size_t ws_bytes, int32_t limit_us, void* stream) {

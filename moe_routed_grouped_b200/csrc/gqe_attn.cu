@@ -48,6 +48,10 @@ struct Cfg {
 };
 
 constexpr int kThreads = 192;
+// Of every 8 column pairs, this many are exponentiated by a polynomial on the
+// FMA pipe; the rest use the MUFU ex2 unit (16 lanes/clock/SM), which would
+// otherwise bound d = 64 attention at about half the tensor-core rate.
+constexpr int kPolyPairs = 3;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 
@@ -324,11 +328,18 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
           for (int e = 0; e < 32; ++e)
             if (kbase + 32 * c + e > pos) sv[c][e] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      // row max: 8 independent chains of 3-input max
+      float mxp[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mxp[q] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[c][e]));
+        for (int e = 0; e < 32; e += 2)
+          mxp[(e >> 1) & 7] = fmax3f(mxp[(e >> 1) & 7], __uint_as_float(sv[c][e]),
+                                     __uint_as_float(sv[c][e + 1]));
+      const float mx = fmax3f(fmax3f(mxp[0], mxp[1], mxp[2]), fmax3f(mxp[3], mxp[4], mxp[5]),
+                              fmaxf(mxp[6], mxp[7]));
       const float mnew = fmaxf(m_used, mx * sl2);
       float factor = 1.f;
       if (mnew - m_used > 8.f) {
@@ -336,35 +347,55 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
         m_used = mnew;
       }
       l *= factor;
-      uint32_t pk[2][32];
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c][e]), sl2, -m_used));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c][e + 1]), sl2, -m_used));
-          rs += p0 + p1;
-          pk[c >> 1][(c & 1) * 16 + e / 2] = pack_half2(p0, p1);
-        }
-      l += rs;
+      // P.V of the previous tile must be done before P and O are touched
       if (j > 0) {
         if (!wait(&bars[kBarODone], (j - 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xFFFFFFFFu, factor != 1.f)) {
+      }
+      // p = 2^(s * scale * log2e - m), packed to fp16 and written to TMEM
+      // 32 columns at a time
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_used, -m_used);
+      uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(tbase + lane_off + C::kTmemO + 32 * c, ov);
-            tmem_ld_wait(ov);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
-            tmem_st32(tbase + lane_off + C::kTmemO + 32 * c, ov);
+        for (int e = 0; e < 32; e += 2) {
+          const uint64_t y2 =
+              f2_fma(f2_pack(__uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1])), sl2x2,
+                     negm2);
+          float p0, p1;
+          if (((e >> 1) & 7) < kPolyPairs) {  // this pair on the FMA pipe
+            exp2_poly_pair(y2, p0, p1);
+          } else {                             // this pair on the MUFU unit
+            float y0, y1;
+            f2_unpack(y2, y0, y1);
+            p0 = ex2_approx(y0);
+            p1 = ex2_approx(y1);
           }
+          rs2[(e >> 1) & 3] = f2_add(rs2[(e >> 1) & 3], f2_pack(p0, p1));
+          pk[e / 2] = pack_half2(p0, p1);
+        }
+        tmem_st16(tbase + lane_off + C::kTmemP + 16 * c, pk);
+      }
+      float r0, r1, r2, r3, r4, r5, r6, r7;
+      f2_unpack(rs2[0], r0, r1);
+      f2_unpack(rs2[1], r2, r3);
+      f2_unpack(rs2[2], r4, r5);
+      f2_unpack(rs2[3], r6, r7);
+      l += ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
+      // rescale O (rare: only when the running max grew by more than 2^8)
+      if (j > 0 && __any_sync(0xFFFFFFFFu, factor != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tbase + lane_off + C::kTmemO + 32 * c, ov);
+          tmem_ld_wait(ov);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+          tmem_st32(tbase + lane_off + C::kTmemO + 32 * c, ov);
         }
       }
-      tmem_st32(tbase + lane_off + C::kTmemP, pk[0]);
-      tmem_st32(tbase + lane_off + C::kTmemP + 32, pk[1]);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

@@ -1,6 +1,6 @@
 // Bucketing, work-list scheduling, V conversion and the k>1 combine.
 //
-// bucket_kernel: one CTA per (batch, group).  Each token appears once in each
+// bucket_body: one CTA per (batch, group).  Each token appears once in each
 // of the k buckets its router picked ("论文综述：分组查询专家" §二 路由器:
 // only the selected heads compute), so the (b, g) block of the token list has
 // the fixed size S*k and starts at (b*G + g)*S*k; the per-expert offsets are
@@ -16,13 +16,13 @@ namespace {
 constexpr int kBucketThreads = 1024;
 constexpr int kBucketWarps = kBucketThreads / 32;
 
-__global__ void __launch_bounds__(kBucketThreads) bucket_kernel(const BucketArgs a) {
+__device__ void bucket_body(const BucketArgs& a, int bg) {
   __shared__ int cnt[kMaxM];
   __shared__ int start[kMaxM];
   __shared__ int running[kMaxM];
   __shared__ int wcnt[kMaxM][kBucketWarps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bg = blockIdx.x, b = bg / a.G, g = bg % a.G;
+  const int b = bg / a.G, g = bg % a.G;
   const int S = a.S, G = a.G, M = a.M, k = a.k;
   const int64_t base = static_cast<int64_t>(bg) * S * k;
   if (tid < kMaxM) {
@@ -126,8 +126,7 @@ __global__ void __launch_bounds__(kBucketThreads) bucket_kernel(const BucketArgs
 // grid's tail is short).  Counting sort on nkv in [1, ceil(S/128)].
 constexpr int kSchedThreads = 1024;
 
-__global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const BucketArgs a) {
-  extern __shared__ int hist[];  // nq + 2 bins
+__device__ void schedule_body(const BucketArgs& a, int* hist /* nq + 2 bins */) {
   const int tid = threadIdx.x;
   const int nq = (a.S + kTileM - 1) / kTileM;
   const int64_t n_routed = static_cast<int64_t>(a.B) * a.G * a.cap_bg;
@@ -167,11 +166,11 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const BucketArg
 
 // V (bf16) -> fp16 for the P.V product; P is rounded to fp16 (11-bit
 // significand), which is what keeps the output within 1e-3 relative L2.
-__global__ void convert_v_kernel(const ConvertArgs a) {
+__device__ void convert_v_body(const ConvertArgs& a, int block, int nblocks) {
   const int64_t n8 = a.n / 8;
   bool bad = false;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+  for (int64_t i = block * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(nblocks) * blockDim.x) {
     const uint4 v = reinterpret_cast<const uint4*>(a.V)[i];
     const uint32_t in[4] = {v.x, v.y, v.z, v.w};
     uint32_t out[4];
@@ -186,6 +185,31 @@ __global__ void convert_v_kernel(const ConvertArgs a) {
   }
   if (bad) latch_status(a.status, GQE_ERR_NONFINITE);
 }
+
+// One launch for the work that precedes attention: CTAs [0, B*G) bucket one
+// (batch, group) each, the remaining CTAs convert V to fp16, and the CTA that
+// finishes last (fenced counter) sorts the work list.
+__global__ void __launch_bounds__(kBucketThreads)
+    prep_kernel(const BucketArgs a, const ConvertArgs cv, int with_schedule) {
+  extern __shared__ int hist[];
+  __shared__ int is_last;
+  const int nbucket = a.B * a.G;
+  if (static_cast<int>(blockIdx.x) < nbucket)
+    bucket_body(a, blockIdx.x);
+  else
+    convert_v_body(cv, blockIdx.x - nbucket, gridDim.x - nbucket);
+  if (!with_schedule) return;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(a.done, 1) == static_cast<int>(gridDim.x) - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  schedule_body(a, hist);
+  if (threadIdx.x == 0) *a.done = 0;  // ready for the next call
+}
+
+__global__ void convert_v_kernel(const ConvertArgs a) { convert_v_body(a, blockIdx.x, gridDim.x); }
 
 // o_bar[t, g] = sum_j w[t, g, j] * O_sel[t, g, j] in slot order
 // (review §二 三个关键部件, the renormalised weighted-sum slot); k > 1 only.
@@ -232,18 +256,25 @@ __global__ void combine_kernel(const CombineArgs a) {
 
 }  // namespace
 
-cudaError_t launch_bucket(const BucketArgs& a, bool with_schedule, cudaStream_t st) {
-  bucket_kernel<<<a.B * a.G, kBucketThreads, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || !with_schedule) return e;
+cudaError_t launch_prep(const BucketArgs& a, const ConvertArgs* cv, bool with_schedule,
+                        cudaStream_t st) {
   const int nq = (a.S + kTileM - 1) / kTileM;
-  const size_t smem = sizeof(int) * (nq + 2);
+  const size_t smem = with_schedule ? sizeof(int) * (nq + 2) : 0;
   if (smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  schedule_kernel<<<1, kSchedThreads, smem, st>>>(a);
+  int nconv = 0;
+  ConvertArgs c{};
+  if (cv) {
+    c = *cv;
+    const int64_t n8 = c.n / 8;
+    nconv = static_cast<int>((n8 + kBucketThreads - 1) / kBucketThreads);
+    if (nconv > 148 * 2) nconv = 148 * 2;
+    if (nconv < 1) nconv = 1;
+  }
+  prep_kernel<<<a.B * a.G + nconv, kBucketThreads, smem, st>>>(a, c, with_schedule ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -229,6 +229,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -238,6 +247,56 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// Packed pairs of float32 (Blackwell f32x2 arithmetic: two lanes per op).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^y for a pair of floats on the FMA pipe instead of the MUFU unit:
+// y = j + f with j = rint(y) (adding and subtracting 1.5 * 2^23), 2^f from a
+// degree-3 polynomial on [-1/2, 1/2] that minimises the relative error
+// (max 7.5e-5; coefficients from csrc/exp2_poly.py), and j added to the
+// exponent field.  Inputs below -120 (masked scores are -inf) give 2^-120.
+__device__ __forceinline__ void exp2_poly_pair(uint64_t y2, float& r0, float& r1) {
+  constexpr float kC0 = 9.999280572e-01f, kC1 = 6.932609677e-01f, kC2 = 2.426111251e-01f,
+                  kC3 = 5.517166853e-02f, kRound = 12582912.0f;
+  float y0, y1;
+  f2_unpack(y2, y0, y1);
+  const uint64_t y = f2_pack(fmaxf(y0, -120.f), fmaxf(y1, -120.f));
+  const uint64_t t = f2_add(y, f2_pack(kRound, kRound));
+  const uint64_t jf = f2_add(t, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(jf, f2_pack(-1.f, -1.f), y);
+  uint64_t p = f2_fma(f2_pack(kC3, kC3), f, f2_pack(kC2, kC2));
+  p = f2_fma(p, f, f2_pack(kC1, kC1));
+  p = f2_fma(p, f, f2_pack(kC0, kC0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  // t's bit pattern is 0x4B400000 + j, and 0x4B400000 << 23 == 0 (mod 2^32)
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -29,8 +29,11 @@ struct TileDesc {
 // Byte offsets of the regions inside the caller's workspace.
 struct WsLayout {
   size_t status;      // int32 status word (latched errors)
-  size_t counters;    // int32[16]: [0] router fixup count, [1] tile count
+  size_t counters;    // int32[16]: [0] exact router decisions (cumulative),
+                      // [1] tile count, [2] prep-kernel completion counter
   size_t fix_list;    // int32[B*S*G]: (token*G + g) pairs needing exact routing
+  size_t wt;          // float32 [d_model][G*M]: W_r transposed for the router
+  size_t wsq;         // float32 [G*M]: column sums of squares of W_r
   size_t v16;         // fp16 [B,S,G,d]: V converted for the P.V product
   size_t bucket_off;  // int32[B*G*M + 1]
   size_t bucket_tok;  // int32[B*G*S*k]
@@ -53,6 +56,8 @@ inline WsLayout make_ws_layout(const gqe_dims& d) {
   L.status = off;     off += 256;
   L.counters = off;   off += 256;
   L.fix_list = off;   off = align_up(off + sizeof(int32_t) * B * S * G, 256);
+  L.wt = off;         off = align_up(off + sizeof(float) * d.d_model * G * M, 256);
+  L.wsq = off;        off = align_up(off + sizeof(float) * G * M, 256);
   L.v16 = off;        off = align_up(off + sizeof(uint16_t) * B * S * G * hd, 256);
   L.bucket_off = off; off = align_up(off + sizeof(int32_t) * (B * G * M + 1), 256);
   L.bucket_tok = off; off = align_up(off + sizeof(int32_t) * B * G * S * k, 256);
@@ -66,6 +71,8 @@ inline WsLayout make_ws_layout(const gqe_dims& d) {
 struct RouteArgs {
   const uint16_t* x;    // bf16 [T, dm]
   const uint16_t* Wr;   // bf16 [G, dm, M]
+  float* wt;            // float32 [dm][G*M] (written by the prep kernel)
+  float* wsq;           // float32 [G*M]
   const float* bias;    // [G*M] or null
   int32_t* topk_idx;    // [T, G, k]
   float* p;             // [T, G, M]
@@ -84,12 +91,12 @@ struct BucketArgs {
   TileDesc* tiles_raw;      // routed slots then shared-head tiles
   TileDesc* tiles;          // sorted output
   int32_t* tile_count;
+  int32_t* done;            // CTA completion counter (self-resetting)
   int* status;
   int B, S, G, M, k;
   int64_t cap_bg;
   int64_t n_raw_tiles;
 };
-cudaError_t launch_bucket(const BucketArgs& a, bool with_schedule, cudaStream_t st);
 
 struct ConvertArgs {
   const uint16_t* V;  // bf16
@@ -97,6 +104,9 @@ struct ConvertArgs {
   int64_t n;          // elements (multiple of 8)
   int* status;
 };
+// Bucketing (+ optional V conversion and work-list sort) in one launch.
+cudaError_t launch_prep(const BucketArgs& a, const ConvertArgs* cv, bool with_schedule,
+                        cudaStream_t st);
 cudaError_t launch_convert_v(const ConvertArgs& a, cudaStream_t st);
 
 struct AttnArgs {

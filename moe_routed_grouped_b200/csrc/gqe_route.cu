@@ -5,13 +5,13 @@
 // K_g(x_i) = TopK_m(p_{i,g,m}, k); §二 三个关键部件: w = p / sum_{K_g} p.
 //
 // Exactness.  Top-k is defined on the exact logits (ties -> lower index).
-// route_kernel computes each logit with a sequential float32 FMA chain over
-// d_model exact bf16*bf16 products, so |l_hat - l| <= (d_model+1) u sum|x_j w_j|
-// (+ the bias rounding), with u = 2^-24; sum|x_j w_j| is bounded by
-// ||x||_2 ||w||_2.  A decision is kept only if every selected logit beats every
-// later one by more than the two bounds; otherwise the (token, group) pair is
-// queued and route_fixup_kernel decides it with an exact fixed-point
-// (Kulisch-style) accumulation of the products.
+// route_kernel sums the exact bf16*bf16 products in float32 with a longest
+// rounding chain of D = 32 + n_chunks + 3 operations, so
+// |l_hat - l| <= D u sum|x_j w_j| (u = 2^-24), and sum|x_j w_j| <= ||x|| ||w||.
+// A decision is kept only if every selected logit beats every later one by
+// more than the two bounds; otherwise the same CTA recomputes that (token,
+// group) pair with an exact fixed-point (Kulisch-style) accumulation of the
+// products.
 #include <cuda_bf16.h>
 
 #include "gqe_device.cuh"
@@ -19,139 +19,262 @@
 namespace gqe {
 namespace {
 
-constexpr int kRouteThreads = 128;  // one token per thread
-constexpr int kRouteChunk = 64;     // d_model rows of W_r staged per step
+constexpr int kRouteWarps = 4;
+constexpr int kRouteThreads = 32 * kRouteWarps;
+constexpr int kRouteChunk = 32;     // d_model rows per chunk; warp w owns chunks w, w+4, ...
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
   return __uint_as_float(b << 16);
 }
 
+__device__ void exact_rank_pair(const RouteArgs& a, int t, int g, int* sel_smem);
+
+// W_r [G][dm][M] (bf16) -> wt [dm][G*M] (float32) and the column sums of
+// squares wsq[G*M].  Block b covers rows 32b .. 32b+31; thread (j, col).
+template <int GM>
+__global__ void __launch_bounds__(32 * GM) route_prep_kernel(const RouteArgs a) {
+  const int col = threadIdx.x % GM, jj = threadIdx.x / GM;
+  const int j = blockIdx.x * 32 + jj;
+  const int g = col / a.M, m = col % a.M;
+  float v = 0.f;
+  if (j < a.dm) {
+    v = bf16_bits_to_float(a.Wr[(static_cast<int64_t>(g) * a.dm + j) * a.M + m]);
+    a.wt[static_cast<int64_t>(j) * GM + col] = v;
+  }
+  __shared__ float part[32][GM + 1];
+  part[jj][col] = v * v;
+  __syncthreads();
+  if (threadIdx.x < GM) {
+    float s2 = 0.f;
+    for (int r = 0; r < 32; ++r) s2 += part[r][threadIdx.x];
+    atomicAdd(&a.wsq[threadIdx.x], s2);
+  }
+}
+
+// Tokens per lane: 2 while the accumulators fit in registers, else 1.
+template <int GM>
+struct RouteShape {
+  static constexpr int kTPL = GM <= 16 ? 2 : 1;
+  static constexpr int kTok = 32 * kTPL;   // tokens per tile
+};
+
+template <int GM>
+struct RouteSmem {
+  using Sh = RouteShape<GM>;
+  float ws[kRouteWarps][kRouteChunk][GM];           // this warp's W_r chunk, [j][col]
+  float red[kRouteWarps][Sh::kTok][GM + 1];         // per-warp partial logits
+  float lgt[Sh::kTok][GM + 1];                      // logits (+ bias)
+  float err[Sh::kTok][GM + 1];                      // their rounding-error bounds
+  float xsq[kRouteWarps][Sh::kTok];
+  int nflag;
+  int flags[Sh::kTok * 32];
+  int sel[kRouteWarps][kMaxM];
+};
+
+// x values of one chunk for one token: 32 bf16 in 4 x 16 bytes
+__device__ __forceinline__ void load_x_chunk(const uint16_t* xrow, bool ok, int c0, int rows,
+                                             uint4 (&v)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    v[q] = (ok && 8 * q < rows) ? __ldg(reinterpret_cast<const uint4*>(xrow + c0 + 8 * q))
+                                : make_uint4(0u, 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ float xval(const uint4 (&v)[4], int j) {
+  const uint4 q = v[j >> 3];
+  const uint32_t w = ((j & 7) >> 1) == 0 ? q.x : ((j & 7) >> 1) == 1 ? q.y : ((j & 7) >> 1) == 2 ? q.z : q.w;
+  return bf16_bits_to_float((w >> ((j & 1) * 16)) & 0xFFFFu);
+}
+
+// Chunk rows [c0, c0 + 32) of the transposed W_r: 32 * GM contiguous floats,
+// GM / 4 16-byte pieces per lane (rows past d_model read as zero).
+template <int GM>
+__device__ __forceinline__ void load_wt_chunk(const float* wt, int c0, int rows,
+                                              float4 (&v)[GM / 4]) {
+  const int lane = threadIdx.x & 31;
+  const float4* src = reinterpret_cast<const float4*>(wt + static_cast<int64_t>(c0) * GM);
+#pragma unroll
+  for (int i = 0; i < GM / 4; ++i) {
+    const int piece = lane + 32 * i;  // rows of 4*... : piece / (GM/4) is the row
+    v[i] = (piece / (GM / 4) < rows) ? __ldg(src + piece) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// Persistent CTAs of 4 warps; a tile is kTok tokens.  Warp w sums the
+// products of the d_model chunks w, w+4, ... ; lane l keeps its tokens' x
+// values in registers and reads each W_r row as a broadcast from the warp's
+// shared-memory copy of the chunk (copied from the float32 transpose made by
+// route_prep_kernel).  Each
+// chunk's 32 products are summed in fresh accumulators, chunk sums are added
+// per warp and the four warp sums are added in warp order, so the longest
+// rounding chain is 32 + ceil(n_chunks/4) + 4 (with the bias): that is the D
+// of the bound |l_hat - l| <= D u ||x|| ||w_c||, u = 2^-24.
 template <int GM>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
-  __shared__ __align__(16) float Ws[kRouteChunk][GM];
-  __shared__ float wsq[GM];
-  __shared__ float lg[kRouteThreads][GM + 1];
-
-  const int tid = threadIdx.x;
-  const int t = blockIdx.x * kRouteThreads + tid;
-  const bool valid = t < a.T;
+  using Sh = RouteShape<GM>;
+  constexpr int TPL = Sh::kTPL, TOK = Sh::kTok;
+  extern __shared__ __align__(16) uint8_t route_smem_raw[];
+  RouteSmem<GM>& sm = *reinterpret_cast<RouteSmem<GM>*>(route_smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dm = a.dm, M = a.M, G = a.G, k = a.k;
+  const int nchunks = (dm + kRouteChunk - 1) / kRouteChunk;
+  const int ntiles = (a.T + TOK - 1) / TOK;
+  const float cerr =
+      static_cast<float>(32 + (nchunks + kRouteWarps - 1) / kRouteWarps + 4) * 5.9604645e-8f *
+      1.01f;
 
-  if (tid < GM) wsq[tid] = 0.f;
-  float acc[GM];
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int t0 = tile * TOK;
+    const int ntok = min(TOK, a.T - t0);
+    if (tid == 0) sm.nflag = 0;
+    const uint16_t* xrow[TPL];
+    bool xok[TPL];
 #pragma unroll
-  for (int c = 0; c < GM; ++c) acc[c] = 0.f;
-  float xsq = 0.f, wpart = 0.f;
-  const uint16_t* xrow = a.x + static_cast<int64_t>(valid ? t : 0) * dm;
-
-  for (int c0 = 0; c0 < dm; c0 += kRouteChunk) {
-    const int rows = min(kRouteChunk, dm - c0);
-    __syncthreads();
-    // stage W_r[g, c0 + j, m] as Ws[j][g*M + m] (fp32); column of this thread
-    // is tid % GM because GM divides the block size.
-    for (int e = tid; e < kRouteChunk * GM; e += kRouteThreads) {
-      const int j = e / GM, col = e % GM;
-      float v = 0.f;
-      if (j < rows) {
-        const int g = col / M, m = col % M;
-        v = bf16_bits_to_float(a.Wr[(static_cast<int64_t>(g) * dm + c0 + j) * M + m]);
-      }
-      Ws[j][col] = v;
-      wpart = fmaf(v, v, wpart);
+    for (int r = 0; r < TPL; ++r) {
+      const int tl = lane + 32 * r;
+      xok[r] = tl < ntok;
+      xrow[r] = a.x + static_cast<int64_t>(t0 + (xok[r] ? tl : 0)) * dm;
     }
-    __syncthreads();
-    if (valid) {
-      for (int jj = 0; jj < rows; jj += 8) {
-        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xrow + c0 + jj));
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    float acc[TPL][GM];
+    float xsq[TPL];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float xf = bf16_bits_to_float((xw[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
-          xsq = fmaf(xf, xf, xsq);
-          const float4* wr = reinterpret_cast<const float4*>(&Ws[jj + e][0]);
+    for (int r = 0; r < TPL; ++r) {
+      xsq[r] = 0.f;
 #pragma unroll
-          for (int c4 = 0; c4 < GM / 4; ++c4) {
-            const float4 w4 = wr[c4];
-            acc[4 * c4 + 0] = fmaf(xf, w4.x, acc[4 * c4 + 0]);
-            acc[4 * c4 + 1] = fmaf(xf, w4.y, acc[4 * c4 + 1]);
-            acc[4 * c4 + 2] = fmaf(xf, w4.z, acc[4 * c4 + 2]);
-            acc[4 * c4 + 3] = fmaf(xf, w4.w, acc[4 * c4 + 3]);
+      for (int c = 0; c < GM; ++c) acc[r][c] = 0.f;
+    }
+    uint4 xv[TPL][4];
+    float4 wv[GM / 4];
+    int ci = warp;
+    if (ci < nchunks) {
+      const int rows = min(kRouteChunk, dm - ci * kRouteChunk);
+#pragma unroll
+      for (int r = 0; r < TPL; ++r) load_x_chunk(xrow[r], xok[r], ci * kRouteChunk, rows, xv[r]);
+      load_wt_chunk<GM>(a.wt, ci * kRouteChunk, rows, wv);
+    }
+    for (; ci < nchunks; ci += kRouteWarps) {
+      const int c0 = ci * kRouteChunk;
+      const int rows = min(kRouteChunk, dm - c0);
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < GM / 4; ++i)
+        reinterpret_cast<float4*>(&sm.ws[warp][0][0])[lane + 32 * i] = wv[i];
+      __syncwarp();
+      uint4 xc[TPL][4];
+#pragma unroll
+      for (int r = 0; r < TPL; ++r)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xc[r][q] = xv[r][q];
+      const int cn = ci + kRouteWarps;  // prefetch this warp's next chunk
+      if (cn < nchunks) {
+        const int rows_n = min(kRouteChunk, dm - cn * kRouteChunk);
+#pragma unroll
+        for (int r = 0; r < TPL; ++r)
+          load_x_chunk(xrow[r], xok[r], cn * kRouteChunk, rows_n, xv[r]);
+        load_wt_chunk<GM>(a.wt, cn * kRouteChunk, rows_n, wv);
+      }
+      float cacc[TPL][GM];
+#pragma unroll
+      for (int r = 0; r < TPL; ++r)
+#pragma unroll
+        for (int c = 0; c < GM; ++c) cacc[r][c] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kRouteChunk; ++j) {
+        float xr[TPL];
+#pragma unroll
+        for (int r = 0; r < TPL; ++r) {
+          xr[r] = xval(xc[r], j);
+          xsq[r] = fmaf(xr[r], xr[r], xsq[r]);
+        }
+        const float4* wrow = reinterpret_cast<const float4*>(&sm.ws[warp][j][0]);
+#pragma unroll
+        for (int c4 = 0; c4 < GM / 4; ++c4) {
+          const float4 w4 = wrow[c4];
+#pragma unroll
+          for (int r = 0; r < TPL; ++r) {
+            cacc[r][4 * c4 + 0] = fmaf(xr[r], w4.x, cacc[r][4 * c4 + 0]);
+            cacc[r][4 * c4 + 1] = fmaf(xr[r], w4.y, cacc[r][4 * c4 + 1]);
+            cacc[r][4 * c4 + 2] = fmaf(xr[r], w4.z, cacc[r][4 * c4 + 2]);
+            cacc[r][4 * c4 + 3] = fmaf(xr[r], w4.w, cacc[r][4 * c4 + 3]);
           }
         }
       }
-    }
-  }
-  atomicAdd(&wsq[tid % GM], wpart);
+      (void)rows;
 #pragma unroll
-  for (int c = 0; c < GM; ++c) lg[tid][c] = acc[c];
-  __syncthreads();
-  if (!valid) return;
+      for (int r = 0; r < TPL; ++r)
+#pragma unroll
+        for (int c = 0; c < GM; ++c) acc[r][c] += cacc[r][c];
+    }
+#pragma unroll
+    for (int r = 0; r < TPL; ++r) {
+      sm.xsq[warp][lane + 32 * r] = xsq[r];
+#pragma unroll
+      for (int c = 0; c < GM; ++c) sm.red[warp][lane + 32 * r][c] = acc[r][c];
+    }
+    __syncthreads();
 
-  const float xn = sqrtf(xsq);
-  // bound factor: (dm + 3) u, inflated by 1% for the rounding of the norms
-  const float cerr = static_cast<float>(dm + 3) * 5.9604645e-8f * 1.01f;
-  const int64_t tG = static_cast<int64_t>(t) * G;
-  bool nonfinite = false;
-
-  for (int g = 0; g < G; ++g) {
-    float l[kMaxM], e[kMaxM];
-    for (int m = 0; m < M; ++m) {
-      const int col = g * M + m;
+    // logits and their bounds, one (token, column) per thread
+    bool nonfinite = false;
+    for (int q = tid; q < ntok * GM; q += kRouteThreads) {
+      const int ql = q / GM, col = q % GM;
       const float b = a.bias ? a.bias[col] : 0.f;
-      l[m] = lg[tid][col] + b;
-      e[m] = cerr * fmaf(xn, sqrtf(wsq[col]), fabsf(b)) + 1e-36f;
-      nonfinite |= !isfinite(l[m]);
+      const float l = (((sm.red[0][ql][col] + sm.red[1][ql][col]) + sm.red[2][ql][col]) +
+                       sm.red[3][ql][col]) + b;
+      const float xn = sqrtf(((sm.xsq[0][ql] + sm.xsq[1][ql]) + sm.xsq[2][ql]) + sm.xsq[3][ql]);
+      sm.lgt[ql][col] = l;
+      sm.err[ql][col] = cerr * fmaf(xn, sqrtf(a.wsq[col]), fabsf(b)) + 1e-36f;
+      nonfinite |= !isfinite(l);
     }
-    // provisional top-k from the float32 logits (ties -> lower index)
-    uint32_t taken = 0;
-    int sel[kMaxM];
-    for (int r = 0; r < k; ++r) {
-      int best = -1;
-      for (int m = 0; m < M; ++m) {
-        if (taken & (1u << m)) continue;
-        if (best < 0 || l[m] > l[best]) best = m;
-      }
-      sel[r] = best;
-      taken |= 1u << best;
-    }
-    // certify: every rank r < min(k, M-1) beats every later candidate
-    bool certain = true;
-    uint32_t above = 0;
-    for (int r = 0; r < k && r < M - 1 && certain; ++r) {
-      const int am = sel[r];
-      above |= 1u << am;
-      for (int m = 0; m < M; ++m) {
-        if (above & (1u << m)) continue;
-        if (!(l[am] - l[m] > (e[am] + e[m]) * 1.001f)) {
-          certain = false;
-          break;
+    if (nonfinite) latch_status(a.status, GQE_ERR_NONFINITE);
+    __syncthreads();
+
+    // per (token, group): softmax, provisional top-k, certification
+    for (int q = tid; q < ntok * G; q += kRouteThreads) {
+      const int ql = q / G, g = q % G;
+      const float* l = &sm.lgt[ql][g * M];
+      const float* e = &sm.err[ql][g * M];
+      const int64_t row = static_cast<int64_t>(t0 + ql) * G + g;
+      float mx = l[0];
+      for (int m = 1; m < M; ++m) mx = fmaxf(mx, l[m]);
+      float s = 0.f;
+      for (int m = 0; m < M; ++m) s += expf(l[m] - mx);
+      float* prow = a.p + row * M;
+      for (int m = 0; m < M; ++m) prow[m] = expf(l[m] - mx) / s;
+      int32_t* irow = a.topk_idx + row * k;
+      uint32_t taken = 0;
+      bool certain = true;
+      float den = 0.f;
+      for (int r = 0; r < k; ++r) {
+        int best = -1;
+        for (int m = 0; m < M; ++m) {
+          if (taken & (1u << m)) continue;
+          if (best < 0 || l[m] > l[best]) best = m;
         }
+        taken |= 1u << best;
+        irow[r] = best;
+        den += expf(l[best] - mx) / s;
+        // rank r must beat every later candidate by more than both bounds
+        if (r < M - 1)
+          for (int m = 0; m < M; ++m)
+            if (!(taken & (1u << m)) && !(l[best] - l[m] > (e[best] + e[m]) * 1.001f))
+              certain = false;
+      }
+      float* wrow = a.w + row * k;
+      for (int r = 0; r < k; ++r)
+        wrow[r] = (k == 1) ? 1.0f : (expf(l[irow[r]] - mx) / s) / den;
+      if (!certain) sm.flags[atomicAdd(&sm.nflag, 1)] = q;
+    }
+    __syncthreads();
+    const int nf = sm.nflag;
+    if (nf > 0) {  // undecided pairs: exact ranks, one warp per pair
+      if (tid == 0) atomicAdd(a.fix_count, nf);
+      for (int f = warp; f < nf; f += kRouteWarps) {
+        const int q = sm.flags[f];
+        exact_rank_pair(a, t0 + q / G, q % G, sm.sel[warp]);
       }
     }
-    if (!certain) {
-      const int slot = atomicAdd(a.fix_count, 1);
-      a.fix_list[slot] = static_cast<int32_t>(tG + g);
-    }
-    // softmax over the group's M experts
-    float mx = l[0];
-    for (int m = 1; m < M; ++m) mx = fmaxf(mx, l[m]);
-    float pe[kMaxM], s = 0.f;
-    for (int m = 0; m < M; ++m) {
-      pe[m] = expf(l[m] - mx);
-      s += pe[m];
-    }
-    float* prow = a.p + (tG + g) * M;
-    for (int m = 0; m < M; ++m) prow[m] = pe[m] / s;
-    int32_t* irow = a.topk_idx + (tG + g) * k;
-    float* wrow = a.w + (tG + g) * k;
-    float den = 0.f;
-    for (int j = 0; j < k; ++j) den += pe[sel[j]] / s;
-    for (int j = 0; j < k; ++j) {
-      irow[j] = sel[j];
-      wrow[j] = (k == 1) ? 1.0f : (pe[sel[j]] / s) / den;
-    }
+    __syncthreads();
   }
-  if (nonfinite) latch_status(a.status, GQE_ERR_NONFINITE);
 }
 
 // ------------------------------------------------------------------------
@@ -165,8 +288,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
 constexpr int kLimbs = 18;
 constexpr int kExpBias = 266;
 
-struct Exact {
-  long long v[kLimbs];
+struct Exact {            // normalised: v[0..16] in [0, 2^32), top signed
+  uint32_t v[kLimbs - 1];
+  int32_t top;
 };
 
 __device__ __forceinline__ void bf16_decompose(uint32_t b, int& sign, int& mant, int& ex) {
@@ -188,77 +312,203 @@ __device__ __forceinline__ void limbs_add(long long* acc, long long mant, int po
   acc[L + 1] += v >> 32;
 }
 
+// Terms of one exact logit: products x_j * w_jm (16-bit integer times
+// 2^(pos-266)) and the bias (24-bit integer).  Returns 0 for a zero term.
+struct Term {
+  long long mant;
+  int pos;
+};
+
+__device__ __forceinline__ Term product_term(uint32_t xb, uint32_t wb) {
+  int sx, mx, ex, sw, mw, ew;
+  bf16_decompose(xb, sx, mx, ex);
+  bf16_decompose(wb, sw, mw, ew);
+  long long prod = static_cast<long long>(mx) * mw;
+  if (sx ^ sw) prod = -prod;
+  return Term{prod, ex + ew + kExpBias};
+}
+
+__device__ __forceinline__ Term bias_term(float bias) {
+  const uint32_t bb = __float_as_uint(bias);
+  const int E = (bb >> 23) & 0xFF;
+  long long mant = (E == 0) ? (bb & 0x7FFFFF) : ((bb & 0x7FFFFF) | 0x800000);
+  if (bb >> 31) mant = -mant;
+  return Term{mant, ((E == 0) ? -149 : E - 150) + kExpBias};
+}
+
+constexpr int kWin = 7;  // register window of 32-bit limbs
+
 __device__ void exact_logit(const RouteArgs& a, int t, int g, int m, Exact& out, bool& bad) {
   const int lane = threadIdx.x & 31;
-  long long acc[kLimbs];
-#pragma unroll
-  for (int i = 0; i < kLimbs; ++i) acc[i] = 0;
   const uint16_t* xr = a.x + static_cast<int64_t>(t) * a.dm;
+  const uint16_t* wr = a.Wr + static_cast<int64_t>(g) * a.dm * a.M + m;
+  const bool has_bias = (lane == 0) && a.bias;
+  // pass 1: range of bit positions occupied by the terms
+  int pmin = 1 << 30, tmax = -(1 << 30);
+#pragma unroll 4
   for (int j = lane; j < a.dm; j += 32) {
-    const uint32_t xb = xr[j];
-    const uint32_t wb = a.Wr[(static_cast<int64_t>(g) * a.dm + j) * a.M + m];
+    const uint32_t xb = xr[j], wb = wr[static_cast<int64_t>(j) * a.M];
     if (((xb >> 7) & 0xFF) == 0xFF || ((wb >> 7) & 0xFF) == 0xFF) {
       bad = true;
       continue;
     }
-    int sx, mx, ex, sw, mw, ew;
-    bf16_decompose(xb, sx, mx, ex);
-    bf16_decompose(wb, sw, mw, ew);
-    long long prod = static_cast<long long>(mx) * mw;
-    if (sx ^ sw) prod = -prod;
-    if (prod != 0) limbs_add(acc, prod, ex + ew + kExpBias);
+    const Term tm = product_term(xb, wb);
+    if (tm.mant != 0) {
+      pmin = min(pmin, tm.pos);
+      tmax = max(tmax, tm.pos + 16);
+    }
   }
-  if (lane == 0 && a.bias) {
-    const uint32_t bb = __float_as_uint(a.bias[g * a.M + m]);
-    const int E = (bb >> 23) & 0xFF;
-    if (E == 0xFF) {
-      bad = true;
-    } else {
-      long long mant = (E == 0) ? (bb & 0x7FFFFF) : ((bb & 0x7FFFFF) | 0x800000);
-      const int e = (E == 0) ? -149 : E - 150;
-      if (bb >> 31) mant = -mant;
-      if (mant != 0) limbs_add(acc, mant, e + kExpBias);
+  Term bt{0, 0};
+  if (has_bias) {
+    const float bv = a.bias[g * a.M + m];
+    if (!isfinite(bv)) bad = true;
+    else bt = bias_term(bv);
+    if (bt.mant != 0) {
+      pmin = min(pmin, bt.pos);
+      tmax = max(tmax, bt.pos + 24);
     }
   }
 #pragma unroll
-  for (int i = 0; i < kLimbs; ++i) {
-    long long v = acc[i];
+  for (int off = 16; off > 0; off >>= 1) {
+    pmin = min(pmin, __shfl_xor_sync(0xFFFFFFFFu, pmin, off));
+    tmax = max(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, off));
+  }
+  long long full[kLimbs];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-    acc[i] = v;
+  for (int i = 0; i < kLimbs; ++i) full[i] = 0;
+  if (tmax >= pmin) {  // at least one non-zero term
+    const int base = pmin >> 5;
+    // at most d_model + 1 terms: the sum stays below 2^(tmax + 13)
+    if (tmax + 14 - 32 * base <= 32 * (kWin - 1) - 1) {
+      // fast path: every term lands in limbs [base, base + kWin) held in registers
+      long long w[kWin];
+#pragma unroll
+      for (int i = 0; i < kWin; ++i) w[i] = 0;
+      auto add = [&](const Term& tm) {
+        const int L = (tm.pos >> 5) - base, o = tm.pos & 31;
+        const long long v = tm.mant * (1ll << o);
+        const long long lo = v & 0xFFFFFFFFll, hi = v >> 32;
+#pragma unroll
+        for (int i = 0; i < kWin; ++i) w[i] += (i == L ? lo : 0) + (i == L + 1 ? hi : 0);
+      };
+      for (int j = lane; j < a.dm; j += 32) {
+        const uint32_t xb = xr[j], wb = wr[static_cast<int64_t>(j) * a.M];
+        if (((xb >> 7) & 0xFF) == 0xFF || ((wb >> 7) & 0xFF) == 0xFF) continue;
+        const Term tm = product_term(xb, wb);
+        if (tm.mant != 0) add(tm);
+      }
+      if (bt.mant != 0) add(bt);
+#pragma unroll
+      for (int i = 0; i < kWin; ++i) {
+        long long v = w[i];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+        w[i] = v;
+      }
+      for (int i = 0; i < kWin && base + i < kLimbs; ++i) full[base + i] = w[i];
+    } else {
+      // wide exponent range: the full 18-limb accumulator
+      for (int j = lane; j < a.dm; j += 32) {
+        const uint32_t xb = xr[j], wb = wr[static_cast<int64_t>(j) * a.M];
+        if (((xb >> 7) & 0xFF) == 0xFF || ((wb >> 7) & 0xFF) == 0xFF) continue;
+        const Term tm = product_term(xb, wb);
+        if (tm.mant != 0) limbs_add(full, tm.mant, tm.pos);
+      }
+      if (bt.mant != 0) limbs_add(full, bt.mant, bt.pos);
+#pragma unroll
+      for (int i = 0; i < kLimbs; ++i) {
+        long long v = full[i];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+        full[i] = v;
+      }
+    }
   }
   // carry pass: limbs 0..16 into [0, 2^32), the top limb keeps the sign
 #pragma unroll
   for (int i = 0; i < kLimbs - 1; ++i) {
-    const long long c = acc[i] >> 32;  // floor division by 2^32
-    acc[i] -= c * 4294967296ll;
-    acc[i + 1] += c;
+    const long long c = full[i] >> 32;  // floor division by 2^32
+    full[i] -= c * 4294967296ll;
+    full[i + 1] += c;
   }
 #pragma unroll
-  for (int i = 0; i < kLimbs; ++i) out.v[i] = acc[i];
+  for (int i = 0; i < kLimbs - 1; ++i) out.v[i] = static_cast<uint32_t>(full[i]);
+  out.top = static_cast<int32_t>(full[kLimbs - 1]);  // |sum| < 2^540: top limb is tiny
 }
 
 // -1, 0, +1 for a < b, a == b, a > b
 __device__ __forceinline__ int exact_cmp(const Exact& a, const Exact& b) {
-  if (a.v[kLimbs - 1] != b.v[kLimbs - 1]) return a.v[kLimbs - 1] < b.v[kLimbs - 1] ? -1 : 1;
+  if (a.top != b.top) return a.top < b.top ? -1 : 1;
   for (int i = kLimbs - 2; i >= 0; --i)
     if (a.v[i] != b.v[i]) return a.v[i] < b.v[i] ? -1 : 1;
   return 0;
 }
 
-constexpr int kFixWarps = 4;
+// Float64 logits of one (token, group) pair, with a rigorous bound: every
+// bf16*bf16 product is exact in float64; each lane sums its ceil(dm/32)
+// products in order, the warp adds the 32 partial sums in a 5-level tree,
+// and the bias is added last, so |l64 - l| <= (ceil(dm/32) + 7) 2^-53 A with
+// A = sum |x_j w_j| + |bias| (bound doubled for the rounding of A itself).
+__device__ void logit64(const RouteArgs& a, int t, int g, int m, double& l, double& err) {
+  const int lane = threadIdx.x & 31;
+  const uint16_t* xr = a.x + static_cast<int64_t>(t) * a.dm;
+  const uint16_t* wr = a.Wr + static_cast<int64_t>(g) * a.dm * a.M + m;
+  double s = 0.0, A = 0.0;
+#pragma unroll 8
+  for (int j = lane; j < a.dm; j += 32) {
+    const double p = static_cast<double>(bf16_bits_to_float(xr[j])) *
+                     static_cast<double>(bf16_bits_to_float(wr[static_cast<int64_t>(j) * a.M]));
+    s += p;
+    A += fabs(p);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
+    A += __shfl_xor_sync(0xFFFFFFFFu, A, off);
+  }
+  if (a.bias) {
+    const double b = a.bias[g * a.M + m];
+    s += b;
+    A += fabs(b);
+  }
+  l = s;
+  err = 2.0 * ((a.dm + 31) / 32 + 7) * 1.1102230246251565e-16 * A;
+}
 
-__global__ void __launch_bounds__(32 * kFixWarps) route_fixup_kernel(const RouteArgs a) {
-  __shared__ Exact ex[kFixWarps][kMaxM];
-  __shared__ int sel[kFixWarps][kMaxM];
+// Exact top-k of one (token, group) pair by one warp: exact logits of the
+// group's M experts, ranks by (logit desc, index asc), then w from p.  The
+// float64 pass decides every pair whose gaps exceed its bound; only pairs
+// still undecided (in practice exact ties) take the fixed-point path.
+__device__ void exact_rank_pair(const RouteArgs& a, int t, int g, int* sel) {
+  __shared__ Exact ex[kRouteWarps][kMaxM];
+  __shared__ double l64[kRouteWarps][kMaxM], e64[kRouteWarps][kMaxM];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = gridDim.x * kFixWarps;
-  const int count = *reinterpret_cast<volatile int32_t*>(a.fix_count);
   const int M = a.M, k = a.k;
-  for (int f = blockIdx.x * kFixWarps + warp; f < count; f += nwarps) {
-    const int pair = a.fix_list[f];
-    const int t = pair / a.G, g = pair % a.G;
-    bool bad = false;
+  bool bad = false;
+  for (int m = 0; m < M; ++m) {
+    double l, e;
+    logit64(a, t, g, m, l, e);
+    if (lane == 0) {
+      l64[warp][m] = l;
+      e64[warp][m] = e;
+    }
+  }
+  __syncwarp();
+  // ranks from the float64 logits (ties -> lower index), certified when every
+  // compared pair is separated by more than the two bounds
+  bool certain = true;
+  int rank = 0;
+  if (lane < M) {
+    const double la = l64[warp][lane], ea = e64[warp][lane];
+    for (int b = 0; b < M; ++b) {
+      if (b == lane) continue;
+      const double lb = l64[warp][b], eb = e64[warp][b];
+      if (lb > la || (lb == la && b < lane)) ++rank;
+      if (!(fabs(la - lb) > (ea + eb) * 1.0000001)) certain = false;
+    }
+  }
+  certain = __all_sync(0xFFFFFFFFu, certain);
+  if (!certain) {
     for (int m = 0; m < M; ++m) {
       Exact e;
       exact_logit(a, t, g, m, e, bad);
@@ -267,46 +517,64 @@ __global__ void __launch_bounds__(32 * kFixWarps) route_fixup_kernel(const Route
     bad = __any_sync(0xFFFFFFFFu, bad);
     __syncwarp();
     if (lane < M) {
-      int rank = 0;
+      rank = 0;
       for (int b = 0; b < M; ++b) {
         if (b == lane) continue;
         const int c = exact_cmp(ex[warp][b], ex[warp][lane]);
         if (c > 0 || (c == 0 && b < lane)) ++rank;
       }
-      if (rank < k) sel[warp][rank] = lane;
     }
-    __syncwarp();
-    if (lane == 0) {
-      if (bad) latch_status(a.status, GQE_ERR_NONFINITE);
-      const int64_t row = static_cast<int64_t>(t) * a.G + g;
-      const float* prow = a.p + row * M;
-      float den = 0.f;
-      for (int j = 0; j < k; ++j) den += prow[sel[warp][j]];
-      for (int j = 0; j < k; ++j) {
-        a.topk_idx[row * k + j] = sel[warp][j];
-        a.w[row * k + j] = (k == 1) ? 1.0f : prow[sel[warp][j]] / den;
-      }
-    }
-    __syncwarp();
   }
+  if (lane < M && rank < k) sel[rank] = lane;
+  __syncwarp();
+  if (lane == 0) {
+    if (bad) latch_status(a.status, GQE_ERR_NONFINITE);
+    const int64_t row = static_cast<int64_t>(t) * a.G + g;
+    const float* prow = a.p + row * M;
+    float den = 0.f;
+    for (int j = 0; j < k; ++j) den += prow[sel[j]];
+    for (int j = 0; j < k; ++j) {
+      a.topk_idx[row * k + j] = sel[j];
+      a.w[row * k + j] = (k == 1) ? 1.0f : prow[sel[j]] / den;
+    }
+  }
+  __syncwarp();
+}
+
+template <int GM>
+cudaError_t launch_route_gm(const RouteArgs& a, cudaStream_t st) {
+  static int configured = -1;
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int smem = static_cast<int>(sizeof(RouteSmem<GM>));
+  if (configured != dev) {
+    e = cudaFuncSetAttribute(route_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = dev;
+  }
+  e = cudaMemsetAsync(a.wsq, 0, sizeof(float) * GM, st);
+  if (e != cudaSuccess) return e;
+  route_prep_kernel<GM><<<(a.dm + 31) / 32, 32 * GM, 0, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int ntiles = (a.T + RouteShape<GM>::kTok - 1) / RouteShape<GM>::kTok;
+  const int grid = ntiles < 4 * sms ? ntiles : 4 * sms;
+  route_kernel<GM><<<grid, kRouteThreads, smem, st>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
-  const int GM = a.G * a.M;
-  const dim3 grid((a.T + kRouteThreads - 1) / kRouteThreads);
-  switch (GM) {
-    case 4: route_kernel<4><<<grid, kRouteThreads, 0, st>>>(a); break;
-    case 8: route_kernel<8><<<grid, kRouteThreads, 0, st>>>(a); break;
-    case 16: route_kernel<16><<<grid, kRouteThreads, 0, st>>>(a); break;
-    case 32: route_kernel<32><<<grid, kRouteThreads, 0, st>>>(a); break;
+  switch (a.G * a.M) {
+    case 4: return launch_route_gm<4>(a, st);
+    case 8: return launch_route_gm<8>(a, st);
+    case 16: return launch_route_gm<16>(a, st);
+    case 32: return launch_route_gm<32>(a, st);
     default: return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  route_fixup_kernel<<<148, 32 * kFixWarps, 0, st>>>(a);
-  return cudaGetLastError();
 }
 
 }  // namespace gqe
