@@ -134,6 +134,34 @@ gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void
                                  void* stream);
 
 /*
+ * gqe_attention_prefill_static - gqe_attention_prefill for callers that
+ * cannot allocate device memory.  (Not a step of the method: the sources
+ * have no counterpart; it only changes where the scratch memory lives.)
+ *
+ * Some callers cannot give the library a workspace: for instance a plugin
+ * whose host framework owns every device allocation, or a loop that must
+ * not pay the device-wide synchronisation of cudaMalloc.  This call takes
+ * the same arguments as gqe_attention_prefill minus `ws`/`ws_bytes`, writes
+ * the same outputs, and allocates nothing: its scratch is one 64 MiB device
+ * array compiled into the library, present on every GPU that loads it until
+ * the process exits.
+ *  - The first call on a device looks up that array's device address (and
+ *    zeroes its header) with the device current; make that first call before
+ *    any stream capture.
+ *  - Shapes whose scratch (V in fp16, token lists, work list) exceeds
+ *    64 MiB return GQE_ERR_WORKSPACE without launching anything.
+ *  - All calls on a device share the one array and it keeps the previous
+ *    call's contents (the call clears what must start at zero).  Calls that
+ *    overlap on the GPU - different streams, or different host threads -
+ *    race on it and give wrong results; order them.
+ *  - Device-side errors are latched in the array and are not reported.
+ */
+gqe_status gqe_attention_prefill_static(const gqe_dims* dims, const void* Q, const void* Qs,
+                                        const void* K, const void* V, const int32_t* topk_idx,
+                                        const float* w, void* O_sel, void* o_bar, void* s_out,
+                                        int64_t out_row_stride, void* stream);
+
+/*
  * gqe_dense_gqa_prefill - the all-active GQA baseline ("16 heads all
  * active", review §四): every query head h attends KV head floor(h/M).
  *  Q device bf16 [B, S, N, d]; K, V device bf16 [B, S, G, d]

@@ -17,6 +17,7 @@ EXPORTS = (
     "gqe_workspace_size", "gqe_route", "gqe_bucket", "gqe_attention_prefill",
     "gqe_dense_gqa_prefill", "gqe_get_device_status", "gqe_kv_cache_bytes",
     "gqe_status_string", "gqe_selftest_bounded_wait", "gqe_set_profile_events",
+    "gqe_attention_prefill_static",
 )
 
 STATUS = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED", 3: "GQE_ERR_CUDA",
@@ -52,6 +53,7 @@ def _load() -> ctypes.CDLL:
         "gqe_status_string": (ctypes.c_char_p, [I32]),
         "gqe_selftest_bounded_wait": (I32, [P, SZ, I32, P]),
         "gqe_set_profile_events": (None, [P, P]),
+        "gqe_attention_prefill_static": (I32, [S, P, P, P, P, P, P, P, P, P, I64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -136,3 +138,12 @@ def gqe_set_profile_events(begin=None, end=None):
     b = None if begin is None else ctypes.c_void_p(begin.cuda_event)
     e = None if end is None else ctypes.c_void_p(end.cuda_event)
     LIB.gqe_set_profile_events(b, e)
+
+
+def gqe_attention_prefill_static(dm, Q, Qs, K, V, topk_idx, w, O_sel, o_bar, s_out,
+                                 out_row_stride, stream=None, check=True):
+    """gqe_attention_prefill without a workspace (scratch in the library)."""
+    r = LIB.gqe_attention_prefill_static(ctypes.byref(dm), _ptr(Q), _ptr(Qs), _ptr(K), _ptr(V),
+                                         _ptr(topk_idx), _ptr(w), _ptr(O_sel), _ptr(o_bar),
+                                         _ptr(s_out), int(out_row_stride), _stream(stream))
+    return _check(r, "gqe_attention_prefill_static") if check else r
