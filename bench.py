@@ -38,6 +38,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_FLUSH_BYTES = 256 << 20
 
 
+def kernel_traffic(key):
+    """DRAM bytes per launch recorded by an ncu capture (profiles/traffic.json),
+    or None when the attention kernel's source changed since that capture."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[key]
+    except (OSError, ValueError, KeyError):
+        return None
+    h = hashlib.sha256()
+    for f in ("gqe_attn.cu", "gqe_device.cuh", "gqe_internal.h"):
+        with open(os.path.join(ROOT, "moe_routed_grouped_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return rec["dram_bytes"] if h.hexdigest()[:16] == rec["kernel_sha"] else None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -400,14 +415,18 @@ def main():
         "routed_over_dense": dense_tot_ms / tot_ms,
         "roofline": {"kernel": "attn_kernel<%d> (routed + shared head)" % w.d, "bound": "tensor",
                      "achieved": attn_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": attn_tf / peak_tf, "traffic": None,
+                     "frac": attn_tf / peak_tf,
+                     "traffic": kernel_traffic(f"attn_kernel<{w.d}>:routed:{w.name}"),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_source": f"{peak_src} bf16 dense (burst)",
                      "attention_kernel_ms": attn_ms,
                      "per_launch_flop": fl_r,
                      "flop_definition": "4*d per visible (query, key) pair, (G*k+1)*B*S*(S+1)/2 pairs"},
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * (6 + (1 if w.k > 1 else 0)),
+        # per routed step: route_prep, route, prep (bucket + V fp16 + sort), attention
+        # (+ combine when k > 1)
+        "gpu_launches": args.steps * (4 + (1 if w.k > 1 else 0)),
         "clocks": clocks.summary(res["t0"], res["t1"]),
     }
 
