@@ -309,7 +309,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      if (!wait(&bars[kBarSFull], j & 1)) { ok = false; break; }
+      // the lanes must agree: they go on to warp-collective tcgen05 instructions
+      if (!__all_sync(0xFFFFFFFFu, wait(&bars[kBarSFull], j & 1))) { ok = false; break; }
       tc_fence_after();
       uint32_t sv[4][32];
 #pragma unroll
@@ -349,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
       l *= factor;
       // P.V of the previous tile must be done before P and O are touched
       if (j > 0) {
-        if (!wait(&bars[kBarODone], (j - 1) & 1)) { ok = false; break; }
+        if (!__all_sync(0xFFFFFFFFu, wait(&bars[kBarODone], (j - 1) & 1))) { ok = false; break; }
         tc_fence_after();
       }
       // p = 2^(s * scale * log2e - m), packed to fp16 and written to TMEM

@@ -141,9 +141,14 @@ def route(x_bits: np.ndarray, Wr_bits: np.ndarray, bias: Optional[np.ndarray], k
     G, _, M = Wr_bits.shape
     if not 1 <= k <= M:
         raise ValueError("need 1 <= k <= M")
-    x = bf16_to_f64(x_bits).reshape(B * S, dm)
     Wr = bf16_to_f64(Wr_bits)
-    L, err = router_logits(x, Wr, bias)
+    xb = np.asarray(x_bits).reshape(B * S, dm)
+    # tokens are independent: evaluate them in blocks to bound memory
+    blk = 1 << 16
+    L = np.empty((B * S, G, M))
+    err = np.empty((B * S, G, M))
+    for t0 in range(0, B * S, blk):
+        L[t0:t0 + blk], err[t0:t0 + blk] = router_logits(bf16_to_f64(xb[t0:t0 + blk]), Wr, bias)
 
     # candidate order from the float64 estimate (stable: lower index first)
     order = np.argsort(-L, axis=-1, kind="stable")
@@ -160,7 +165,7 @@ def route(x_bits: np.ndarray, Wr_bits: np.ndarray, bias: Optional[np.ndarray], k
 
     unsure = np.argwhere(~certain)
     for t, g in unsure:
-        ordr = topk_exact_order(x[t], Wr[g], None if bias is None else bias[g])
+        ordr = topk_exact_order(bf16_to_f64(xb[t]), Wr[g], None if bias is None else bias[g])
         idx[t, g] = ordr[:k]
 
     # p = softmax over the group's M experts (float64)
@@ -206,7 +211,7 @@ def bucket(topk_idx: np.ndarray, M: int) -> Tuple[np.ndarray, np.ndarray]:
 # ---------------------------------------------------------------------------
 
 def causal_attention(q: np.ndarray, pos: np.ndarray, K: np.ndarray, V: np.ndarray,
-                     dtype=np.float64, row_chunk: int = 512) -> np.ndarray:
+                     dtype=np.float64, row_chunk: int = 0) -> np.ndarray:
     """Softmax attention of query rows at absolute positions ``pos``.
 
     o_r = sum_{t <= pos_r} softmax_t(q_r . K_t / sqrt(d)) V_t.
@@ -221,6 +226,8 @@ def causal_attention(q: np.ndarray, pos: np.ndarray, K: np.ndarray, V: np.ndarra
     R, d = q.shape
     out = np.empty((R, V.shape[1]), dtype=dtype)
     sc = dtype(_scale(d))
+    if row_chunk <= 0:  # about 2^25 scores per block
+        row_chunk = max(1, min(512, (1 << 25) // max(1, int(pos.max()) + 1)))
     for s in range(0, R, row_chunk):
         e = min(R, s + row_chunk)
         pm = int(pos[s:e].max())
