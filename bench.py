@@ -268,6 +268,24 @@ def run_reference(args, rank, world):
     return 0
 
 
+def reduce_max(values, dist, device=None):
+    """Element-wise max of per-rank values over all ranks (identity without a
+    process group).  Ranks are independent replicas; this is the only
+    cross-rank step of the benchmark."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(tokens_per_rank, steps, world, max_total_ms):
+    """Whole-job tokens/s: every rank processed `tokens_per_rank * steps`
+    tokens; the job took the slowest rank's device time."""
+    return world * tokens_per_rank * steps / (max_total_ms / 1e3)
+
+
 def config_of(w, world):
     return {"workload": w.name, "B": w.B, "S": w.S, "N": w.N, "G": w.G, "M": w.M, "k": w.k,
             "d": w.d, "d_model": w.d_model, "router_bias_expert0": w.bias0,
@@ -380,15 +398,12 @@ def main():
     dense_tot_ms = sum(res["dense_ms"])
     attn_ms = statistics.mean(res["routed_attn_ms"])
     dense_attn_ms = statistics.mean(res["dense_attn_ms"])
-    if dist is not None:
-        t = torch.tensor([tot_ms, dense_tot_ms, attn_ms, dense_attn_ms], device=device,
-                         dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms, dense_tot_ms, attn_ms, dense_attn_ms = t.tolist()
+    tot_ms, dense_tot_ms, attn_ms, dense_attn_ms = reduce_max(
+        [tot_ms, dense_tot_ms, attn_ms, dense_attn_ms], dist, device)
 
     tokens = w.B * w.S
-    value = world * tokens * args.steps / (tot_ms / 1e3)
-    dense_value = world * tokens * args.steps / (dense_tot_ms / 1e3)
+    value = job_throughput(tokens, args.steps, world, tot_ms)
+    dense_value = job_throughput(tokens, args.steps, world, dense_tot_ms)
     ms_step = tot_ms / args.steps
     fl_r, fl_d = w.useful_flop_routed(), w.useful_flop_dense()
     useful_tf = fl_r / (ms_step / 1e3) / 1e12

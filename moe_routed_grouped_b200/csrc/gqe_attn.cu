@@ -51,7 +51,7 @@ constexpr int kThreads = 192;
 // Of every 8 column pairs, this many are exponentiated by a polynomial on the
 // FMA pipe; the rest use the MUFU ex2 unit (16 lanes/clock/SM), which would
 // otherwise bound d = 64 attention at about half the tensor-core rate.
-constexpr int kPolyPairs = 3;
+constexpr int kPolyPairs = 2;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 
