@@ -200,6 +200,16 @@ gqe_status gqe_selftest_bounded_wait(void* ws, size_t ws_bytes, int32_t limit_us
  * not thread-safe: meant for benchmarks. */
 void gqe_set_profile_events(void* begin, void* end);
 
+/* Kernel choice for d = 64 (tuning; no counterpart on the pages).  The
+ * attention calls use a pair kernel - two 128-row query tiles of one KV head
+ * per CTA, sharing every K/V tile load - once the KV working set of the call,
+ * B*S*G*d*4 bytes (K bf16 + V fp16), reaches `kv_bytes`; below it they use one
+ * tile per CTA and two CTAs per SM, which is faster while K and V stay in L2.
+ * Default 96 MiB.  0 selects the pair kernel always, a negative value never.
+ * Results agree within rounding either way.  Process-wide setting, read at
+ * each call; returns the previous value. */
+int64_t gqe_set_pair_threshold(int64_t kv_bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -17,7 +17,7 @@ EXPORTS = (
     "gqe_workspace_size", "gqe_route", "gqe_bucket", "gqe_attention_prefill",
     "gqe_dense_gqa_prefill", "gqe_get_device_status", "gqe_kv_cache_bytes",
     "gqe_status_string", "gqe_selftest_bounded_wait", "gqe_set_profile_events",
-    "gqe_attention_prefill_static",
+    "gqe_attention_prefill_static", "gqe_set_pair_threshold",
 )
 
 STATUS = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED", 3: "GQE_ERR_CUDA",
@@ -54,6 +54,7 @@ def _load() -> ctypes.CDLL:
         "gqe_selftest_bounded_wait": (I32, [P, SZ, I32, P]),
         "gqe_set_profile_events": (None, [P, P]),
         "gqe_attention_prefill_static": (I32, [S, P, P, P, P, P, P, P, P, P, I64, P]),
+        "gqe_set_pair_threshold": (I64, [I64]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -138,6 +139,12 @@ def gqe_set_profile_events(begin=None, end=None):
     b = None if begin is None else ctypes.c_void_p(begin.cuda_event)
     e = None if end is None else ctypes.c_void_p(end.cuda_event)
     LIB.gqe_set_profile_events(b, e)
+
+
+def gqe_set_pair_threshold(kv_bytes):
+    """Working-set size (bytes) from which d = 64 attention uses the pair
+    kernel (0: always, negative: never); returns the previous value."""
+    return int(LIB.gqe_set_pair_threshold(int(kv_bytes)))
 
 
 def gqe_attention_prefill_static(dm, Q, Qs, K, V, topk_idx, w, O_sel, o_bar, s_out,

@@ -104,10 +104,10 @@ gqe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GQE_OK : GQE_ERR
 
 cudaEvent_t g_prof_begin = nullptr, g_prof_end = nullptr;
 
-cudaError_t timed_attention(const AttnArgs& a, int64_t grid, cudaStream_t s) {
+cudaError_t timed_attention(const AttnArgs& a, int64_t n_list, cudaStream_t s) {
   const bool prof = g_prof_begin && g_prof_end;
   if (prof && cudaEventRecord(g_prof_begin, s) != cudaSuccess) return cudaErrorUnknown;
-  cudaError_t e = launch_attention(a, grid, s);
+  cudaError_t e = launch_attention(a, n_list, s);
   if (e == cudaSuccess && prof) e = cudaEventRecord(g_prof_end, s);
   return e;
 }
@@ -224,8 +224,11 @@ gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void
 
   ConvertArgs cv{static_cast<const uint16_t*>(V), reinterpret_cast<uint16_t*>(wb + L.v16),
                  B * S * G * d, reinterpret_cast<int*>(wb + L.status)};
-  const BucketArgs ba = bucket_args(dims, topk_idx, reinterpret_cast<int32_t*>(wb + L.bucket_off),
-                                    reinterpret_cast<int32_t*>(wb + L.bucket_tok), wb, L);
+  // one decision for the call: the work-list format and the kernel follow it
+  const bool pair = pair_kernel_for(*dims);
+  BucketArgs ba = bucket_args(dims, topk_idx, reinterpret_cast<int32_t*>(wb + L.bucket_off),
+                              reinterpret_cast<int32_t*>(wb + L.bucket_tok), wb, L);
+  ba.pairs = pair ? 1 : 0;
   cudaError_t e = launch_prep(ba, &cv, true, s);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
 
@@ -247,6 +250,7 @@ gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void
   a.s_out = s_out;
   a.out_row_stride = out_row_stride;
   a.dense = 0;
+  a.pair = pair ? 1 : 0;
   e = timed_attention(a, L.n_raw_tiles, s);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
 
@@ -284,9 +288,10 @@ gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void
   a.Q = static_cast<const uint16_t*>(Q);
   a.O_dense = O;
   a.dense = 1;
-  const int64_t nq = (S + kTileM - 1) / kTileM;
-  return from_cuda(timed_attention(a, B * dims->N * nq, s));
+  return from_cuda(timed_attention(a, 0, s));
 }
+
+int64_t gqe_set_pair_threshold(int64_t kv_bytes) { return set_pair_threshold(kv_bytes); }
 
 gqe_status gqe_get_device_status(void* ws, int32_t clear, void* stream) {
   if (!aligned16(ws)) return GQE_ERR_INVALID_ARG;

@@ -24,6 +24,8 @@
 // TMEM).  Q.K^T of tile j+1 runs while the softmax of tile j is computed.
 // The running max is only moved when it grows by more than 2^8, so O is
 // rescaled rarely; the final division by the row sum makes this exact.
+#include <atomic>
+
 #include "gqe_device.cuh"
 
 namespace gqe {
@@ -132,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
   } else {
     if (static_cast<int>(blockIdx.x) >= *a.tile_count) return;
     const TileDesc td = a.tiles[blockIdx.x];
+    if (td.nkv == 0) return;  // empty second half of a pair
     kind = td.code >> 24;
     const int id = td.code & 0xFFFFFF;
     if (kind == kRouted) {
@@ -448,6 +451,425 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
   }
 }
 
+// ---------------------------------------------------------------------------
+// d = 64, long sequences: the pair kernel.  One CTA (one per SM: it takes
+// all 512 TMEM columns) computes TWO 128-row tiles that read the same KV
+// head: two expert buckets of one (batch, group) or two query tiles of the
+// shared head.  Each K/V tile is loaded once for both, which halves the K/V
+// traffic.  That matters once K and V
+// no longer fit in L2: CTAs that start at different times sweep the KV
+// sequence at different offsets, so each tile read by attn_kernel comes from
+// DRAM (at S = 1M the launch is bound by HBM bandwidth).  While K and V fit
+// in L2 attn_kernel is faster (two independent CTAs per SM).  Dense calls
+// keep attn_kernel: their query-tile-major order already lets the CTAs that
+// run together share K/V tiles in L2.
+// Warp roles (352 threads):
+//   warps 0-3 / 4-7  softmax + epilogue of tile 0 / tile 1 (thread = row)
+//   warp 8           producer: Q of both tiles, then K/V via TMA (3 stages)
+//   warps 9 / 10     tcgen05.mma issuer of tile 0 / tile 1 (warp 9 owns TMEM)
+// A K/V stage is refilled once both issuers are done with it, so the two
+// tiles run independently within the depth of the stage ring.
+// TMEM: tile s at column 256*s: S (128 fp32), P (128 fp16 = 64), O (64).
+struct PairCfg {
+  static constexpr int D = 64;
+  static constexpr int kStages = 3;
+  static constexpr int kAtom = kTileM * 128;
+  static constexpr int kQBytes = kTileM * D * 2;
+  static constexpr int kKVBytes = kTileN * D * 2;
+  static constexpr int kSmemQ = 0;  // two Q tiles
+  static constexpr int kSmemK = 2 * kQBytes;
+  static constexpr int kSmemV = kSmemK + kStages * kKVBytes;
+  static constexpr int kSmemBar = kSmemV + kStages * kKVBytes;
+  static constexpr int kSmemBytes = kSmemBar + 256 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t kTmemSlot = 256, kTmemS = 0, kTmemP = 128, kTmemO = 192;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kIdescQK = make_idesc_f16(kTileM, kTileN, /*bf16*/ 1, 0, 0);
+  static constexpr uint32_t kIdescPV = make_idesc_f16(kTileM, D, /*f16*/ 0, 0, /*MN*/ 1);
+};
+constexpr int kPairThreads = 352;
+constexpr int kPairProducerWarp = 8;
+constexpr int kPairMmaWarp = 9;
+
+enum {
+  kPbQFull = 0,    // +tile
+  kPbKFull = 2,    // +stage
+  kPbKEmpty = 5,   // +stage
+  kPbVFull = 8,    // +stage
+  kPbVEmpty = 11,  // +stage
+  kPbSFull = 14,   // +tile
+  kPbSFree = 16,   // +tile
+  kPbPFull = 18,   // +tile
+  kPbODone = 20,   // +tile
+  kPbSpare = 22,   // +tile
+  kPbNum = 24
+};
+
+struct Slot {
+  int kind, b, h, g, m, row0, nrows, nkv, bstart;
+};
+
+__device__ __forceinline__ Slot decode_tile(const TileDesc& td, const AttnArgs& a) {
+  Slot t{};
+  t.nkv = td.nkv;
+  if (td.nkv == 0) return t;
+  t.kind = td.code >> 24;
+  const int id = td.code & 0xFFFFFF;
+  if (t.kind == kRouted) {
+    t.b = id / (a.G * a.M);
+    t.g = (id / a.M) % a.G;
+    t.m = id % a.M;
+    t.h = t.g * a.M + t.m;
+    t.bstart = a.bucket_off[id];
+  } else {
+    t.b = id;
+    t.g = 0;  // the shared head reads KV head 0
+  }
+  t.row0 = td.row0;
+  t.nrows = td.nrows;
+  return t;
+}
+
+__global__ void __launch_bounds__(kPairThreads, 1)
+    attn_pair_kernel(const __grid_constant__ AttnArgs a) {
+  using C = PairCfg;
+  constexpr int D = C::D;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.S, N = a.N, G = a.G;
+
+  // ---------------------------------------------------------- work item
+  Slot sl[2];
+  {
+    if (2 * static_cast<int>(blockIdx.x) >= *a.tile_count) return;
+    sl[0] = decode_tile(a.tiles[2 * blockIdx.x], a);
+    sl[1] = decode_tile(a.tiles[2 * blockIdx.x + 1], a);
+    if (sl[0].nkv == 0) return;
+    if (sl[1].nkv > 0 && (sl[1].b != sl[0].b || sl[1].g != sl[0].g || sl[1].nkv > sl[0].nkv)) {
+      // not a valid pair (the scheduler writes none): refuse the second tile
+      if (threadIdx.x == 0) latch_status(a.status, GQE_ERR_CUDA);
+      sl[1].nkv = 0;
+    }
+  }
+  const int b = sl[0].b, g = sl[0].g, nkv0 = sl[0].nkv;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kPbNum);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kPbNum + 1);
+  const Waiter wait{abort_flag, a.status, a.wait_limit_ns};
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[kPbQFull + s], 1);
+      mbar_init(&bars[kPbSFull + s], 1);
+      mbar_init(&bars[kPbSFree + s], 4);
+      mbar_init(&bars[kPbPFull + s], 4);
+      mbar_init(&bars[kPbODone + s], 1);
+    }
+#pragma unroll
+    for (int st = 0; st < C::kStages; ++st) {
+      mbar_init(&bars[kPbKFull + st], 1);
+      mbar_init(&bars[kPbKEmpty + st], 2);
+      mbar_init(&bars[kPbVFull + st], 1);
+      mbar_init(&bars[kPbVEmpty + st], 2);
+    }
+    mbar_init(&bars[kPbSpare], 1);
+    mbar_init(&bars[kPbSpare + 1], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kPairMmaWarp) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kPairProducerWarp && lane == 0) {
+    tma_prefetch_desc(&a.tmK);
+    tma_prefetch_desc(&a.tmV);
+    tma_prefetch_desc(&a.tmQs);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+
+  if (warp == kPairProducerWarp) {
+    // ------------------------------------------------------ producer
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const Slot t = sl[s];
+      if (t.nkv == 0) continue;
+      uint8_t* sQ = smem + C::kSmemQ + s * C::kQBytes;
+      if (t.kind == kRouted) {
+        // gather the bucket's query rows in the 128-byte swizzle of the UMMA
+        // descriptor (16-byte chunk c of row r at c ^ (r & 7))
+        for (int rr = 0; rr < kTileM / 32; ++rr) {
+          const int r = lane + 32 * rr;
+          const bool ok = r < t.nrows;
+          const int tok = ok ? a.bucket_tok[t.bstart + t.row0 + r] : 0;
+          const uint16_t* src = a.Q + ((static_cast<int64_t>(t.b) * S + tok) * N + t.h) * D;
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c)
+            cp_async_16(sQ + r * 128 + ((c ^ (r & 7)) << 4), src + c * 8, ok ? 16u : 0u);
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kPbQFull + s]);
+      } else if (lane == 0) {
+        mbar_arrive_expect_tx(&bars[kPbQFull + s], C::kQBytes);
+        tma_load_3d(sQ, &a.tmQs, &bars[kPbQFull + s], 0, t.row0, t.b);
+      }
+    }
+    if (lane == 0) {
+      int nk = 0, nv = 0;  // K and V loads issued
+      for (int j = 0; j < nkv0; ++j) {
+        const int st = j % C::kStages;
+        const uint32_t round = static_cast<uint32_t>(j / C::kStages);
+        if (round > 0 && !wait(&bars[kPbKEmpty + st], (round - 1) & 1)) break;
+        mbar_arrive_expect_tx(&bars[kPbKFull + st], C::kKVBytes);
+        tma_load_4d(smem + C::kSmemK + st * C::kKVBytes, &a.tmK, &bars[kPbKFull + st], 0, g,
+                    j * kTileN, b);
+        ++nk;
+        if (round > 0 && !wait(&bars[kPbVEmpty + st], (round - 1) & 1)) break;
+        mbar_arrive_expect_tx(&bars[kPbVFull + st], C::kKVBytes);
+        tma_load_4d(smem + C::kSmemV + st * C::kKVBytes, &a.tmV, &bars[kPbVFull + st], 0, g,
+                    j * kTileN, b);
+        ++nv;
+      }
+      if (*abort_flag) {
+        // let the copies still in flight land before the CTA exits
+        for (int s = 0; s < 2; ++s)
+          if (sl[s].nkv > 0 && sl[s].kind != kRouted)
+            mbar_wait(&bars[kPbQFull + s], 0, nullptr, a.status, a.wait_limit_ns);
+        for (int q = max(0, nk - C::kStages); q < nk; ++q)
+          mbar_wait(&bars[kPbKFull + q % C::kStages], (q / C::kStages) & 1, nullptr, a.status,
+                    a.wait_limit_ns);
+        for (int q = max(0, nv - C::kStages); q < nv; ++q)
+          mbar_wait(&bars[kPbVFull + q % C::kStages], (q / C::kStages) & 1, nullptr, a.status,
+                    a.wait_limit_ns);
+      }
+    }
+  } else if (warp == kPairMmaWarp || warp == kPairMmaWarp + 1) {
+    // ------------------------------------------------------ MMA issuers
+    // one thread per tile: S_s = Q_s K_j^T, then O_s += P_s V_{j-1}.  Each K/V
+    // stage is released when both tiles are done with it; the shorter tile
+    // releases the longer one's remaining stages as they arrive.
+    const int s = warp - kPairMmaWarp;
+    const int nk = sl[s].nkv;
+    if (lane == 0) {
+      const uint32_t tS = tbase + s * C::kTmemSlot + C::kTmemS;
+      const uint32_t tP = tbase + s * C::kTmemSlot + C::kTmemP;
+      const uint32_t tO = tbase + s * C::kTmemSlot + C::kTmemO;
+      const uint32_t qaddr = smem_u32(smem + C::kSmemQ) + s * C::kQBytes;
+      auto issue_pv = [&](int jj) -> bool {
+        const int st = jj % C::kStages;
+        if (!wait(&bars[kPbVFull + st], (jj / C::kStages) & 1)) return false;
+        if (!wait(&bars[kPbPFull + s], jj & 1)) return false;
+        tc_fence_after();
+        const uint32_t vaddr = smem_u32(smem + C::kSmemV + st * C::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk)
+          umma_ts(tO, tP + kk * 8, make_sdesc_sw128(vaddr + kk * 2048, C::kAtom, 1024),
+                  C::kIdescPV, (jj > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&bars[kPbODone + s]);
+        tc_commit(&bars[kPbVEmpty + st]);
+        return true;
+      };
+      bool ok = nk == 0 || wait(&bars[kPbQFull + s], 0);
+      tc_fence_after();
+      for (int j = 0; ok && j < nk; ++j) {
+        const int st = j % C::kStages;
+        if (!wait(&bars[kPbKFull + st], (j / C::kStages) & 1)) { ok = false; break; }
+        if (j > 0 && !wait(&bars[kPbSFree + s], (j - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(smem + C::kSmemK + st * C::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tS, make_sdesc_sw128(qaddr + kk * 32, 16, 1024),
+                  make_sdesc_sw128(kaddr + kk * 32, 16, 1024), C::kIdescQK, kk > 0 ? 1u : 0u);
+        tc_commit(&bars[kPbSFull + s]);
+        tc_commit(&bars[kPbKEmpty + st]);
+        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok && nk > 0) ok = issue_pv(nk - 1);
+      for (int j = nk; ok && j < nkv0; ++j) {  // stages only the other tile uses
+        const int st = j % C::kStages;
+        if (!wait(&bars[kPbKFull + st], (j / C::kStages) & 1)) { ok = false; break; }
+        mbar_arrive(&bars[kPbKEmpty + st]);
+        if (!wait(&bars[kPbVFull + st], (j / C::kStages) & 1)) { ok = false; break; }
+        mbar_arrive(&bars[kPbVEmpty + st]);
+      }
+      if (!ok) {
+        // drain whatever was issued before giving up
+        tc_commit(&bars[kPbSpare + s]);
+        mbar_wait(&bars[kPbSpare + s], 0, nullptr, a.status, a.wait_limit_ns);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ softmax warps
+    const int s = warp >> 2, quarter = warp & 3;
+    const Slot t = s ? sl[1] : sl[0];
+    if (t.nkv > 0) {
+      const int r = quarter * 32 + lane;
+      const uint32_t tsl = tbase + (static_cast<uint32_t>(quarter * 32) << 16) + s * C::kTmemSlot;
+      const int rv = min(r, t.nrows - 1);
+      int pos, pos_first;
+      if (t.kind == kRouted) {
+        pos = a.bucket_tok[t.bstart + t.row0 + rv];
+        pos_first = a.bucket_tok[t.bstart + t.row0];
+      } else {
+        pos = t.row0 + rv;
+        pos_first = t.row0;
+      }
+      const float sl2 = a.scale_log2;
+      float m_used = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < t.nkv; ++j) {
+        // the lanes must agree: they go on to warp-collective tcgen05 instructions
+        if (!__all_sync(0xFFFFFFFFu, wait(&bars[kPbSFull + s], j & 1))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sv[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tsl + C::kTmemS + 32 * c, sv[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kPbSFree + s]);
+
+        const int kbase = j * kTileN;
+        if (kbase + kTileN - 1 > pos_first) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (kbase + 32 * c + e > pos) sv[c][e] = __float_as_uint(-INFINITY);
+        }
+        float mxp[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mxp[q] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            mxp[(e >> 1) & 7] = fmax3f(mxp[(e >> 1) & 7], __uint_as_float(sv[c][e]),
+                                       __uint_as_float(sv[c][e + 1]));
+        const float mx = fmax3f(fmax3f(mxp[0], mxp[1], mxp[2]), fmax3f(mxp[3], mxp[4], mxp[5]),
+                                fmaxf(mxp[6], mxp[7]));
+        const float mnew = fmaxf(m_used, mx * sl2);
+        float factor = 1.f;
+        if (mnew - m_used > 8.f) {
+          factor = ex2_approx(m_used - mnew);
+          m_used = mnew;
+        }
+        l *= factor;
+        // P.V of the previous tile must be done before P and O are touched
+        if (j > 0) {
+          if (!__all_sync(0xFFFFFFFFu, wait(&bars[kPbODone + s], (j - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        // the turn: tile 1 exponentiates its j-th KV tile after tile 0 has,
+        // and tile 0 its j-th after tile 1 its (j-1)-th (while tile 1 has one)
+
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_used, -m_used);
+        uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t y2 =
+                f2_fma(f2_pack(__uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1])), sl2x2,
+                       negm2);
+            float p0, p1;
+            if (((e >> 1) & 7) < kPolyPairs) {
+              exp2_poly_pair(y2, p0, p1);
+            } else {
+              float y0, y1;
+              f2_unpack(y2, y0, y1);
+              p0 = ex2_approx(y0);
+              p1 = ex2_approx(y1);
+            }
+            rs2[(e >> 1) & 3] = f2_add(rs2[(e >> 1) & 3], f2_pack(p0, p1));
+            pk[e / 2] = pack_half2(p0, p1);
+          }
+          tmem_st16(tsl + C::kTmemP + 16 * c, pk);
+        }
+        float r0, r1, r2, r3, r4, r5, r6, r7;
+        f2_unpack(rs2[0], r0, r1);
+        f2_unpack(rs2[1], r2, r3);
+        f2_unpack(rs2[2], r4, r5);
+        f2_unpack(rs2[3], r6, r7);
+        l += ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
+        if (j > 0 && __any_sync(0xFFFFFFFFu, factor != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tsl + C::kTmemO + 32 * c, ov);
+            tmem_ld_wait(ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+            tmem_st32(tsl + C::kTmemO + 32 * c, ov);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars[kPbPFull + s]);
+
+        }
+      }
+      ok = __all_sync(0xFFFFFFFFu, ok && wait(&bars[kPbODone + s], (t.nkv - 1) & 1));
+      if (ok) {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        const bool fp32 = a.out_fp32 != 0;
+        const size_t esz = fp32 ? 4 : 2;
+        uint8_t* dst = nullptr;
+        uint8_t* dst2 = nullptr;
+        if (r < t.nrows) {
+          const int64_t tokrow = static_cast<int64_t>(t.b) * S + pos;
+          if (t.kind == kShared) {
+            dst = static_cast<uint8_t*>(a.s_out) + (tokrow * a.out_row_stride) * esz;
+          } else {
+            const int32_t* sel = a.topk_idx + (tokrow * G + t.g) * a.k;
+            int slot = 0;
+            for (int q = 0; q < a.k; ++q)
+              if (sel[q] == t.m) slot = q;
+            dst = static_cast<uint8_t*>(a.O_sel) +
+                  (tokrow * a.out_row_stride + static_cast<int64_t>(t.g * a.k + slot) * D) * esz;
+            if (a.k == 1)
+              dst2 = static_cast<uint8_t*>(a.o_bar) +
+                     (tokrow * a.out_row_stride + static_cast<int64_t>(t.g) * D) * esz;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tsl + C::kTmemO + 32 * c, ov);
+          tmem_ld_wait(ov);
+          if (dst) store_row32(dst + 32 * c * esz, ov, inv, fp32);
+          if (dst2) store_row32(dst2 + 32 * c * esz, ov, inv, fp32);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kPairMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::kTmemCols);
+  }
+}
+
 __global__ void selftest_wait_kernel(int* status, uint64_t limit_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -477,12 +899,52 @@ cudaError_t launch_d(const AttnArgs& a, int64_t grid, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// K/V working set (bytes) from which the d = 64 calls use the pair kernel:
+// below about 3/4 of the 126 MB L2 the K/V tiles are served from L2 and
+// attn_kernel is faster.
+std::atomic<int64_t> g_pair_min_kv_bytes{int64_t(96) << 20};
+
+cudaError_t launch_pair(const AttnArgs& a, int64_t grid, cudaStream_t st) {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (configured_device != dev) {
+    e = cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PairCfg::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  attn_pair_kernel<<<static_cast<unsigned>(grid), kPairThreads, PairCfg::kSmemBytes, st>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-cudaError_t launch_attention(const AttnArgs& a, int64_t grid, cudaStream_t st) {
-  if (grid <= 0) return cudaSuccess;
-  if (a.d == 64) return launch_d<64>(a, grid, st);
-  if (a.d == 128) return launch_d<128>(a, grid, st);
+int64_t set_pair_threshold(int64_t kv_bytes) { return g_pair_min_kv_bytes.exchange(kv_bytes); }
+
+bool pair_kernel_for(const gqe_dims& d) {
+  if (d.d != 64) return false;
+  // K (bf16) and V (fp16) of every KV head the call reads
+  const int64_t kv_bytes = static_cast<int64_t>(d.B) * d.S * d.G * d.d * 4;
+  const int64_t thr = g_pair_min_kv_bytes.load();
+  return thr >= 0 && kv_bytes >= thr;
+}
+
+cudaError_t launch_attention(const AttnArgs& a, int64_t n_list, cudaStream_t st) {
+  const int64_t nq = (a.S + kTileM - 1) / kTileM;
+  if (a.d == 64) {
+    if (a.pair && !a.dense) {
+      const int64_t grid = n_list / 2;
+      return grid > 0 ? launch_pair(a, grid, st) : cudaSuccess;
+    }
+    const int64_t grid = a.dense ? static_cast<int64_t>(a.B) * a.N * nq : n_list;
+    return grid > 0 ? launch_d<64>(a, grid, st) : cudaSuccess;
+  }
+  if (a.d == 128) {
+    const int64_t grid = a.dense ? static_cast<int64_t>(a.B) * a.N * nq : n_list;
+    return grid > 0 ? launch_d<128>(a, grid, st) : cudaSuccess;
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -102,49 +102,108 @@ __device__ void bucket_body(const BucketArgs& a, int bg) {
 
   // routed work items: ceil(cnt/128) tiles per expert; unused slots get nkv 0
   TileDesc* slots = a.tiles_raw + static_cast<int64_t>(bg) * a.cap_bg;
-  int first = 0;
-  for (int m = 0; m < M; ++m) {
-    const int nt = (cnt[m] + kTileM - 1) / kTileM;
-    for (int t = tid; t < nt; t += kBucketThreads) {
-      const int row0 = t * kTileM;
-      const int nrows = min(kTileM, cnt[m] - row0);
-      const int last = a.bucket_tok[base + start[m] + row0 + nrows - 1];
-      TileDesc d;
-      d.code = (kRouted << 24) | (bg * M + m);
-      d.row0 = row0;
-      d.nrows = nrows;
-      d.nkv = last / kTileN + 1;
-      slots[first + t] = d;
+  if (!a.pairs) {
+    int first = 0;
+    for (int m = 0; m < M; ++m) {
+      const int nt = (cnt[m] + kTileM - 1) / kTileM;
+      for (int t = tid; t < nt; t += kBucketThreads) {
+        const int row0 = t * kTileM;
+        const int nrows = min(kTileM, cnt[m] - row0);
+        const int last = a.bucket_tok[base + start[m] + row0 + nrows - 1];
+        TileDesc d;
+        d.code = (kRouted << 24) | (bg * M + m);
+        d.row0 = row0;
+        d.nrows = nrows;
+        d.nkv = last / kTileN + 1;
+        slots[first + t] = d;
+      }
+      first += nt;
     }
-    first += nt;
+    for (int t = first + tid; t < a.cap_bg; t += kBucketThreads) slots[t] = TileDesc{0, 0, 0, 0};
+    return;
   }
-  for (int t = first + tid; t < a.cap_bg; t += kBucketThreads) slots[t] = TileDesc{0, 0, 0, 0};
+  // For the pair kernel the (b, g) block's tiles are placed in descending nkv
+  // order, a stable merge of the M per-expert lists (each ascending, as the
+  // bucket lists ascending positions), so that neighbours 2p, 2p+1 form a
+  // pair of nearly equal length.
+  __shared__ int tfirst[kMaxM + 1];
+  if (tid == 0) {
+    int s = 0;
+    for (int m = 0; m < M; ++m) {
+      tfirst[m] = s;
+      s += (cnt[m] + kTileM - 1) / kTileM;
+    }
+    tfirst[M] = s;
+  }
+  __syncthreads();
+  const int ntiles = tfirst[M];
+  const int32_t* tok = a.bucket_tok + base;
+  auto tile_nkv = [&](int m, int t) {
+    return tok[start[m] + min(t * kTileM + kTileM - 1, cnt[m] - 1)] / kTileN + 1;
+  };
+  for (int i = tid; i < ntiles; i += kBucketThreads) {
+    int m = 0;
+    while (i >= tfirst[m + 1]) ++m;
+    const int t = i - tfirst[m];
+    const int v = tile_nkv(m, t);
+    // ascending position under the key (nkv, m, t): t tiles of expert m come
+    // first, then, from every other expert, those with smaller nkv (or equal
+    // nkv and smaller m), found by binary search
+    int asc = t;
+    for (int m2 = 0; m2 < M; ++m2) {
+      if (m2 == m) continue;
+      int lo = 0, hi = tfirst[m2 + 1] - tfirst[m2];
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const int w = tile_nkv(m2, mid);
+        if (m2 < m ? w <= v : w < v) lo = mid + 1;
+        else hi = mid;
+      }
+      asc += lo;
+    }
+    const int row0 = t * kTileM;
+    TileDesc d;
+    d.code = (kRouted << 24) | (bg * M + m);
+    d.row0 = row0;
+    d.nrows = min(kTileM, cnt[m] - row0);
+    d.nkv = v;
+    slots[ntiles - 1 - asc] = d;
+  }
+  for (int t = ntiles + tid; t < a.cap_bg; t += kBucketThreads) slots[t] = TileDesc{0, 0, 0, 0};
 }
 
-// One CTA: shared-head tiles are appended, then every work item is sorted by
-// its KV-tile count, longest first (so the heaviest tiles start first and the
-// grid's tail is short).  Counting sort on nkv in [1, ceil(S/128)].
+// One CTA: the shared head's tiles are appended (for the pair kernel in
+// pairs: query tiles q and q-1 of one batch), then the work items (tiles, or
+// pairs by the KV-tile count of their first tile) are sorted longest first,
+// so the heaviest work starts first and the grid's tail is short.  Counting
+// sort on nkv in [1, ceil(S/128)].
 constexpr int kSchedThreads = 1024;
 
 __device__ void schedule_body(const BucketArgs& a, int* hist /* nq + 2 bins */) {
   const int tid = threadIdx.x;
   const int nq = (a.S + kTileM - 1) / kTileM;
+  const int nq2 = nq + (nq & 1);
   const int64_t n_routed = static_cast<int64_t>(a.B) * a.G * a.cap_bg;
   TileDesc* shared_tiles = a.tiles_raw + n_routed;
   for (int v = tid; v < nq + 2; v += kSchedThreads) hist[v] = 0;
-  // the shared head's tiles: every token, KV head 0
-  for (int64_t t = tid; t < static_cast<int64_t>(a.B) * nq; t += kSchedThreads) {
-    const int b = static_cast<int>(t / nq), q = static_cast<int>(t % nq);
-    TileDesc d;
-    d.code = (kShared << 24) | b;
-    d.row0 = q * kTileM;
-    d.nrows = min(kTileM, a.S - q * kTileM);
-    d.nkv = q + 1;
+  // the shared head's tiles: every token, KV head 0; slot i of a batch holds
+  // query tile nq-1-i (so pair i/2 is tiles nq-1-2(i/2) and nq-2-2(i/2))
+  for (int64_t t = tid; t < static_cast<int64_t>(a.B) * nq2; t += kSchedThreads) {
+    const int b = static_cast<int>(t / nq2), q = nq - 1 - static_cast<int>(t % nq2);
+    TileDesc d{0, 0, 0, 0};
+    if (q >= 0) {
+      d.code = (kShared << 24) | b;
+      d.row0 = q * kTileM;
+      d.nrows = min(kTileM, a.S - q * kTileM);
+      d.nkv = q + 1;
+    }
     shared_tiles[t] = d;
   }
   __syncthreads();
-  for (int64_t t = tid; t < a.n_raw_tiles; t += kSchedThreads) {
-    const int v = a.tiles_raw[t].nkv;
+  const int per = a.pairs ? 2 : 1;  // list entries per work item
+  const int64_t nitems = a.n_raw_tiles / per;
+  for (int64_t p = tid; p < nitems; p += kSchedThreads) {
+    const int v = a.tiles_raw[per * p].nkv;
     if (v > 0) atomicAdd(&hist[v], 1);
   }
   __syncthreads();
@@ -155,12 +214,16 @@ __device__ void schedule_body(const BucketArgs& a, int* hist /* nq + 2 bins */) 
       hist[v] = s;
       s += c;
     }
-    *a.tile_count = s;
+    *a.tile_count = per * s;
   }
   __syncthreads();
-  for (int64_t t = tid; t < a.n_raw_tiles; t += kSchedThreads) {
-    const TileDesc d = a.tiles_raw[t];
-    if (d.nkv > 0) a.tiles[atomicAdd(&hist[d.nkv], 1)] = d;
+  for (int64_t p = tid; p < nitems; p += kSchedThreads) {
+    const TileDesc d0 = a.tiles_raw[per * p];
+    if (d0.nkv > 0) {
+      const int64_t dst = atomicAdd(&hist[d0.nkv], 1);
+      a.tiles[per * dst] = d0;
+      if (per == 2) a.tiles[2 * dst + 1] = a.tiles_raw[2 * p + 1];
+    }
   }
 }
 

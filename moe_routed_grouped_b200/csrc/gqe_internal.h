@@ -22,9 +22,23 @@ enum TileKind : int { kRouted = 0, kShared = 1, kDense = 2 };
 //   code  = (kind << 24) | id   (routed: bucket (b*G+g)*M+m; shared: b)
 //   row0  = first row inside the bucket (routed) or first token (shared)
 //   nrows = valid rows (1..128); nkv = KV tiles to visit (0 = empty slot)
+// For the pair kernel (d = 64, K and V larger than L2) the work list holds
+// tiles in pairs (entries 2p, 2p+1) of the same batch and KV head, the first
+// with the larger nkv; the second may be empty.  A pair is one CTA, which
+// loads each K/V tile once for both.  Otherwise it is a list of single tiles.
 struct TileDesc {
   int32_t code, row0, nrows, nkv;
 };
+
+// Work-list capacity: routed tile slots per (b, g) and the list length
+// (routed slots, then the shared head's tiles), both even so pairs align.
+inline void tile_list_dims(int64_t B, int64_t S, int64_t G, int64_t M, int64_t k,
+                           int64_t* cap_bg, int64_t* n_raw_tiles) {
+  const int64_t nq = (S + kTileM - 1) / kTileM;
+  const int64_t c = (S * k + kTileM - 1) / kTileM + M;
+  *cap_bg = c + (c & 1);
+  *n_raw_tiles = B * G * *cap_bg + B * (nq + (nq & 1));
+}
 
 // Byte offsets of the regions inside the caller's workspace.
 struct WsLayout {
@@ -37,11 +51,11 @@ struct WsLayout {
   size_t v16;         // fp16 [B,S,G,d]: V converted for the P.V product
   size_t bucket_off;  // int32[B*G*M + 1]
   size_t bucket_tok;  // int32[B*G*S*k]
-  size_t tiles_raw;   // TileDesc[n_raw_tiles]
-  size_t tiles;       // TileDesc[n_raw_tiles] sorted by nkv, descending
+  size_t tiles_raw;   // TileDesc[n_raw_tiles], in pairs
+  size_t tiles;       // TileDesc[n_raw_tiles]: pairs sorted by nkv, descending
   size_t total;
-  int64_t cap_bg;       // routed tile slots per (b, g)
-  int64_t n_raw_tiles;  // B*G*cap_bg + B*nq (routed + shared)
+  int64_t cap_bg;       // routed tile slots per (b, g), even
+  int64_t n_raw_tiles;  // B*G*cap_bg + B*nq rounded up to even (routed + shared)
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -49,9 +63,7 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline WsLayout make_ws_layout(const gqe_dims& d) {
   WsLayout L{};
   const int64_t B = d.B, S = d.S, G = d.G, M = d.N / d.G, k = d.k, hd = d.d;
-  const int64_t nq = (S + kTileM - 1) / kTileM;
-  L.cap_bg = (S * k + kTileM - 1) / kTileM + M;
-  L.n_raw_tiles = B * G * L.cap_bg + B * nq;
+  tile_list_dims(B, S, G, M, k, &L.cap_bg, &L.n_raw_tiles);
   size_t off = 0;
   L.status = off;     off += 256;
   L.counters = off;   off += 256;
@@ -94,6 +106,7 @@ struct BucketArgs {
   int32_t* done;            // CTA completion counter (self-resetting)
   int* status;
   int B, S, G, M, k;
+  int pairs;                // 1: build the paired list of the pair kernel
   int64_t cap_bg;
   int64_t n_raw_tiles;
 };
@@ -118,8 +131,8 @@ struct AttnArgs {
   const int32_t* bucket_off;
   const int32_t* bucket_tok;
   const int32_t* topk_idx;
-  const TileDesc* tiles;
-  const int32_t* tile_count;
+  const TileDesc* tiles;      // pairs, sorted
+  const int32_t* tile_count;  // list entries in use (2 x pairs)
   void* O_sel;
   void* o_bar;
   void* s_out;
@@ -129,10 +142,18 @@ struct AttnArgs {
   int B, S, N, G, M, k, d;
   int out_fp32;
   int dense;          // 1: dense GQA tiles from blockIdx; 0: routed/shared list
+  int pair;           // 1: the pair kernel on a paired list (d = 64 only)
   float scale_log2;   // log2(e) / sqrt(d)
   uint64_t wait_limit_ns;
 };
-cudaError_t launch_attention(const AttnArgs& a, int64_t grid, cudaStream_t st);
+// n_list: length of the work list (routed/shared); unused for dense tiles.
+cudaError_t launch_attention(const AttnArgs& a, int64_t n_list, cudaStream_t st);
+// K/V working-set size from which routed d = 64 calls use the pair kernel;
+// returns the previous value (negative: never).  pair_kernel_for() is the
+// decision for one call: taken once, then passed to the bucketing (list
+// format) and to the attention launch.
+int64_t set_pair_threshold(int64_t kv_bytes);
+bool pair_kernel_for(const gqe_dims& d);
 
 struct CombineArgs {
   const void* O_sel;

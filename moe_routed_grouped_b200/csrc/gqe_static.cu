@@ -38,9 +38,7 @@ struct StaticLayout {
 StaticLayout static_layout(const gqe_dims& d) {
   StaticLayout L{};
   const int64_t B = d.B, S = d.S, G = d.G, M = d.N / d.G, k = d.k, hd = d.d;
-  const int64_t nq = (S + gqe::kTileM - 1) / gqe::kTileM;
-  L.cap_bg = (S * k + gqe::kTileM - 1) / gqe::kTileM + M;
-  L.n_raw_tiles = B * G * L.cap_bg + B * nq;
+  gqe::tile_list_dims(B, S, G, M, k, &L.cap_bg, &L.n_raw_tiles);
   size_t off = 0;
   L.status = off;     off += 256;
   L.counters = off;   off += 256;
@@ -166,6 +164,8 @@ extern "C" gqe_status gqe_attention_prefill_static(
   ba.k = dims->k;
   ba.cap_bg = L.cap_bg;
   ba.n_raw_tiles = L.n_raw_tiles;
+  const bool pair = gqe::pair_kernel_for(*dims);  // one decision: list format and kernel
+  ba.pairs = pair ? 1 : 0;
   if (gqe::launch_prep(ba, &cv, true, s) != cudaSuccess) return GQE_ERR_CUDA;
 
   gqe::AttnArgs a;
@@ -198,6 +198,7 @@ extern "C" gqe_status gqe_attention_prefill_static(
   a.d = dims->d;
   a.out_fp32 = dims->out_fp32;
   a.dense = 0;
+  a.pair = pair ? 1 : 0;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   a.wait_limit_ns = gqe::kWaitLimitNs;
   if (gqe::launch_attention(a, L.n_raw_tiles, s) != cudaSuccess) return GQE_ERR_CUDA;
