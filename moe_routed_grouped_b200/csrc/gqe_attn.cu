@@ -81,29 +81,70 @@ struct Waiter {
   }
 };
 
-__device__ __forceinline__ void store_row32(void* dst, const uint32_t (&v)[32], float scale,
-                                            bool fp32) {
-  if (fp32) {
-    float4* o = reinterpret_cast<float4*>(dst);
+// Output rows of one softmax warp: lane l holds query row l of the warp's
+// TMEM lane quarter (O at taddr_o), its 1/l scale and its destination(s)
+// (null: not stored).  The rows are normalised into shared memory (32 rows
+// of D + 4 floats: conflict-free for both access patterns below) and then
+// written row by row with consecutive lanes on consecutive 16-byte pieces, so
+// each store instruction covers whole 128-byte segments of one or a few rows
+// instead of 32 scattered pieces.
+template <int D>
+__device__ __noinline__ void store_rows_coalesced(float* stage, uint32_t taddr_o, float inv,
+                                               uint8_t* dst, uint8_t* dst2, bool fp32) {
+  constexpr int kStr = D + 4;
+  const int lane = threadIdx.x & 31;
+  float* mine = stage + lane * kStr;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t ov[32];
+    tmem_ld32(taddr_o + 32 * c, ov);
+    tmem_ld_wait(ov);
 #pragma unroll
     for (int q = 0; q < 8; ++q)
-      o[q] = make_float4(__uint_as_float(v[4 * q]) * scale, __uint_as_float(v[4 * q + 1]) * scale,
-                         __uint_as_float(v[4 * q + 2]) * scale,
-                         __uint_as_float(v[4 * q + 3]) * scale);
+      reinterpret_cast<float4*>(mine + 32 * c)[q] =
+          make_float4(__uint_as_float(ov[4 * q]) * inv, __uint_as_float(ov[4 * q + 1]) * inv,
+                      __uint_as_float(ov[4 * q + 2]) * inv, __uint_as_float(ov[4 * q + 3]) * inv);
+  }
+  __syncwarp();
+  const unsigned long long d1 = reinterpret_cast<unsigned long long>(dst);
+  const unsigned long long d2 = reinterpret_cast<unsigned long long>(dst2);
+  if (fp32) {
+    constexpr int kLanesPerRow = D / 4;  // 16-byte pieces of 4 floats
+    constexpr int kRows = 32 / kLanesPerRow;
+    const int sub = lane / kLanesPerRow, piece = lane % kLanesPerRow;
+#pragma unroll 4
+    for (int r0 = 0; r0 < 32; r0 += kRows) {
+      const int row = r0 + sub;
+      float4* o1 = reinterpret_cast<float4*>(__shfl_sync(0xFFFFFFFFu, d1, row));
+      float4* o2 = reinterpret_cast<float4*>(__shfl_sync(0xFFFFFFFFu, d2, row));
+      const float4 v = reinterpret_cast<const float4*>(stage + row * kStr)[piece];
+      if (o1) o1[piece] = v;
+      if (o2) o2[piece] = v;
+    }
   } else {
-    uint4* o = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    constexpr int kLanesPerRow = D / 8;  // 16-byte pieces of 8 bf16
+    constexpr int kRows = 32 / kLanesPerRow;
+    const int sub = lane / kLanesPerRow, piece = lane % kLanesPerRow;
+#pragma unroll 4
+    for (int r0 = 0; r0 < 32; r0 += kRows) {
+      const int row = r0 + sub;
+      uint4* o1 = reinterpret_cast<uint4*>(__shfl_sync(0xFFFFFFFFu, d1, row));
+      uint4* o2 = reinterpret_cast<uint4*>(__shfl_sync(0xFFFFFFFFu, d2, row));
+      const float4* src = reinterpret_cast<const float4*>(stage + row * kStr + 8 * piece);
+      const float4 x0 = src[0], x1 = src[1];
+      const float f[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]) * scale,
-                                                 __uint_as_float(v[8 * q + 2 * e + 1]) * scale);
+        __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
         w[e] = *reinterpret_cast<uint32_t*>(&h);
       }
-      o[q] = make_uint4(w[0], w[1], w[2], w[3]);
+      const uint4 v = make_uint4(w[0], w[1], w[2], w[3]);
+      if (o1) o1[piece] = v;
+      if (o2) o2[piece] = v;
     }
   }
+  __syncwarp();
 }
 
 template <int D>
@@ -407,39 +448,33 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
     }
     if (ok) ok = wait(&bars[kBarODone], (nkv - 1) & 1);
     ok = __all_sync(0xFFFFFFFFu, ok);
+    const bool fp32 = a.out_fp32 != 0;
+    const size_t esz = fp32 ? 4 : 2;
+    uint8_t* dst = nullptr;
+    uint8_t* dst2 = nullptr;
+    if (ok && r < nrows) {
+      const int64_t tokrow = static_cast<int64_t>(b) * S + pos;
+      if (kind == kDense) {
+        dst = static_cast<uint8_t*>(a.O_dense) + ((tokrow * N + h) * D) * esz;
+      } else if (kind == kShared) {
+        dst = static_cast<uint8_t*>(a.s_out) + (tokrow * a.out_row_stride) * esz;
+      } else {
+        const int32_t* sel = a.topk_idx + (tokrow * G + g) * a.k;
+        int slot = 0;
+        for (int q = 0; q < a.k; ++q)
+          if (sel[q] == m) slot = q;
+        dst = static_cast<uint8_t*>(a.O_sel) +
+              (tokrow * a.out_row_stride + static_cast<int64_t>(g * a.k + slot) * D) * esz;
+        if (a.k == 1)
+          dst2 = static_cast<uint8_t*>(a.o_bar) +
+                 (tokrow * a.out_row_stride + static_cast<int64_t>(g) * D) * esz;
+      }
+    }
     if (ok) {
       tc_fence_after();
-      const float inv = 1.f / l;
-      const bool fp32 = a.out_fp32 != 0;
-      const size_t esz = fp32 ? 4 : 2;
-      uint8_t* dst = nullptr;
-      uint8_t* dst2 = nullptr;
-      if (r < nrows) {
-        const int64_t tokrow = static_cast<int64_t>(b) * S + pos;
-        if (kind == kDense) {
-          dst = static_cast<uint8_t*>(a.O_dense) + ((tokrow * N + h) * D) * esz;
-        } else if (kind == kShared) {
-          dst = static_cast<uint8_t*>(a.s_out) + (tokrow * a.out_row_stride) * esz;
-        } else {
-          const int32_t* sel = a.topk_idx + (tokrow * G + g) * a.k;
-          int slot = 0;
-          for (int q = 0; q < a.k; ++q)
-            if (sel[q] == m) slot = q;
-          dst = static_cast<uint8_t*>(a.O_sel) +
-                (tokrow * a.out_row_stride + static_cast<int64_t>(g * a.k + slot) * D) * esz;
-          if (a.k == 1)
-            dst2 = static_cast<uint8_t*>(a.o_bar) +
-                   (tokrow * a.out_row_stride + static_cast<int64_t>(g) * D) * esz;
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(tbase + lane_off + C::kTmemO + 32 * c, ov);
-        tmem_ld_wait(ov);
-        if (dst) store_row32(dst + 32 * c * esz, ov, inv, fp32);
-        if (dst2) store_row32(dst2 + 32 * c * esz, ov, inv, fp32);
-      }
+      // every product is done, so the K/V stages are free for the staging rows
+      float* stage = reinterpret_cast<float*>(smem + C::kSmemK) + warp * 32 * (D + 4);
+      store_rows_coalesced<D>(stage, tbase + lane_off + C::kTmemO, 1.f / l, dst, dst2, fp32);
     }
   }
 
@@ -479,7 +514,9 @@ struct PairCfg {
   static constexpr int kSmemQ = 0;  // two Q tiles
   static constexpr int kSmemK = 2 * kQBytes;
   static constexpr int kSmemV = kSmemK + kStages * kKVBytes;
-  static constexpr int kSmemBar = kSmemV + kStages * kKVBytes;
+  // output staging: 8 softmax warps x 32 rows x (D + 4) floats
+  static constexpr int kSmemStage = kSmemV + kStages * kKVBytes;
+  static constexpr int kSmemBar = kSmemStage + 8 * 32 * (D + 4) * 4;
   static constexpr int kSmemBytes = kSmemBar + 256 + 1024;  // barriers + alignment slack
   static constexpr uint32_t kTmemSlot = 256, kTmemS = 0, kTmemP = 128, kTmemO = 192;
   static constexpr uint32_t kTmemCols = 512;
@@ -827,37 +864,31 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
       }
       ok = __all_sync(0xFFFFFFFFu, ok && wait(&bars[kPbODone + s], (t.nkv - 1) & 1));
+      const bool fp32 = a.out_fp32 != 0;
+      const size_t esz = fp32 ? 4 : 2;
+      uint8_t* dst = nullptr;
+      uint8_t* dst2 = nullptr;
+      if (ok && r < t.nrows) {
+        const int64_t tokrow = static_cast<int64_t>(t.b) * S + pos;
+        if (t.kind == kShared) {
+          dst = static_cast<uint8_t*>(a.s_out) + (tokrow * a.out_row_stride) * esz;
+        } else {
+          const int32_t* sel = a.topk_idx + (tokrow * G + t.g) * a.k;
+          int slot = 0;
+          for (int q = 0; q < a.k; ++q)
+            if (sel[q] == t.m) slot = q;
+          dst = static_cast<uint8_t*>(a.O_sel) +
+                (tokrow * a.out_row_stride + static_cast<int64_t>(t.g * a.k + slot) * D) * esz;
+          if (a.k == 1)
+            dst2 = static_cast<uint8_t*>(a.o_bar) +
+                   (tokrow * a.out_row_stride + static_cast<int64_t>(t.g) * D) * esz;
+        }
+      }
       if (ok) {
         tc_fence_after();
-        const float inv = 1.f / l;
-        const bool fp32 = a.out_fp32 != 0;
-        const size_t esz = fp32 ? 4 : 2;
-        uint8_t* dst = nullptr;
-        uint8_t* dst2 = nullptr;
-        if (r < t.nrows) {
-          const int64_t tokrow = static_cast<int64_t>(t.b) * S + pos;
-          if (t.kind == kShared) {
-            dst = static_cast<uint8_t*>(a.s_out) + (tokrow * a.out_row_stride) * esz;
-          } else {
-            const int32_t* sel = a.topk_idx + (tokrow * G + t.g) * a.k;
-            int slot = 0;
-            for (int q = 0; q < a.k; ++q)
-              if (sel[q] == t.m) slot = q;
-            dst = static_cast<uint8_t*>(a.O_sel) +
-                  (tokrow * a.out_row_stride + static_cast<int64_t>(t.g * a.k + slot) * D) * esz;
-            if (a.k == 1)
-              dst2 = static_cast<uint8_t*>(a.o_bar) +
-                     (tokrow * a.out_row_stride + static_cast<int64_t>(t.g) * D) * esz;
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(tsl + C::kTmemO + 32 * c, ov);
-          tmem_ld_wait(ov);
-          if (dst) store_row32(dst + 32 * c * esz, ov, inv, fp32);
-          if (dst2) store_row32(dst2 + 32 * c * esz, ov, inv, fp32);
-        }
+        // K/V stages may still feed the other tile: stage in this warp's own region
+        float* stage = reinterpret_cast<float*>(smem + C::kSmemStage) + warp * 32 * (D + 4);
+        store_rows_coalesced<D>(stage, tsl + C::kTmemO, 1.f / l, dst, dst2, fp32);
       }
     }
   }
