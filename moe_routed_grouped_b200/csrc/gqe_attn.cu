@@ -81,6 +81,24 @@ struct Waiter {
   }
 };
 
+// One query row of a routed tile: row r of the token's Q head, copied with
+// cp.async into the 128-byte swizzle the UMMA descriptor expects (16-byte
+// chunk c of row r at c ^ (r & 7)); zero-filled when the row is past the
+// bucket's end.  Each softmax thread copies its own row, so the 128 rows are
+// in flight at once; the copies are complete and visible to the tensor core
+// when this returns.
+template <int D, int kAtom>
+__device__ __forceinline__ void gather_q_row(uint8_t* sQ, int r, const uint16_t* src, bool valid) {
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const int atom = c >> 3, ch = c & 7;
+    cp_async_16(sQ + atom * kAtom + r * 128 + ((ch ^ (r & 7)) << 4), src + c * 8,
+                valid ? 16u : 0u);
+  }
+  cp_async_wait_all();
+  fence_proxy_async_smem();
+}
+
 // Output rows of one softmax warp: lane l holds query row l of the warp's
 // TMEM lane quarter (O at taddr_o), its 1/l scale and its destination(s)
 // (null: not stored).  The rows are normalised into shared memory (32 rows
@@ -199,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
   const Waiter wait{abort_flag, a.status, a.wait_limit_ns};
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[kBarQFull], 1);
+    // routed Q rows are gathered by the 4 softmax warps, other Q tiles by TMA
+    mbar_init(&bars[kBarQFull], kind == kRouted ? 4 : 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&bars[kBarKFull + s], 1);
       mbar_init(&bars[kBarKEmpty + s], 1);
@@ -231,26 +250,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
   if (warp == kProducerWarp) {
     // ------------------------------------------------------ producer
     uint8_t* sQ = smem + C::kSmemQ;
-    if (kind == kRouted) {
-      // gather the bucket's query rows, writing the 128-byte swizzle that
-      // the UMMA descriptor expects (16-byte chunk c of row r at c ^ (r & 7))
-      for (int rr = 0; rr < kTileM / 32; ++rr) {
-        const int r = lane + 32 * rr;
-        const bool ok = r < nrows;
-        const int tok = ok ? a.bucket_tok[bstart + row0 + r] : 0;
-        const uint16_t* src = a.Q + ((static_cast<int64_t>(b) * S + tok) * N + h) * D;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const int atom = c >> 3, ch = c & 7;
-          uint8_t* dst = sQ + atom * C::kAtom + r * 128 + ((ch ^ (r & 7)) << 4);
-          cp_async_16(dst, src + c * 8, ok ? 16u : 0u);
-        }
-      }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarQFull]);
-    } else if (lane == 0) {
+    if (kind != kRouted && lane == 0) {
       mbar_arrive_expect_tx(&bars[kBarQFull], C::kQBytes);
 #pragma unroll
       for (int atom = 0; atom < D / 64; ++atom) {
@@ -345,6 +345,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
     if (kind == kRouted) {
       pos = a.bucket_tok[bstart + row0 + rv];
       pos_first = a.bucket_tok[bstart + row0];
+      gather_q_row<D, C::kAtom>(smem + C::kSmemQ, r,
+                                a.Q + ((static_cast<int64_t>(b) * S + pos) * N + h) * D,
+                                r < nrows);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarQFull]);
     } else {
       pos = row0 + rv;
       pos_first = row0;
@@ -599,7 +604,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars[kPbQFull + s], 1);
+      mbar_init(&bars[kPbQFull + s], sl[s].kind == kRouted ? 4 : 1);
       mbar_init(&bars[kPbSFull + s], 1);
       mbar_init(&bars[kPbSFree + s], 4);
       mbar_init(&bars[kPbPFull + s], 4);
@@ -638,23 +643,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const Slot t = sl[s];
       if (t.nkv == 0) continue;
       uint8_t* sQ = smem + C::kSmemQ + s * C::kQBytes;
-      if (t.kind == kRouted) {
-        // gather the bucket's query rows in the 128-byte swizzle of the UMMA
-        // descriptor (16-byte chunk c of row r at c ^ (r & 7))
-        for (int rr = 0; rr < kTileM / 32; ++rr) {
-          const int r = lane + 32 * rr;
-          const bool ok = r < t.nrows;
-          const int tok = ok ? a.bucket_tok[t.bstart + t.row0 + r] : 0;
-          const uint16_t* src = a.Q + ((static_cast<int64_t>(t.b) * S + tok) * N + t.h) * D;
-#pragma unroll
-          for (int c = 0; c < D / 8; ++c)
-            cp_async_16(sQ + r * 128 + ((c ^ (r & 7)) << 4), src + c * 8, ok ? 16u : 0u);
-        }
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kPbQFull + s]);
-      } else if (lane == 0) {
+      if (t.kind != kRouted && lane == 0) {  // routed rows: gathered by the softmax warps
         mbar_arrive_expect_tx(&bars[kPbQFull + s], C::kQBytes);
         tma_load_3d(sQ, &a.tmQs, &bars[kPbQFull + s], 0, t.row0, t.b);
       }
@@ -757,6 +746,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       if (t.kind == kRouted) {
         pos = a.bucket_tok[t.bstart + t.row0 + rv];
         pos_first = a.bucket_tok[t.bstart + t.row0];
+        gather_q_row<D, C::kAtom>(smem + C::kSmemQ + s * C::kQBytes, r,
+                                  a.Q + ((static_cast<int64_t>(t.b) * S + pos) * N + t.h) * D,
+                                  r < t.nrows);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kPbQFull + s]);
       } else {
         pos = t.row0 + rv;
         pos_first = t.row0;

@@ -93,6 +93,7 @@ struct RouteArgs {
   int32_t* fix_count;
   int* status;
   int T, dm, G, M, k;
+  int tok;              // tokens per route_kernel tile (set by the launcher)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 

@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(32 * GM) route_prep_kernel(const RouteArgs a) 
 template <int GM>
 struct RouteShape {
   static constexpr int kTPL = GM <= 16 ? 2 : 1;
-  static constexpr int kTok = 32 * kTPL;   // tokens per tile
+  static constexpr int kTok = 32 * kTPL;   // most tokens per tile (RouteArgs::tok)
 };
 
 template <int GM>
@@ -68,6 +68,8 @@ struct RouteSmem {
   float xsq[kRouteWarps][Sh::kTok];
   int nflag;
   int flags[Sh::kTok * 32];
+  float wnorm[GM];                                  // ||W_r[:, col]||
+  float bias[GM];
   int sel[kRouteWarps][kMaxM];
 };
 
@@ -100,7 +102,8 @@ __device__ __forceinline__ void load_wt_chunk(const float* wt, int c0, int rows,
   }
 }
 
-// Persistent CTAs of 4 warps; a tile is kTok tokens.  Warp w sums the
+// Persistent CTAs of 4 warps; a tile is a.tok <= kTok tokens (sized so the
+// tiles fill the SMs evenly; lane l takes tokens l and l + 32).  Warp w sums the
 // products of the d_model chunks w, w+4, ... ; lane l keeps its tokens' x
 // values in registers and reads each W_r row as a broadcast from the warp's
 // shared-memory copy of the chunk (copied from the float32 transpose made by
@@ -112,7 +115,8 @@ __device__ __forceinline__ void load_wt_chunk(const float* wt, int c0, int rows,
 template <int GM>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
   using Sh = RouteShape<GM>;
-  constexpr int TPL = Sh::kTPL, TOK = Sh::kTok;
+  constexpr int TPL = Sh::kTPL;
+  const int TOK = a.tok;
   extern __shared__ __align__(16) uint8_t route_smem_raw[];
   RouteSmem<GM>& sm = *reinterpret_cast<RouteSmem<GM>*>(route_smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -123,6 +127,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
       static_cast<float>(32 + (nchunks + kRouteWarps - 1) / kRouteWarps + 4) * 5.9604645e-8f *
       1.01f;
 
+  for (int c = tid; c < GM; c += kRouteThreads) {
+    sm.wnorm[c] = sqrtf(a.wsq[c]);
+    sm.bias[c] = a.bias ? a.bias[c] : 0.f;
+  }
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const int t0 = tile * TOK;
     const int ntok = min(TOK, a.T - t0);
@@ -217,12 +225,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     bool nonfinite = false;
     for (int q = tid; q < ntok * GM; q += kRouteThreads) {
       const int ql = q / GM, col = q % GM;
-      const float b = a.bias ? a.bias[col] : 0.f;
+      const float b = sm.bias[col];
       const float l = (((sm.red[0][ql][col] + sm.red[1][ql][col]) + sm.red[2][ql][col]) +
                        sm.red[3][ql][col]) + b;
       const float xn = sqrtf(((sm.xsq[0][ql] + sm.xsq[1][ql]) + sm.xsq[2][ql]) + sm.xsq[3][ql]);
       sm.lgt[ql][col] = l;
-      sm.err[ql][col] = cerr * fmaf(xn, sqrtf(a.wsq[col]), fabsf(b)) + 1e-36f;
+      sm.err[ql][col] = cerr * fmaf(xn, sm.wnorm[col], fabsf(b)) + 1e-36f;
       nonfinite |= !isfinite(l);
     }
     if (nonfinite) latch_status(a.status, GQE_ERR_NONFINITE);
@@ -559,9 +567,14 @@ cudaError_t launch_route_gm(const RouteArgs& a, cudaStream_t st) {
   route_prep_kernel<GM><<<(a.dm + 31) / 32, 32 * GM, 0, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int ntiles = (a.T + RouteShape<GM>::kTok - 1) / RouteShape<GM>::kTok;
+  // tokens per tile: about two tiles per SM when the tokens allow it, at most
+  // kTok (two per lane)
+  RouteArgs b = a;
+  const int64_t want = (static_cast<int64_t>(a.T) + 2 * sms - 1) / (2 * sms);
+  b.tok = static_cast<int>(want < 1 ? 1 : (want > RouteShape<GM>::kTok ? RouteShape<GM>::kTok : want));
+  const int ntiles = (a.T + b.tok - 1) / b.tok;
   const int grid = ntiles < 4 * sms ? ntiles : 4 * sms;
-  route_kernel<GM><<<grid, kRouteThreads, smem, st>>>(a);
+  route_kernel<GM><<<grid, kRouteThreads, smem, st>>>(b);
   return cudaGetLastError();
 }
 
