@@ -332,9 +332,16 @@ cudaError_t launch_prep(const BucketArgs& a, const ConvertArgs* cv, bool with_sc
   ConvertArgs c{};
   if (cv) {
     c = *cv;
+    // the conversion CTAs take the slots the bucket CTAs leave free (two
+    // 1024-thread CTAs per SM), so the launch runs in one wave
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t n8 = c.n / 8;
+    const int slots = 2 * sms, nb = a.B * a.G;
+    const int cap = nb < slots - slots / 4 ? slots - nb : slots / 4;
     nconv = static_cast<int>((n8 + kBucketThreads - 1) / kBucketThreads);
-    if (nconv > 148 * 2) nconv = 148 * 2;
+    if (nconv > cap) nconv = cap;
     if (nconv < 1) nconv = 1;
   }
   prep_kernel<<<a.B * a.G + nconv, kBucketThreads, smem, st>>>(a, c, with_schedule ? 1 : 0);
