@@ -76,7 +76,41 @@ def test_empty_buckets_pair_kernel(pair_kernel):
     check_close(L.s_out().cpu().numpy(), s, "s")
 
 
-@pytest.mark.parametrize("name", ["layer250m"])
+def test_bf16_output_pair_kernel(pair_kernel):
+    """bf16 concat output through the pair kernel's staged stores: within the
+    float32 bound plus 2^-8 |ref| (half an ulp for the output, half for the
+    k > 1 sum of rounded slots)."""
+    shape = (1, 300, 16, 8, 2, 64, 64)
+    B, S, N, G, k, d, dm = shape
+    inp = make_case(B, S, N, G, k, d, dm, 14000)
+    dev = upload(inp)
+    L = GqePrefill(B, S, N, G, k, d, dm, out_fp32=False)
+    L.forward(dev["x"], dev["W_r"], None, dev["Q"], dev["Qs"], dev["K"], dev["V"])
+    torch.cuda.synchronize()
+    assert L.device_status() == 0
+    idx, _, w, _ = oracle.route(inp["x"], inp["W_r"], None, k)
+    O_sel, o_bar, s = oracle.gqe_prefill(inp["Q"], inp["Qs"], inp["K"], inp["V"], idx, w)
+    for got, ref, what in ((L.O_sel(), O_sel, "O_sel"), (L.o_bar(), o_bar, "o_bar"),
+                           (L.s_out(), s, "s")):
+        g = got.float().cpu().numpy()
+        assert (np.abs(g - ref) <= 1e-2 + 2 ** -8 * np.abs(ref)).all(), what
+
+
+def test_static_entry_with_pair_kernel(pair_kernel):
+    """The no-workspace entry takes the same kernel decision: with the pair
+    kernel forced it writes what the workspace call writes, bit for bit."""
+    shape = (2, 300, 16, 8, 2, 64, 64)
+    inp, dev, L = _forward(shape, seed=15000)
+    out = torch.full_like(L.concat, float("nan"))
+    a = L.G * L.k * L.d
+    gqe.gqe_attention_prefill_static(L.dims, dev["Q"], dev["Qs"], dev["K"], dev["V"],
+                                     L.topk_idx, L.w, out, out.view(-1)[a:],
+                                     out.view(-1)[a + L.G * L.d:], L.row)
+    torch.cuda.synchronize()
+    assert torch.equal(out, L.concat)
+
+
+@pytest.mark.parametrize("name", ["layer250m", "imbalanced32k"])
 def test_pair_kernel_equals_one_tile_kernel(name):
     """Same bits from both kernels on a full-size workload; dense calls keep
     the one-tile kernel whatever the threshold."""
@@ -84,12 +118,13 @@ def test_pair_kernel_equals_one_tile_kernel(name):
     inp = make_inputs(w)
     dev = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(torch.bfloat16).cuda()
            for k, v in inp.items() if k != "bias"}
+    bias = None if inp.get("bias") is None else torch.from_numpy(inp["bias"]).cuda()
     L = GqePrefill(w.B, w.S, w.N, w.G, w.k, w.d, w.d_model, out_fp32=True)
     outs = []
     for thr in (-1, 0):
         prev = gqe.gqe_set_pair_threshold(thr)
         try:
-            L.forward(dev["x"], dev["W_r"], None, dev["Q"], dev["Qs"], dev["K"], dev["V"])
+            L.forward(dev["x"], dev["W_r"], bias, dev["Q"], dev["Qs"], dev["K"], dev["V"])
             O = L.dense(dev["Q"], dev["K"], dev["V"])
             torch.cuda.synchronize()
             assert L.device_status() == 0
