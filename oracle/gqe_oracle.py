@@ -106,6 +106,17 @@ def router_logits(x: np.ndarray, Wr: np.ndarray, bias: Optional[np.ndarray]
     return L, err
 
 
+def exact_logits(x_row: np.ndarray, W_g: np.ndarray, bias_g: Optional[np.ndarray]
+                 ) -> np.ndarray:
+    """The M logits of one (token, group), each the exact sum of its float64
+    products (exact for bf16 operands) and bias, correctly rounded to float64
+    by ``math.fsum``."""
+    M = W_g.shape[1]
+    bias_g = np.zeros(M) if bias_g is None else np.asarray(bias_g, dtype=np.float64)
+    return np.array([math.fsum((x_row * W_g[:, m]).tolist() + [float(bias_g[m])])
+                     for m in range(M)])
+
+
 def topk_exact_order(x_row: np.ndarray, W_g: np.ndarray, bias_g: Optional[np.ndarray]
                      ) -> list:
     """All M experts of one (token, group) ordered by EXACT logit, desc.
@@ -165,8 +176,14 @@ def route(x_bits: np.ndarray, Wr_bits: np.ndarray, bias: Optional[np.ndarray], k
 
     unsure = np.argwhere(~certain)
     for t, g in unsure:
-        ordr = topk_exact_order(bf16_to_f64(xb[t]), Wr[g], None if bias is None else bias[g])
+        xt = bf16_to_f64(xb[t])
+        bg = None if bias is None else bias[g]
+        ordr = topk_exact_order(xt, Wr[g], bg)
         idx[t, g] = ordr[:k]
+        # where the float64 estimate cannot order the experts it cannot serve
+        # the softmax either (products that cancel by far more than 2^53):
+        # take the correctly rounded logits of this pair
+        L[t, g] = exact_logits(xt, Wr[g], bg)
 
     # p = softmax over the group's M experts (float64)
     mx = L.max(axis=-1, keepdims=True)

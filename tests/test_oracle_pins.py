@@ -348,6 +348,31 @@ def check_buckets(idx, M):
     assert n == B * G * S * k
 
 
+def test_router_p_from_exact_logits_under_cancellation():
+    """Products spanning ~190 binary orders cancel far below float64's reach:
+    the selection comes from exact arithmetic, and so must p (softmax of the
+    logits, [GQE review] 路由器).  Checked against logits summed in Fractions:
+    the selected expert is the exact argmax, its p is the largest and the
+    weights are finite."""
+    rng = np.random.default_rng(11)
+    S, dm, G, M = 64, 64, 2, 4
+    mags = np.array([2.0 ** -90, 2.0 ** -40, 1.0, 2.0 ** 30, 2.0 ** 60])
+    x = (mags[rng.integers(0, 5, (1, S, dm))] * rng.choice([-1, 1], (1, S, dm))).astype(np.float32)
+    W = (mags[rng.integers(0, 5, (G, dm, M))] * rng.choice([-1, 1], (G, dm, M)) * 2.0 ** -20
+         ).astype(np.float32)
+    xb, Wb = f32_to_bf16_bits(x), f32_to_bf16_bits(W)
+    idx, p, w, n_exact = oracle.route(xb, Wb, None, 1)
+    assert n_exact > 0 and np.isfinite(w).all() and np.isfinite(p).all()
+    xf, Wf = og.bf16_to_f64(xb)[0], og.bf16_to_f64(Wb)
+    for t in range(S):
+        for g in range(G):
+            exact = [sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xf[t], Wf[g][:, m]))
+                     for m in range(M)]
+            best = max(range(M), key=lambda m: (exact[m], -m))
+            assert idx[0, t, g, 0] == best
+            assert p[0, t, g, best] == p[0, t, g].max()
+
+
 def test_bucket_bruteforce():
     xb = normal_bf16((3, 50, 16), 51)
     Wb = normal_bf16((4, 16, 4), 52, std=0.3)
