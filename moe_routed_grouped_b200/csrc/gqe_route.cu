@@ -444,6 +444,15 @@ __device__ void exact_logit(const RouteArgs& a, int t, int g, int m, Exact& out,
   out.top = static_cast<int32_t>(full[kLimbs - 1]);  // |sum| < 2^540: top limb is tiny
 }
 
+// The value of an exact logit as a double (the limbs from the top down, then
+// the 2^-266 scale): within a few ulps, enough for the softmax; the ordering
+// itself uses exact_cmp.
+__device__ __forceinline__ double exact_to_double(const Exact& e) {
+  double v = static_cast<double>(e.top);
+  for (int i = kLimbs - 2; i >= 0; --i) v = v * 4294967296.0 + static_cast<double>(e.v[i]);
+  return ldexp(v, -kExpBias);
+}
+
 // -1, 0, +1 for a < b, a == b, a > b
 __device__ __forceinline__ int exact_cmp(const Exact& a, const Exact& b) {
   if (a.top != b.top) return a.top < b.top ? -1 : 1;
@@ -534,11 +543,20 @@ __device__ void exact_rank_pair(const RouteArgs& a, int t, int g, int* sel) {
     }
   }
   if (lane < M && rank < k) sel[rank] = lane;
+  // p of this pair again, from the float64 logits or (when those could not
+  // order the experts) the exact ones: the float32 logits of the main pass
+  // may have cancelled catastrophically for a pair that needed this path
+  if (lane < M && !certain) l64[warp][lane] = exact_to_double(ex[warp][lane]);
   __syncwarp();
   if (lane == 0) {
     if (bad) latch_status(a.status, GQE_ERR_NONFINITE);
     const int64_t row = static_cast<int64_t>(t) * a.G + g;
-    const float* prow = a.p + row * M;
+    float* prow = a.p + row * M;
+    double mx = l64[warp][0];
+    for (int m = 1; m < M; ++m) mx = fmax(mx, l64[warp][m]);
+    double s = 0.0;
+    for (int m = 0; m < M; ++m) s += exp(l64[warp][m] - mx);
+    for (int m = 0; m < M; ++m) prow[m] = static_cast<float>(exp(l64[warp][m] - mx) / s);
     float den = 0.f;
     for (int j = 0; j < k; ++j) den += prow[sel[j]];
     for (int j = 0; j < k; ++j) {

@@ -189,3 +189,9 @@ def test_router_exact_wide_exponent_range():
     got = L.topk_idx.cpu().numpy()
     assert np.array_equal(got, idx)
     assert not (got == 1).any()             # the tie always goes to expert 0
+    # p of the re-decided pairs comes from their exact (or float64) logits on
+    # both sides, so it stays a proper distribution even where the products
+    # cancel far below float32's reach
+    gp = L.p.cpu().numpy()
+    assert np.isfinite(gp).all() and np.isfinite(L.w.cpu().numpy()).all()
+    check_close(gp, p, "p", atol=1e-5, rtol_l2=1e-5)
