@@ -452,6 +452,9 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        # this rank's per-step spread (the mean above is the max over ranks)
+        "ms_per_step_median": statistics.median(res["routed_ms"]),
+        "ms_per_step_best": min(res["routed_ms"]),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 inputs; random-init router)",
         "config": config_of(w, world),
@@ -492,6 +495,10 @@ def main():
             dm = sum(r["dense_ms"]) / k_steps
             sweep.append({
                 "workload": name, "S": ws.S, "routed_ms": rm, "dense_ms": dm,
+                "routed_ms_median": statistics.median(r["routed_ms"]),
+                "routed_ms_best": min(r["routed_ms"]),
+                "dense_ms_median": statistics.median(r["dense_ms"]),
+                "dense_ms_best": min(r["dense_ms"]),
                 "routed_tokens_per_s": ws.B * ws.S / (rm / 1e3),
                 "routed_useful_tflops": ws.useful_flop_routed() / (rm / 1e3) / 1e12,
                 "dense_useful_tflops": ws.useful_flop_dense() / (dm / 1e3) / 1e12,
