@@ -63,6 +63,19 @@ def test_routed_parity_pair_kernel(shape, pair_kernel):
     check_close(L.s_out().cpu().numpy(), s, "shared head")
 
 
+def test_biased_batch_pair_kernel(pair_kernel):
+    """A batch of 3 with routing biased towards expert 0 (uneven buckets, so
+    uneven pairs) and k = 2."""
+    shape = (3, 257, 16, 4, 2, 64, 64)
+    inp, _, L = _forward(shape, seed=16000, bias0=1.5)
+    idx, _, w, _ = oracle.route(inp["x"], inp["W_r"], inp["bias"], 2)
+    assert np.array_equal(L.topk_idx.cpu().numpy(), idx)
+    O_sel, o_bar, s = oracle.gqe_prefill(inp["Q"], inp["Qs"], inp["K"], inp["V"], idx, w)
+    check_close(L.O_sel().cpu().numpy(), O_sel, "O_sel")
+    check_close(L.o_bar().cpu().numpy(), o_bar, "o_bar")
+    check_close(L.s_out().cpu().numpy(), s, "shared head")
+
+
 def test_empty_buckets_pair_kernel(pair_kernel):
     """Every token picks expert 0: the other buckets are empty and some pairs
     have an empty second tile."""

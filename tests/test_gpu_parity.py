@@ -195,3 +195,39 @@ def test_router_exact_wide_exponent_range():
     gp = L.p.cpu().numpy()
     assert np.isfinite(gp).all() and np.isfinite(L.w.cpu().numpy()).all()
     check_close(gp, p, "p", atol=1e-5, rtol_l2=1e-5)
+
+
+# more shapes: d = 128 with every expert selected (k = M), a batch of 3 with
+# biased routing and k = 2, and the bf16 output at d = 128
+MORE = [
+    ((1, 300, 16, 4, 4, 128, 128), 0.0),
+    ((3, 257, 16, 4, 2, 64, 64), 1.5),
+]
+
+
+@pytest.mark.parametrize("shape,bias0", MORE, ids=lambda v: "x".join(map(str, v))
+                         if isinstance(v, tuple) else str(v))
+def test_routed_prefill_parity_more(shape, bias0):
+    B, S, N, G, k, d, dm = shape
+    inp, L = _run(shape, seed=17000 + sum(shape), bias0=bias0)
+    idx, p, w, _ = oracle.route(inp["x"], inp["W_r"], inp["bias"], k)
+    assert np.array_equal(L.topk_idx.cpu().numpy(), idx), "top-k indices differ"
+    check_close(L.w.cpu().numpy(), w, "w", atol=1e-5, rtol_l2=1e-5)
+    O_sel, o_bar, s = oracle.gqe_prefill(inp["Q"], inp["Qs"], inp["K"], inp["V"], idx, w)
+    check_close(L.O_sel().cpu().numpy(), O_sel, "O_sel")
+    check_close(L.o_bar().cpu().numpy(), o_bar, "o_bar")
+    check_close(L.s_out().cpu().numpy(), s, "shared head")
+
+
+def test_bf16_output_mode_d128():
+    shape = (1, 300, 16, 4, 2, 128, 128)
+    B, S, N, G, k, d, dm = shape
+    inp, L = _run(shape, seed=18000, out_fp32=False)
+    idx, p, w, _ = oracle.route(inp["x"], inp["W_r"], None, k)
+    O_sel, o_bar, s = oracle.gqe_prefill(inp["Q"], inp["Qs"], inp["K"], inp["V"], idx, w)
+    # float32 bound plus 2^-8 |ref|: half an ulp for the bf16 output, half
+    # for the k > 1 sum of already rounded slots
+    for got, ref, what in ((L.O_sel(), O_sel, "O_sel"), (L.o_bar(), o_bar, "o_bar"),
+                           (L.s_out(), s, "s")):
+        g = got.float().cpu().numpy()
+        assert (np.abs(g - ref) <= 1e-2 + 2 ** -8 * np.abs(ref)).all(), what
