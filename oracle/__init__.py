@@ -1,4 +1,4 @@
-"""CPU oracle for GQE prefill (test infrastructure, not product code).
+"""CPU oracle for GQE prefill and decode (test infrastructure, not product code).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The library under
@@ -13,6 +13,8 @@ from .gqe_oracle import (  # noqa: F401
     causal_attention,
     gqe_prefill,
     gqe_prefill_rows,
+    gqe_decode_step,
+    exact_logits,
     dense_gqa,
     dense_gqa_repeat,
     kv_cache_bytes,

@@ -23,7 +23,7 @@ Sources (web pages; cited by title and section):
 * [MQA/GQA explainer] "MQA、GQA、稀疏/滑动窗口注意力及混合范式": the MQA and
   GQA numeric examples and the KV-cache byte examples.
 
-Readings where the pages are silent (also listed in the design doc):
+Readings where the pages are silent:
 
 * r_g is linear, ``l = x · W_r[g]`` (+ an optional per-(g, m) bias).
 * Top-k is decided on the EXACT real-valued logits (softmax is strictly
@@ -301,6 +301,45 @@ def gqe_prefill_rows(Q_bits, Qs_bits, K_bits, V_bits, topk_idx, w, rows, dtype=n
         o_bar.append(ob)
         s_out.append(sb)
     return O_sel, o_bar, s_out
+
+
+def gqe_decode_step(x_bits, Wr_bits, bias, Q_bits, Qs_bits, Kc_bits, Vc_bits, pos, k,
+                    dtype=np.float64):
+    """One incremental decode step of GQE, for each sequence b of a batch.
+
+    [GQA article] 工程实操 非方形因果遮罩: at an incremental decode step the query
+    length is 1 and the key length is the whole history; the mask is taken on
+    the query's absolute position.  The new token of sequence b sits at
+    position pos[b]; its own K/V are already in the caches at that position
+    (Kc, Vc [B, T, G, d] with T > pos[b]) and later slots are not visible.  It
+    routes as in prefill ([GQE review] §二 路由器), each selected head attends
+    with its group's KV head, the shared head with KV head 0, and ō is the
+    weighted sum of the slots (三个关键部件).  x [B, dm], Q [B, N, d], Qs [B, d]
+    are bf16 bit patterns.  Returns (topk_idx [B,G,k], p [B,G,M], w [B,G,k],
+    O_sel [B,G,k,d], o_bar [B,G,d], s [B,d]).
+    """
+    B = x_bits.shape[0]
+    idx, p, w, _ = route(np.asarray(x_bits)[:, None, :], Wr_bits, bias, k)
+    idx, p, w = idx[:, 0], p[:, 0], w[:, 0]
+    N, d = Q_bits.shape[1], Q_bits.shape[2]
+    G = Kc_bits.shape[2]
+    M = N // G
+    O_sel = np.zeros((B, G, k, d), dtype=dtype)
+    o_bar = np.zeros((B, G, d), dtype=dtype)
+    s_out = np.zeros((B, d), dtype=dtype)
+    for b in range(B):
+        r = np.array([int(pos[b])])
+        Kb, Vb = bf16_to_f64(Kc_bits[b]), bf16_to_f64(Vc_bits[b])
+        for g in range(G):
+            for j in range(k):
+                h = _expert_head(g, int(idx[b, g, j]), M)
+                q = bf16_to_f64(Q_bits[b, h])[None, :]
+                O_sel[b, g, j] = causal_attention(q, r, Kb[:, g], Vb[:, g], dtype=dtype)[0]
+        for j in range(k):  # ascending slot order
+            o_bar[b] = o_bar[b] + np.asarray(w[b, :, j, None], dtype=dtype) * O_sel[b, :, j]
+        s_out[b] = causal_attention(bf16_to_f64(Qs_bits[b])[None, :], r, Kb[:, 0], Vb[:, 0],
+                                    dtype=dtype)[0]
+    return idx, p, w, O_sel, o_bar, s_out
 
 
 def dense_gqa(Q_bits, K_bits, V_bits, dtype=np.float64, rows=None):

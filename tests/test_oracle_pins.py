@@ -373,6 +373,52 @@ def test_router_p_from_exact_logits_under_cancellation():
             assert p[0, t, g, best] == p[0, t, g].max()
 
 
+def _decode_case(seed):
+    B, S, N, G, k, d, dm = 2, 40, 8, 4, 2, 16, 32
+    return (B, S, N, G, k, d, dm), dict(
+        x=normal_bf16((B, S, dm), seed), W_r=normal_bf16((G, dm, N // G), seed + 1, std=dm ** -0.5),
+        Q=normal_bf16((B, S, N, d), seed + 2), Qs=normal_bf16((B, S, d), seed + 3),
+        K=normal_bf16((B, S, G, d), seed + 4), V=normal_bf16((B, S, G, d), seed + 5))
+
+
+def test_decode_step_equals_prefill_row():
+    """A decode step at position t over the caches of the first t+1 tokens is
+    prefill's row t: the same routing, slots, weighted sum and shared head."""
+    (B, S, N, G, k, d, dm), c = _decode_case(19000)
+    idx, p, w, _ = oracle.route(c["x"], c["W_r"], None, k)
+    O_sel, o_bar, s = oracle.gqe_prefill(c["Q"], c["Qs"], c["K"], c["V"], idx, w)
+    for pos in ([0, 0], [17, 39], [39, 5]):
+        b_ = np.arange(B)
+        t = np.array(pos)
+        di, dp, dw, dO, dob, ds = oracle.gqe_decode_step(
+            c["x"][b_, t], c["W_r"], None, c["Q"][b_, t], c["Qs"][b_, t], c["K"], c["V"], t, k)
+        assert np.array_equal(di, idx[b_, t])
+        assert np.allclose(dp, p[b_, t], rtol=0, atol=1e-15)
+        assert np.allclose(dO, O_sel[b_, t], rtol=1e-12, atol=1e-12)
+        assert np.allclose(dob, o_bar[b_, t], rtol=1e-12, atol=1e-12)
+        assert np.allclose(ds, s[b_, t], rtol=1e-12, atol=1e-12)
+
+
+def test_decode_step_ignores_later_cache_slots_and_position0():
+    """Slots after the query's position are invisible (garbage there changes
+    nothing); at position 0 every head returns V[0] of its KV head exactly."""
+    (B, S, N, G, k, d, dm), c = _decode_case(19100)
+    t = np.array([0, 11])
+    b_ = np.arange(B)
+    args = (c["x"][b_, t], c["W_r"], None, c["Q"][b_, t], c["Qs"][b_, t])
+    ref = oracle.gqe_decode_step(*args, c["K"], c["V"], t, k)
+    K2, V2 = c["K"].copy(), c["V"].copy()
+    for b in range(B):
+        K2[b, t[b] + 1:] = f32_to_bf16_bits(np.full(K2[b, t[b] + 1:].shape, 3.0e4, np.float32))
+        V2[b, t[b] + 1:] = f32_to_bf16_bits(np.full(V2[b, t[b] + 1:].shape, -7.0e3, np.float32))
+    got = oracle.gqe_decode_step(*args, K2, V2, t, k)
+    for a_, b2 in zip(ref, got):
+        assert np.array_equal(a_, b2)
+    V0 = og.bf16_to_f64(c["V"][0, 0])          # [G, d]
+    assert np.array_equal(ref[3][0], np.repeat(V0[:, None, :], k, axis=1))
+    assert np.array_equal(ref[5][0], V0[0])
+
+
 def test_bucket_bruteforce():
     xb = normal_bf16((3, 50, 16), 51)
     Wb = normal_bf16((4, 16, 4), 52, std=0.3)
