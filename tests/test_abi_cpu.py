@@ -96,3 +96,17 @@ def test_workspace_grows_with_shape():
     b = _lib.gqe_workspace_size(_lib.dims(8, 2048, 16, 8, 1, 64, 1024))
     c = _lib.gqe_workspace_size(_lib.dims(1, 131072, 32, 8, 2, 128, 4096))
     assert 0 < a < b < c
+
+
+def test_pair_threshold_is_a_host_setting():
+    """The d = 64 kernel choice is a process-wide host value: set, read back
+    through the previous-value return, restored.  No device is touched."""
+    prev = gqe.gqe_set_pair_threshold(1 << 20)
+    try:
+        assert gqe.gqe_set_pair_threshold(0) == 1 << 20
+        assert gqe.gqe_set_pair_threshold(-1) == 0
+        assert gqe.gqe_set_pair_threshold(96 << 20) == -1
+    finally:
+        gqe.gqe_set_pair_threshold(prev)
+    assert prev == 96 << 20  # the default: 96 MiB of K/V
+
