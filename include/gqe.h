@@ -1,5 +1,6 @@
 /*
- * gqe.h - C ABI of the GQE (Grouped Query Experts) causal-prefill library.
+ * gqe.h - C ABI of the GQE (Grouped Query Experts) library: causal prefill
+ * and incremental decode.
  *
  * Grouped Query Experts puts a per-group router on grouped-query attention:
  * N query heads form G groups of M = N/G "query-head experts" that share one
@@ -22,7 +23,8 @@
  *  - Every device pointer must be 16-byte aligned.  Tensors are dense,
  *    row-major, in the layouts stated per argument (B batch, S tokens).
  *  - `ws` is a caller-owned device workspace of at least
- *    gqe_workspace_size(dims) bytes, zero-filled once before its first use
+ *    gqe_workspace_size(dims) bytes (gqe_decode_workspace_size for the
+ *    decode call), zero-filled once before its first use
  *    (it holds a latched device status word; the library keeps the rest
  *    consistent itself).  Calls that share one workspace must be ordered
  *    (same stream or explicit events).
@@ -31,9 +33,9 @@
  *    shapes are rejected, never silently remapped ("AI 大模型之 GQA",
  *    工程实操: unsupported H/G combinations must be refused explicitly).
  *  - Errors found on the device (a bounded wait that ran out, an expert index
- *    out of range, non-finite router logits, V outside the fp16 range) are
- *    latched into the workspace status word; read them with
- *    gqe_get_device_status().  Nothing is thrown across the ABI.
+ *    or a decode position out of range, non-finite router logits, V outside
+ *    the fp16 range) are latched into the workspace status word; read them
+ *    with gqe_get_device_status().  Nothing is thrown across the ABI.
  *
  * Supported shapes: N % G == 0, M = N/G <= 32, 1 <= k <= M,
  * d in {64, 128}; for the router G*M in {4, 8, 16, 32} and d_model % 8 == 0;
@@ -57,7 +59,8 @@ typedef enum gqe_status {
   GQE_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out           */
   GQE_ERR_WORKSPACE = 5,    /* workspace missing or smaller than required   */
   GQE_ERR_BAD_INDEX = 6,    /* a top-k index outside [0, M) reached a kernel */
-  GQE_ERR_NONFINITE = 7     /* non-finite logit, or |V| above the fp16 range */
+  GQE_ERR_NONFINITE = 7,    /* non-finite logit, or |V| above the fp16 range */
+  GQE_ERR_BAD_POSITION = 8  /* a decode position outside [0, T) reached a kernel */
 } gqe_status;
 
 /* Problem size.  M = N / G is derived.  `out_fp32` selects the element type
@@ -171,6 +174,47 @@ gqe_status gqe_attention_prefill_static(const gqe_dims* dims, const void* Q, con
 gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void* K,
                                  const void* V, void* O, void* ws, size_t ws_bytes,
                                  void* stream);
+
+/* Bytes of workspace gqe_attention_decode needs for `dims` (0 if invalid).
+ * Its status word sits at offset 0 and its scratch starts at byte 512, after
+ * the region gqe_route keeps its counters in; so one zero-filled buffer of
+ * max(gqe_workspace_size(route dims), gqe_decode_workspace_size(dims)) bytes
+ * serves a decode step's gqe_route and gqe_attention_decode in stream order. */
+size_t gqe_decode_workspace_size(const gqe_dims* dims);
+
+/*
+ * gqe_attention_decode - one incremental decode step of GQE.
+ * "AI 大模型之 GQA", 工程实操 非方形因果遮罩: at a decode step the query length
+ * is 1 and the key length is the whole history; the causal mask is taken on
+ * the query's absolute position.  The new token of sequence b sits at
+ * position pos[b] and sees cache slots 0..pos[b].  As in prefill (review §二),
+ * slot j of group g is the head h = g*M + topk_idx[b,g,j] against KV head g,
+ * o_bar is the w-weighted sum of the group's slots, and the shared head
+ * attends KV head 0.
+ *
+ *  dims     B sequences, S = T (capacity of the caches' time axis), N, G, k,
+ *           d as for prefill; d_model is not used.
+ *  Q        device bf16 [B, N, d]     queries of the new tokens
+ *  Qs       device bf16 [B, d]        shared-head queries
+ *  Kc, Vc   device bf16 [B, T, G, d]  caches; slot pos[b] must already hold
+ *           the new token's K and V (the append is the caller's copy)
+ *  pos      device int32 [B]          0 <= pos[b] < T, may differ per b
+ *  topk_idx device int32 [B, G, k]; w device fp32 [B, G, k]: gqe_route with
+ *           dims S = 1 on the new tokens' x
+ *  O_sel, o_bar, s_out, out_row_stride: as for gqe_attention_prefill, one
+ *           output row per sequence b.
+ * Output element type: float32 if dims->out_fp32 else bf16.  A position out
+ * of range latches GQE_ERR_BAD_POSITION and that sequence's outputs are NaN;
+ * an expert index out of range latches GQE_ERR_BAD_INDEX and its slot and
+ * o_bar are NaN.  The cache is read once per step: each CTA serves every
+ * selected head of its KV head (and the shared head for KV head 0) over one
+ * chunk of keys, and a second kernel merges the chunks.
+ */
+gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void* Qs,
+                                const void* Kc, const void* Vc, const int32_t* pos,
+                                const int32_t* topk_idx, const float* w, void* O_sel,
+                                void* o_bar, void* s_out, int64_t out_row_stride, void* ws,
+                                size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, then returns the status word latched in `ws`
  * (GQE_OK if no device-side error was recorded).  If `clear` is non-zero the

@@ -1,11 +1,12 @@
-"""GQE (Grouped Query Experts) causal prefill for B200 (sm_100a).
+"""GQE (Grouped Query Experts) causal prefill and decode for B200 (sm_100a).
 
 The compute lives in ``libgqe.so`` (CUDA kernels behind the C ABI of
 ``include/gqe.h``); this package only loads it (``_lib``) and offers a thin
 torch-facing layer (``layer``) that allocates device buffers and calls the ABI.
 """
 from ._lib import (  # noqa: F401
-    EXPORTS, GqeDims, GqeError, LIB, LIB_PATH, STATUS, dims, gqe_attention_prefill,
+    EXPORTS, GqeDims, GqeError, LIB, LIB_PATH, STATUS, dims, gqe_attention_decode,
+    gqe_attention_prefill, gqe_decode_workspace_size,
     gqe_attention_prefill_static, gqe_bucket,
     gqe_dense_gqa_prefill, gqe_get_device_status, gqe_kv_cache_bytes, gqe_route,
     gqe_selftest_bounded_wait, gqe_set_pair_threshold, gqe_set_profile_events, gqe_status_string,

@@ -17,12 +17,13 @@ EXPORTS = (
     "gqe_workspace_size", "gqe_route", "gqe_bucket", "gqe_attention_prefill",
     "gqe_dense_gqa_prefill", "gqe_get_device_status", "gqe_kv_cache_bytes",
     "gqe_status_string", "gqe_selftest_bounded_wait", "gqe_set_profile_events",
-    "gqe_attention_prefill_static", "gqe_set_pair_threshold",
+    "gqe_attention_prefill_static", "gqe_set_pair_threshold", "gqe_decode_workspace_size",
+    "gqe_attention_decode",
 )
 
 STATUS = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED", 3: "GQE_ERR_CUDA",
           4: "GQE_ERR_TIMEOUT", 5: "GQE_ERR_WORKSPACE", 6: "GQE_ERR_BAD_INDEX",
-          7: "GQE_ERR_NONFINITE"}
+          7: "GQE_ERR_NONFINITE", 8: "GQE_ERR_BAD_POSITION"}
 
 
 class GqeDims(ctypes.Structure):
@@ -55,6 +56,8 @@ def _load() -> ctypes.CDLL:
         "gqe_set_profile_events": (None, [P, P]),
         "gqe_attention_prefill_static": (I32, [S, P, P, P, P, P, P, P, P, P, I64, P]),
         "gqe_set_pair_threshold": (I64, [I64]),
+        "gqe_decode_workspace_size": (SZ, [S]),
+        "gqe_attention_decode": (I32, [S, P, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -154,3 +157,17 @@ def gqe_attention_prefill_static(dm, Q, Qs, K, V, topk_idx, w, O_sel, o_bar, s_o
                                          _ptr(topk_idx), _ptr(w), _ptr(O_sel), _ptr(o_bar),
                                          _ptr(s_out), int(out_row_stride), _stream(stream))
     return _check(r, "gqe_attention_prefill_static") if check else r
+
+
+def gqe_decode_workspace_size(dm: GqeDims) -> int:
+    return LIB.gqe_decode_workspace_size(ctypes.byref(dm))
+
+
+def gqe_attention_decode(dm, Q, Qs, Kc, Vc, pos, topk_idx, w, O_sel, o_bar, s_out,
+                         out_row_stride, ws, stream=None, check=True):
+    """One decode step; dm.S is the cache capacity T."""
+    r = LIB.gqe_attention_decode(ctypes.byref(dm), _ptr(Q), _ptr(Qs), _ptr(Kc), _ptr(Vc),
+                                 _ptr(pos), _ptr(topk_idx), _ptr(w), _ptr(O_sel), _ptr(o_bar),
+                                 _ptr(s_out), int(out_row_stride), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_attention_decode") if check else r

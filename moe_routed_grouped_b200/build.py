@@ -14,7 +14,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgqe.so")
-SOURCES = ["gqe_route.cu", "gqe_bucket.cu", "gqe_attn.cu", "gqe_api.cu", "gqe_static.cu"]
+SOURCES = ["gqe_route.cu", "gqe_bucket.cu", "gqe_attn.cu", "gqe_decode.cu", "gqe_api.cu",
+           "gqe_static.cu"]
 HEADERS = ["gqe_device.cuh", "gqe_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC = os.environ.get("NVCC", "nvcc")

@@ -1,6 +1,6 @@
 // C-ABI entry points of the GQE prefill library (declared in include/gqe.h).
 // Argument validation happens here, before any launch; the kernels live in
-// gqe_route.cu, gqe_bucket.cu and gqe_attn.cu.
+// gqe_route.cu, gqe_bucket.cu, gqe_attn.cu and gqe_decode.cu.
 #include <cmath>
 #include <cstring>
 
@@ -293,6 +293,58 @@ gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void
 
 int64_t gqe_set_pair_threshold(int64_t kv_bytes) { return set_pair_threshold(kv_bytes); }
 
+size_t gqe_decode_workspace_size(const gqe_dims* dims) {
+  if (check_dims(dims, false) != GQE_OK) return 0;
+  return make_decode_plan(*dims).total;
+}
+
+gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void* Qs,
+                                const void* Kc, const void* Vc, const int32_t* pos,
+                                const int32_t* topk_idx, const float* w, void* O_sel,
+                                void* o_bar, void* s_out, int64_t out_row_stride, void* ws,
+                                size_t ws_bytes, void* stream) {
+  gqe_status st = check_dims(dims, false);
+  if (st != GQE_OK) return st;
+  if (!aligned16(Q) || !aligned16(Qs) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(pos) ||
+      !aligned16(topk_idx) || !aligned16(w) || !aligned16(O_sel) || !aligned16(o_bar) ||
+      !aligned16(s_out))
+    return GQE_ERR_INVALID_ARG;
+  if (out_row_stride < dims->d || out_row_stride % 8 != 0) return GQE_ERR_INVALID_ARG;
+  const DecodePlan P = make_decode_plan(*dims);
+  if (!aligned16(ws) || ws_bytes < P.total) return GQE_ERR_WORKSPACE;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  DecodeArgs a{};
+  a.Q = static_cast<const uint16_t*>(Q);
+  a.Qs = static_cast<const uint16_t*>(Qs);
+  a.Kc = static_cast<const uint16_t*>(Kc);
+  a.Vc = static_cast<const uint16_t*>(Vc);
+  a.pos = pos;
+  a.topk_idx = topk_idx;
+  a.w = w;
+  a.part_m = reinterpret_cast<float*>(wb + P.part_m);
+  a.part_l = reinterpret_cast<float*>(wb + P.part_l);
+  a.part_o = reinterpret_cast<float*>(wb + P.part_o);
+  a.O_sel = O_sel;
+  a.o_bar = o_bar;
+  a.s_out = s_out;
+  a.out_row_stride = out_row_stride;
+  a.status = reinterpret_cast<int*>(wb + P.status);
+  a.B = dims->B;
+  a.T = dims->S;
+  a.N = dims->N;
+  a.G = dims->G;
+  a.M = dims->N / dims->G;
+  a.k = dims->k;
+  a.d = dims->d;
+  a.heads = static_cast<int>(P.heads);
+  a.passes = static_cast<int>(P.passes);
+  a.nchunks = static_cast<int>(P.nchunks);
+  a.chunk = static_cast<int>(P.chunk);
+  a.out_fp32 = dims->out_fp32;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dims->d)));
+  return from_cuda(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
 gqe_status gqe_get_device_status(void* ws, int32_t clear, void* stream) {
   if (!aligned16(ws)) return GQE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -301,7 +353,7 @@ gqe_status gqe_get_device_status(void* ws, int32_t clear, void* stream) {
   if (cudaMemcpy(&code, ws, sizeof(code), cudaMemcpyDeviceToHost) != cudaSuccess)
     return GQE_ERR_CUDA;
   if (clear && cudaMemset(ws, 0, sizeof(int32_t)) != cudaSuccess) return GQE_ERR_CUDA;
-  if (code < GQE_OK || code > GQE_ERR_NONFINITE) return GQE_ERR_CUDA;
+  if (code < GQE_OK || code > GQE_ERR_BAD_POSITION) return GQE_ERR_CUDA;
   return static_cast<gqe_status>(code);
 }
 
@@ -323,6 +375,7 @@ const char* gqe_status_string(gqe_status s) {
     case GQE_ERR_WORKSPACE: return "workspace missing or too small";
     case GQE_ERR_BAD_INDEX: return "expert index out of range";
     case GQE_ERR_NONFINITE: return "non-finite value or value outside the fp16 range";
+    case GQE_ERR_BAD_POSITION: return "decode position out of range";
   }
   return "unknown status";
 }

@@ -38,7 +38,7 @@ def test_kv_cache_bytes_matches_pages():
 
 
 def test_status_strings():
-    for code in range(8):
+    for code in range(9):
         assert gqe.gqe_status_string(code)
     assert gqe.gqe_status_string(99) == "unknown status"
 
@@ -110,3 +110,38 @@ def test_pair_threshold_is_a_host_setting():
         gqe.gqe_set_pair_threshold(prev)
     assert prev == 96 << 20  # the default: 96 MiB of K/V
 
+
+
+def test_decode_rejects_bad_arguments():
+    """gqe_attention_decode validates before launching (dims.S is the cache
+    capacity T); nothing here reaches a device."""
+    dm = _lib.dims(2, 4096, 16, 8, 1, 64)
+    L = _lib.LIB
+    need = _lib.gqe_decode_workspace_size(dm)
+    assert need > 512
+
+    def call(stride=17 * 64, ws_bytes=1 << 40, pos=FAKE, d=dm):
+        return L.gqe_attention_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, pos, FAKE, FAKE,
+                                      FAKE, FAKE, FAKE, stride, FAKE, ws_bytes, None)
+    assert call(stride=60) == 1                      # not a multiple of 8
+    assert call(pos=None) == 1                       # positions are required
+    assert call(pos=ctypes.c_void_p(0x10004)) == 1   # misaligned
+    assert call(ws_bytes=need - 1) == 5
+    assert call(d=_lib.dims(2, 4096, 16, 8, 3, 64)) == 1   # k > M
+    assert call(d=_lib.dims(2, 4096, 16, 8, 1, 96)) == 2   # head dim outside {64, 128}
+    assert _lib.gqe_decode_workspace_size(_lib.dims(2, 4096, 16, 8, 3, 64)) == 0
+
+
+def test_decode_workspace_scales_with_the_split():
+    """The split-KV scratch holds (max, sum, d outputs) per head slot (k
+    routed + shared) and chunk; chunks are at least 256 keys, so a short
+    cache has one chunk, and the router's counters (bytes 256..511) stay out
+    of the decode scratch."""
+    one = _lib.gqe_decode_workspace_size(_lib.dims(1, 200, 16, 8, 1, 64))
+    # one chunk: 8 groups x 2 slots x (1 + 1 + 64) floats, each block 256-aligned
+    assert one == 512 + 256 + 256 + 8 * 2 * 64 * 4
+    long = _lib.gqe_decode_workspace_size(_lib.dims(1, 32768, 16, 8, 1, 64))
+    wide = _lib.gqe_decode_workspace_size(_lib.dims(1, 32768, 32, 8, 2, 128))
+    assert one < long < wide
+    # the scratch does not grow past the CTA target once chunks are long
+    assert _lib.gqe_decode_workspace_size(_lib.dims(1, 1 << 20, 16, 8, 1, 64)) <= 2 * long

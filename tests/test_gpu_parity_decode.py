@@ -1,0 +1,179 @@
+"""GPU parity of the decode step (query length 1 over a KV cache) through the
+C ABI against the CPU oracle's decode step.
+
+Routing indices must match bit for bit; float32 outputs must be within 1e-2
+max-abs and 1e-3 relative L2 of the float64 oracle.  The positions are chosen
+on the split-KV chunk edges (the first and last key of a chunk, a single key)
+so that the chunk merge is exercised with ragged tails.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import check_close, dev_bf16
+from synth import normal_bf16
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import moe_routed_grouped_b200 as gqe  # noqa: E402
+from moe_routed_grouped_b200.layer import GqeDecode, GqePrefill  # noqa: E402
+
+
+def _case(B, T, N, G, k, d, dm, seed, bias0=0.0):
+    M = N // G
+    c = dict(
+        x=normal_bf16((B, dm), seed),
+        W_r=normal_bf16((G, dm, M), seed + 1, std=dm ** -0.5),
+        Q=normal_bf16((B, N, d), seed + 2),
+        Qs=normal_bf16((B, d), seed + 3),
+        Kc=normal_bf16((B, T, G, d), seed + 4),
+        Vc=normal_bf16((B, T, G, d), seed + 5),
+        bias=None,
+    )
+    if bias0:
+        b = np.zeros((G, M), np.float32)
+        b[:, 0] = bias0
+        c["bias"] = b
+    return c
+
+
+def _run(shape, pos, seed, out_fp32=True, bias0=0.0):
+    B, T, N, G, k, d, dm = shape
+    c = _case(B, T, N, G, k, d, dm, seed, bias0)
+    L = GqeDecode(B, T, N, G, k, d, dm, out_fp32=out_fp32)
+    bias = None if c["bias"] is None else torch.from_numpy(c["bias"]).cuda()
+    pos_d = torch.tensor(pos, dtype=torch.int32, device="cuda")
+    L.forward(dev_bf16(c["x"]), dev_bf16(c["W_r"]), bias, dev_bf16(c["Q"]), dev_bf16(c["Qs"]),
+              dev_bf16(c["Kc"]), dev_bf16(c["Vc"]), pos_d)
+    torch.cuda.synchronize()
+    return c, L
+
+
+def _oracle(c, pos, k):
+    return oracle.gqe_decode_step(c["x"], c["W_r"], c["bias"], c["Q"], c["Qs"], c["Kc"], c["Vc"],
+                                  np.asarray(pos), k)
+
+
+# (B, T, N, G, k, d, d_model), positions.  With a short cache the chunk is
+# 256 keys: positions 255 / 256 are the last key of chunk 0 and the first of
+# chunk 1.  k = 1 runs two head slots per CTA, k >= 2 four, k = 5 (six slots
+# with the shared head) two passes.
+CASES = [
+    ((4, 700, 16, 8, 1, 64, 256), [0, 255, 256, 699]),
+    ((2, 1000, 32, 8, 2, 128, 512), [999, 517]),
+    ((3, 300, 8, 4, 2, 64, 64), [1, 299, 128]),
+    ((2, 600, 32, 4, 5, 64, 128), [599, 300]),
+    ((1, 1, 16, 8, 1, 64, 64), [0]),
+    ((2, 513, 16, 8, 1, 128, 64), [512, 511]),
+]
+
+
+@pytest.mark.parametrize("shape,pos", CASES, ids=lambda v: "x".join(map(str, v)))
+def test_decode_parity(shape, pos):
+    B, T, N, G, k, d, dm = shape
+    c, L = _run(shape, pos, seed=30000 + sum(shape))
+    assert L.device_status() == 0
+    idx, p, w, O_sel, o_bar, s = _oracle(c, pos, k)
+    assert np.array_equal(L.topk_idx.cpu().numpy(), idx), "top-k indices differ"
+    check_close(L.p.cpu().numpy(), p, "p", atol=1e-5, rtol_l2=1e-5)
+    check_close(L.w.cpu().numpy(), w, "w", atol=1e-5, rtol_l2=1e-5)
+    check_close(L.O_sel().cpu().numpy(), O_sel, "O_sel")
+    check_close(L.o_bar().cpu().numpy(), o_bar, "o_bar")
+    check_close(L.s_out().cpu().numpy(), s, "shared head")
+    if k == 1:  # w = 1 exactly, so o_bar is the selected slot bit for bit
+        assert torch.equal(L.o_bar(), L.O_sel()[:, :, 0])
+
+
+def test_decode_long_cache_many_chunks():
+    """A 40k cache: chunks longer than the minimum (several hundred keys), a
+    biased router, positions inside and at the end of the cache."""
+    shape = (2, 40000, 16, 8, 1, 64, 256)
+    pos = [39999, 12345]
+    c, L = _run(shape, pos, seed=31000, bias0=1.5)
+    assert L.device_status() == 0
+    idx, p, w, O_sel, o_bar, s = _oracle(c, pos, 1)
+    assert np.array_equal(L.topk_idx.cpu().numpy(), idx)
+    check_close(L.O_sel().cpu().numpy(), O_sel, "O_sel")
+    check_close(L.o_bar().cpu().numpy(), o_bar, "o_bar")
+    check_close(L.s_out().cpu().numpy(), s, "shared head")
+
+
+def test_decode_bf16_output():
+    shape = (2, 700, 32, 8, 2, 128, 256)
+    pos = [699, 256]
+    c, L = _run(shape, pos, seed=32000, out_fp32=False)
+    assert L.device_status() == 0
+    _, _, _, O_sel, o_bar, s = _oracle(c, pos, 2)
+    # half a bf16 ulp (2^-9 relative) on top of the float32 bound; o_bar is
+    # summed from unrounded slots, so the same bound covers it
+    for got, ref, what in ((L.O_sel(), O_sel, "O_sel"), (L.o_bar(), o_bar, "o_bar"),
+                           (L.s_out(), s, "s")):
+        g = got.float().cpu().numpy()
+        assert (np.abs(g - ref) <= 1e-2 + 2 ** -9 * np.abs(ref)).all(), what
+
+
+def test_decode_matches_prefill_rows():
+    """Decode at position t over the prefill's own K/V is prefill's row t:
+    identical routing, outputs equal within rounding (two different kernels)."""
+    B, S, N, G, k, d, dm = 2, 520, 16, 8, 2, 64, 128
+    M = N // G
+    seed = 33000
+    x = normal_bf16((B, S, dm), seed)
+    W = normal_bf16((G, dm, M), seed + 1, std=dm ** -0.5)
+    Q = normal_bf16((B, S, N, d), seed + 2)
+    Qs = normal_bf16((B, S, d), seed + 3)
+    K = normal_bf16((B, S, G, d), seed + 4)
+    V = normal_bf16((B, S, G, d), seed + 5)
+    P = GqePrefill(B, S, N, G, k, d, dm)
+    Kd, Vd, Wd = dev_bf16(K), dev_bf16(V), dev_bf16(W)
+    P.forward(dev_bf16(x), Wd, None, dev_bf16(Q), dev_bf16(Qs), Kd, Vd)
+    D = GqeDecode(B, S, N, G, k, d, dm)
+    for t in ([0, 519], [257, 3]):
+        b_ = np.arange(B)
+        tt = np.array(t)
+        D.forward(dev_bf16(x[b_, tt]), Wd, None, dev_bf16(Q[b_, tt]), dev_bf16(Qs[b_, tt]), Kd, Vd,
+                  torch.tensor(t, dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+        assert D.device_status() == 0
+        ti = torch.tensor(t, device="cuda")
+        bi = torch.arange(B, device="cuda")
+        assert torch.equal(D.topk_idx, P.topk_idx[bi, ti])
+        for a, b, what in ((D.O_sel(), P.O_sel()[bi, ti], "O_sel"),
+                           (D.o_bar(), P.o_bar()[bi, ti], "o_bar"),
+                           (D.s_out(), P.s_out()[bi, ti], "s")):
+            # prefill rounds P to fp16 for its tensor-core P.V product
+            err = (a - b).abs().max().item()
+            assert err <= 5e-3, (what, t, err)
+    assert P.device_status() == 0
+
+
+def test_decode_rejects_bad_position_and_index_on_device():
+    """Positions and expert indices live on the device, so the kernels check
+    them: an out-of-range value latches a status code, its outputs are NaN,
+    and the other sequences are unaffected."""
+    B, T, N, G, k, d, dm = 3, 300, 16, 8, 1, 64, 64
+    c = _case(B, T, N, G, k, d, dm, 34000)
+    L = GqeDecode(B, T, N, G, k, d, dm)
+    dev = {n: dev_bf16(c[n]) for n in ("x", "W_r", "Q", "Qs", "Kc", "Vc")}
+    L.route(dev["x"], dev["W_r"])
+    pos = torch.tensor([T, 5, -1], dtype=torch.int32, device="cuda")
+    L.attention(dev["Q"], dev["Qs"], dev["Kc"], dev["Vc"], pos)
+    assert L.device_status(clear=True) == 8          # GQE_ERR_BAD_POSITION
+    out = L.concat.cpu()
+    assert torch.isnan(out[0]).all() and torch.isnan(out[2]).all()
+    assert torch.isfinite(out[1]).all()
+    ref = _oracle(c, [0, 5, 0], k)
+    check_close(L.O_sel()[1].cpu().numpy(), ref[3][1], "O_sel of the valid sequence")
+
+    good = torch.tensor([7, 5, 299], dtype=torch.int32, device="cuda")
+    L.topk_idx[1, 3, 0] = N // G                     # expert index == M
+    L.attention(dev["Q"], dev["Qs"], dev["Kc"], dev["Vc"], good)
+    assert L.device_status(clear=True) == 6          # GQE_ERR_BAD_INDEX
+    assert torch.isnan(L.O_sel()[1, 3]).all() and torch.isnan(L.o_bar()[1, 3]).all()
+    assert torch.isfinite(L.O_sel()[1, :3]).all() and torch.isfinite(L.s_out()).all()
+    assert torch.isfinite(L.O_sel()[0]).all() and torch.isfinite(L.O_sel()[2]).all()
+    assert L.device_status() == 0
