@@ -13,7 +13,7 @@ collective on the data path); ranks only meet for barriers and the max-over-
 ranks of the device time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                  [--sweep] [--impl ours|reference] [--no-cpu-baseline]
+                  [--sweep] [--impl ours|reference] [--no-cpu-baseline] [--decode]
 """
 from __future__ import annotations
 
@@ -294,6 +294,70 @@ def config_of(w, world):
             "l2": "256 MiB buffer written between steps; the write is outside the step time"}
 
 
+# ----------------------------------------------------------------- decode mode
+DECODE_METRIC = "GQE decode tokens/s (one new token per sequence over a full T-token KV cache)"
+
+
+def run_decode(args, torch, w, device, rank, world, dist, peaks, peak_src, flush):
+    """One decode step per sequence of the workload, its KV cache full (T = S,
+    position T-1): gqe_route on the B new tokens, then gqe_attention_decode
+    (split-KV partials + merge).  HBM-bound: the roofline counts the cache
+    rows every step must read, K and V of all G KV heads."""
+    from moe_routed_grouped_b200.layer import GqeDecode
+    g = torch.Generator(device=device)
+    g.manual_seed(7000 + 100 * rank)
+
+    def rn(*shape, std=1.0):
+        t = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        t.normal_(0.0, std, generator=g)
+        return t
+    B, T = w.B, w.S
+    dev = dict(x=rn(B, w.d_model), W_r=rn(w.G, w.d_model, w.M, std=w.wr_std), Q=rn(B, w.N, w.d),
+               Qs=rn(B, w.d), Kc=rn(B, T, w.G, w.d), Vc=rn(B, T, w.G, w.d))
+    pos = torch.full((B,), T - 1, dtype=torch.int32, device=device)
+    L = GqeDecode(B, T, w.N, w.G, w.k, w.d, w.d_model, out_fp32=True, device=device)
+    aev = []
+
+    def step():
+        L.route(dev["x"], dev["W_r"])
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        L.attention(dev["Q"], dev["Qs"], dev["Kc"], dev["Vc"], pos)
+        b.record()
+        aev.append((a, b))
+
+    clocks = ClockSampler(device.index)
+    clocks.start()
+    step_ms, _, t0, t1 = timed_loop(torch, step, args.steps, args.warmup, flush)
+    clocks.stop()
+    torch.cuda.synchronize()
+    attn = [a.elapsed_time(b) for a, b in aev[-args.steps:]]
+    st = L.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} in the decode loop")
+    tot_ms, attn_ms = reduce_max([sum(step_ms), statistics.mean(attn)], dist, device)
+    kv_bytes = 2 * B * T * w.G * w.d * 2  # K and V rows 0..T-1 of every KV head, bf16
+    gbs = kv_bytes / (attn_ms / 1e3) / 1e9
+    line = {
+        "metric": DECODE_METRIC, "value": world * B * args.steps / (tot_ms / 1e3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 in, float32 arithmetic", "data": "synthetic",
+        "config": dict(config_of(w, world), mode="decode", T=T, position=T - 1),
+        "roofline": {"kernel": "decode_partial_kernel + decode_merge_kernel", "bound": "hbm",
+                     "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peak_src} HBM copy bandwidth",
+                     "attention_ms": attn_ms, "per_launch_bytes": kv_bytes},
+        # per step: route_prep, route, decode partial, decode merge
+        "gpu_launches": args.steps * 4,
+        "clocks": clocks.summary(t0, t1),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------- our arm
 def measure_workload(torch, w, device, rank, steps, warmup, flush, host_gen, with_attn_events):
     from moe_routed_grouped_b200.layer import GqePrefill
@@ -390,6 +454,9 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="also time the S=32k, 131k and 1M workloads (routed and dense)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time one decode step per sequence over a full cache of S tokens "
+                         "instead of the prefill (prints its own line)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -421,6 +488,12 @@ def main():
     flush = lambda: flush_buf.zero_()  # noqa: E731
 
     w = WORKLOADS[args.workload]
+    if args.decode:
+        rc = run_decode(args, torch, w, device, rank, world, dist, peaks, peak_src, flush)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return rc
     clocks = ClockSampler(local)
     clocks.start()
     barrier()
