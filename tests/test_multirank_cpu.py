@@ -50,3 +50,34 @@ def test_job_throughput_is_weak_scaling():
     # 2 ranks x 16384 tokens x 10 steps in the slowest rank's 2 ms
     assert bench.job_throughput(16384, 10, 2, 2.0) == pytest.approx(2 * 16384 * 10 / 2e-3)
     assert bench.reduce_max([1.0, 2.0], None) == [1.0, 2.0]
+
+
+def _bench(env_extra, *args):
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **env_extra)
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], cwd=root, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_line_on_cpu():
+    """The reference arm times the oracle on the host and prints the same
+    contract line, marked as the reference, with its sample described."""
+    (line,) = _bench({"RANK": "0", "WORLD_SIZE": "1"}, "--impl", "reference", "--workload",
+                     "tiny", "--steps", "2", "--warmup", "3")
+    assert line["impl"] == "reference"
+    assert line["unit"] == "tokens/s" and line["value"] > 0 and line["higher_is_better"]
+    assert line["config"]["workload"] == "tiny" and line["config"]["S"] == 128
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    assert _bench({"RANK": "1", "WORLD_SIZE": "2"}, "--impl", "reference", "--workload", "tiny",
+                  "--steps", "2", "--warmup", "3") == []
