@@ -298,11 +298,11 @@ def config_of(w, world):
 DECODE_METRIC = "GQE decode tokens/s (one new token per sequence over a full T-token KV cache)"
 
 
-def run_decode(args, torch, w, device, rank, world, dist, peaks, peak_src, flush):
+def measure_decode(torch, w, device, rank, steps, warmup, flush):
     """One decode step per sequence of the workload, its KV cache full (T = S,
     position T-1): gqe_route on the B new tokens, then gqe_attention_decode
-    (split-KV partials + merge).  HBM-bound: the roofline counts the cache
-    rows every step must read, K and V of all G KV heads."""
+    (split-KV partials + merge).  Returns this rank's step times and the mean
+    time of the decode attention (the two decode kernels) alone."""
     from moe_routed_grouped_b200.layer import GqeDecode
     g = torch.Generator(device=device)
     g.manual_seed(7000 + 100 * rank)
@@ -326,33 +326,45 @@ def run_decode(args, torch, w, device, rank, world, dist, peaks, peak_src, flush
         b.record()
         aev.append((a, b))
 
-    clocks = ClockSampler(device.index)
-    clocks.start()
-    step_ms, _, t0, t1 = timed_loop(torch, step, args.steps, args.warmup, flush)
-    clocks.stop()
+    step_ms, _, t0, t1 = timed_loop(torch, step, steps, warmup, flush)
     torch.cuda.synchronize()
-    attn = [a.elapsed_time(b) for a, b in aev[-args.steps:]]
+    attn = [a.elapsed_time(b) for a, b in aev[-steps:]]
     st = L.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} in the decode loop")
-    tot_ms, attn_ms = reduce_max([sum(step_ms), statistics.mean(attn)], dist, device)
-    kv_bytes = 2 * B * T * w.G * w.d * 2  # K and V rows 0..T-1 of every KV head, bf16
+    return dict(step_ms=step_ms, attn_ms=statistics.mean(attn), t0=t0, t1=t1,
+                kv_bytes=2 * B * T * w.G * w.d * 2)  # K and V rows 0..T-1 of every KV head
+
+
+def decode_summary(w, world, steps, tot_ms, attn_ms, kv_bytes, peaks, peak_src):
     gbs = kv_bytes / (attn_ms / 1e3) / 1e9
-    line = {
-        "metric": DECODE_METRIC, "value": world * B * args.steps / (tot_ms / 1e3),
-        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": tot_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 in, float32 arithmetic", "data": "synthetic",
-        "config": dict(config_of(w, world), mode="decode", T=T, position=T - 1),
+    return {
+        "metric": DECODE_METRIC, "value": world * w.B * steps / (tot_ms / 1e3),
+        "unit": "tokens/s", "ms_per_step": tot_ms / steps,
+        "config": dict(config_of(w, world), mode="decode", T=w.S, position=w.S - 1),
         "roofline": {"kernel": "decode_partial_kernel + decode_merge_kernel", "bound": "hbm",
                      "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": f"{peak_src} HBM copy bandwidth",
-                     "attention_ms": attn_ms, "per_launch_bytes": kv_bytes},
+                     "attention_ms": attn_ms, "per_launch_bytes": kv_bytes,
+                     "bytes_definition": "K and V cache rows 0..T-1 of all G KV heads, bf16"},
         # per step: route_prep, route, decode partial, decode merge
-        "gpu_launches": args.steps * 4,
-        "clocks": clocks.summary(t0, t1),
+        "gpu_launches": steps * 4,
     }
+
+
+def run_decode(args, torch, w, device, rank, world, dist, peaks, peak_src, flush):
+    """`--decode`: the decode step alone, as its own contract line."""
+    clocks = ClockSampler(device.index)
+    clocks.start()
+    r = measure_decode(torch, w, device, rank, args.steps, args.warmup, flush)
+    clocks.stop()
+    tot_ms, attn_ms = reduce_max([sum(r["step_ms"]), r["attn_ms"]], dist, device)
+    line = decode_summary(w, world, args.steps, tot_ms, attn_ms, r["kv_bytes"], peaks, peak_src)
+    line.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                 "dtype": "bf16 in, float32 arithmetic", "data": "synthetic",
+                 "clocks": clocks.summary(r["t0"], r["t1"])})
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -454,6 +466,8 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="also time the S=32k, 131k and 1M workloads (routed and dense)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="leave the decode-step measurements out of the prefill line")
     ap.add_argument("--decode", action="store_true",
                     help="time one decode step per sequence over a full cache of S tokens "
                          "instead of the prefill (prints its own line)")
@@ -582,6 +596,33 @@ def main():
             del r
             torch.cuda.empty_cache()
         line["sweep"] = sweep
+
+    if world == 1 and not args.no_decode:
+        # the decode step (one new token per sequence over a full cache) at the
+        # bench's own shape and over a 1M-token cache; a failure here is
+        # reported in the line and leaves the prefill numbers above standing
+        if "res" in locals():
+            del res
+        torch.cuda.empty_cache()
+        dec = []
+        for name in ("layer250m", "million"):
+            wd = WORKLOADS[name]
+            cs = ClockSampler(local)
+            cs.start()
+            try:
+                r = measure_decode(torch, wd, device, rank, 20, 3, flush)
+                cs.stop()
+                e = decode_summary(wd, world, 20, sum(r["step_ms"]), r["attn_ms"], r["kv_bytes"],
+                                   peaks, peak_src)
+                e.update(workload=name, steps=20, warmup=3, clocks=cs.summary(r["t0"], r["t1"]))
+                dec.append(e)
+                del r
+            except Exception as ex:  # noqa: BLE001
+                dec.append({"workload": name, "error": f"{type(ex).__name__}: {ex}"[:300]})
+            finally:
+                cs.stop()
+            torch.cuda.empty_cache()
+        line["decode"] = dec
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = make_inputs(w)
