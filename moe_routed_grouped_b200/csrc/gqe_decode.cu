@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const De
   for (int qi = threadIdx.x; qi < HB * D; qi += kDecThreads) {
     const int h = qi / D, e = qi % D;
     const int j = pass * HB + h;
-    bool use = false;
+    bool use = false;  // live[h], read with constant indices so live[] stays in registers
 #pragma unroll
     for (int hh = 0; hh < HB; ++hh)
       if (hh == h) use = live[hh];
