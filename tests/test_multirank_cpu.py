@@ -81,3 +81,18 @@ def test_reference_arm_line_on_cpu():
 def test_reference_arm_other_ranks_exit_quietly():
     assert _bench({"RANK": "1", "WORLD_SIZE": "2"}, "--impl", "reference", "--workload", "tiny",
                   "--steps", "2", "--warmup", "3") == []
+
+
+def test_decode_summary_counts_cache_bytes():
+    """The decode roofline divides the cache bytes a step must read (K and V
+    rows of every KV head, bf16) by the decode kernels' time."""
+    from synth import WORKLOADS
+    w = WORKLOADS["million"]
+    kv = 2 * w.B * w.S * w.G * w.d * 2
+    assert kv == 2 * 2 ** 30                       # 1M tokens x 8 heads x 64 x (K, V) x 2 B
+    s = bench.decode_summary(w, 1, 20, 20 * 0.5, 0.4, kv, {"hbm_gbs": 6650.0}, "measured")
+    assert s["value"] == pytest.approx(1 * 20 / (10.0 / 1e3))   # B = 1 token per step
+    assert s["roofline"]["achieved"] == pytest.approx(kv / 0.4e-3 / 1e9)
+    assert s["roofline"]["frac"] == pytest.approx(kv / 0.4e-3 / 1e9 / 6650.0)
+    assert s["roofline"]["bound"] == "hbm" and s["gpu_launches"] == 80
+    assert s["config"]["mode"] == "decode" and s["config"]["position"] == w.S - 1
