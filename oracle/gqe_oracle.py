@@ -72,9 +72,14 @@ def _scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
 
 
-def _visible(key_pos: np.ndarray, query_pos: np.ndarray) -> np.ndarray:
-    """[GQA article] 工程实操 step 1: a key is visible iff key pos <= query pos."""
-    return key_pos[None, :] <= query_pos[:, None]
+def _visible(key_pos: np.ndarray, query_pos: np.ndarray, key_start=None) -> np.ndarray:
+    """[GQA article] 工程实操 step 1: a key is visible iff key pos <= query pos.
+    With padding (step 4) the causal condition is intersected with key
+    validity: here the valid keys of a row are slots key_start..query pos."""
+    vis = key_pos[None, :] <= query_pos[:, None]
+    if key_start is not None:
+        vis &= key_pos[None, :] >= key_start[:, None]
+    return vis
 
 
 # ---------------------------------------------------------------------------
@@ -228,18 +233,22 @@ def bucket(topk_idx: np.ndarray, M: int) -> Tuple[np.ndarray, np.ndarray]:
 # ---------------------------------------------------------------------------
 
 def causal_attention(q: np.ndarray, pos: np.ndarray, K: np.ndarray, V: np.ndarray,
-                     dtype=np.float64, row_chunk: int = 0) -> np.ndarray:
+                     dtype=np.float64, row_chunk: int = 0, key_start=None) -> np.ndarray:
     """Softmax attention of query rows at absolute positions ``pos``.
 
     o_r = sum_{t <= pos_r} softmax_t(q_r . K_t / sqrt(d)) V_t.
     [GQA article] 最小参考实现 (scaled dot product, softmax, times V) and
-    工程实操 (mask by absolute position, not by a top-left triangle).
+    工程实操 (mask by absolute position, not by a top-left triangle).  With
+    ``key_start`` (one per row; padding, 工程实操 step 4) the sum runs over
+    key_start_r <= t <= pos_r only.
     Rows are independent; they are processed in chunks only to bound memory.
     """
     q = np.asarray(q, dtype=dtype)
     K = np.asarray(K, dtype=dtype)
     V = np.asarray(V, dtype=dtype)
     pos = np.asarray(pos, dtype=np.int64)
+    if key_start is not None:
+        key_start = np.asarray(key_start, dtype=np.int64)
     R, d = q.shape
     out = np.empty((R, V.shape[1]), dtype=dtype)
     sc = dtype(_scale(d))
@@ -250,7 +259,8 @@ def causal_attention(q: np.ndarray, pos: np.ndarray, K: np.ndarray, V: np.ndarra
         pm = int(pos[s:e].max())
         keys = np.arange(pm + 1)
         sco = (q[s:e] @ K[: pm + 1].T) * sc
-        sco = np.where(_visible(keys, pos[s:e]), sco, -np.inf)
+        ks = None if key_start is None else key_start[s:e]
+        sco = np.where(_visible(keys, pos[s:e], ks), sco, -np.inf)
         mx = sco.max(axis=1, keepdims=True)
         p = np.exp(sco - mx)
         out[s:e] = (p @ V[: pm + 1]) / p.sum(axis=1, keepdims=True)
@@ -304,7 +314,7 @@ def gqe_prefill_rows(Q_bits, Qs_bits, K_bits, V_bits, topk_idx, w, rows, dtype=n
 
 
 def gqe_decode_step(x_bits, Wr_bits, bias, Q_bits, Qs_bits, Kc_bits, Vc_bits, pos, k,
-                    dtype=np.float64):
+                    dtype=np.float64, kv_start=None):
     """One incremental decode step of GQE, for each sequence b of a batch.
 
     [GQA article] 工程实操 非方形因果遮罩: at an incremental decode step the query
@@ -315,8 +325,11 @@ def gqe_decode_step(x_bits, Wr_bits, bias, Q_bits, Qs_bits, Kc_bits, Vc_bits, po
     routes as in prefill ([GQE review] §二 路由器), each selected head attends
     with its group's KV head, the shared head with KV head 0, and ō is the
     weighted sum of the slots (三个关键部件).  x [B, dm], Q [B, N, d], Qs [B, d]
-    are bf16 bit patterns.  Returns (topk_idx [B,G,k], p [B,G,M], w [B,G,k],
-    O_sel [B,G,k,d], o_bar [B,G,d], s [B,d]).
+    are bf16 bit patterns.  ``kv_start`` [B] (padding, 工程实操 step 4: causal
+    condition intersected with key validity) makes slots before kv_start[b]
+    invalid: sequence b then sees slots kv_start[b]..pos[b].  Returns
+    (topk_idx [B,G,k], p [B,G,M], w [B,G,k], O_sel [B,G,k,d], o_bar [B,G,d],
+    s [B,d]).
     """
     B = x_bits.shape[0]
     idx, p, w, _ = route(np.asarray(x_bits)[:, None, :], Wr_bits, bias, k)
@@ -329,16 +342,18 @@ def gqe_decode_step(x_bits, Wr_bits, bias, Q_bits, Qs_bits, Kc_bits, Vc_bits, po
     s_out = np.zeros((B, d), dtype=dtype)
     for b in range(B):
         r = np.array([int(pos[b])])
+        ks = None if kv_start is None else np.array([int(kv_start[b])])
         Kb, Vb = bf16_to_f64(Kc_bits[b]), bf16_to_f64(Vc_bits[b])
         for g in range(G):
             for j in range(k):
                 h = _expert_head(g, int(idx[b, g, j]), M)
                 q = bf16_to_f64(Q_bits[b, h])[None, :]
-                O_sel[b, g, j] = causal_attention(q, r, Kb[:, g], Vb[:, g], dtype=dtype)[0]
+                O_sel[b, g, j] = causal_attention(q, r, Kb[:, g], Vb[:, g], dtype=dtype,
+                                                  key_start=ks)[0]
         for j in range(k):  # ascending slot order
             o_bar[b] = o_bar[b] + np.asarray(w[b, :, j, None], dtype=dtype) * O_sel[b, :, j]
         s_out[b] = causal_attention(bf16_to_f64(Qs_bits[b])[None, :], r, Kb[:, 0], Vb[:, 0],
-                                    dtype=dtype)[0]
+                                    dtype=dtype, key_start=ks)[0]
     return idx, p, w, O_sel, o_bar, s_out
 
 

@@ -143,6 +143,55 @@ def test_nonsquare_causal_positions():
     check_nonsquare_positions()
 
 
+def check_padding_key_validity():
+    """[GQA article] 工程实操 step 4: with padding the visible keys are the
+    intersection of the causal condition and key validity.  Identical keys
+    make the weights uniform over exactly the visible slots, so the output is
+    the mean of V over key_start..pos (one-hot V rows show which slots);
+    key_start = pos leaves one key, whose V comes back exactly."""
+    n = 9
+    q = np.ones((4, 8))
+    K = np.ones((n, 8))
+    V = np.eye(n)
+    pos = np.array([8, 8, 5, 3])
+    start = np.array([0, 3, 5, 1])
+    o = oracle.causal_attention(q, pos, K, V, key_start=start)
+    for r in range(4):
+        nv = pos[r] - start[r] + 1
+        want = np.zeros(n)
+        want[start[r]: pos[r] + 1] = 1.0 / nv
+        assert np.allclose(o[r], want, atol=1e-15, rtol=0), (r, o[r])
+    assert np.array_equal(o[2], V[5])
+
+
+def test_padding_key_validity():
+    check_padding_key_validity()
+
+
+def test_left_padded_decode_equals_unpadded():
+    """A sequence stored at cache slots s..s+n-1 behind s padding slots (any
+    finite garbage there) decodes, with kv_start = s, exactly as the same
+    sequence stored from slot 0."""
+    B, n, s, N, G, k, d, dm = 2, 23, 7, 8, 4, 2, 16, 32
+    x = normal_bf16((B, dm), 19200)
+    W = normal_bf16((G, dm, N // G), 19201, std=dm ** -0.5)
+    Q = normal_bf16((B, N, d), 19202)
+    Qs = normal_bf16((B, d), 19203)
+    K = normal_bf16((B, n, G, d), 19204)
+    V = normal_bf16((B, n, G, d), 19205)
+    pad = f32_to_bf16_bits(np.full((B, s, G, d), 2.5e3, np.float32))
+    Kp, Vp = np.concatenate([pad, K], axis=1), np.concatenate([-pad, V], axis=1)
+    pos = np.array([n - 1, 10])
+    ref = oracle.gqe_decode_step(x, W, None, Q, Qs, K, V, pos, k)
+    got = oracle.gqe_decode_step(x, W, None, Q, Qs, Kp, Vp, pos + s, k,
+                                 kv_start=np.array([s, s]))
+    for a_, b_ in zip(ref, got):
+        assert np.allclose(a_, b_, rtol=1e-12, atol=1e-12)
+    # without the validity bound the padding would be attended
+    bad = oracle.gqe_decode_step(x, W, None, Q, Qs, Kp, Vp, pos + s, k)
+    assert not np.allclose(bad[3], ref[3], atol=1e-3)
+
+
 def check_head_to_kv_map():
     """8 query heads, 2 KV heads: heads 0-3 read KV 0, heads 4-7 read KV 1.
     KV heads are made numerically distinct (GQA article: make KV heads differ
@@ -530,7 +579,7 @@ ALL_CHECKS = [check_kv_bytes, check_worked_examples, check_worked_example_routed
               check_geometric_scores, check_nonsquare_positions, check_head_to_kv_map,
               check_row0_and_hull, check_explicit_equals_repeat, check_router_sums,
               check_routed_kM_equals_dense, check_shared_head_is_dense_head_on_kv0,
-              check_k1_obar, check_obar_weighted_sum_k2]
+              check_k1_obar, check_obar_weighted_sum_k2, check_padding_key_validity]
 
 
 def _caught(monkeypatch, name, fn):
@@ -545,8 +594,11 @@ def _caught(monkeypatch, name, fn):
 
 
 @pytest.mark.parametrize("name,fn", [
-    ("_visible", lambda k, q: k[None, :] < q[:, None]),             # diagonal dropped
-    ("_visible", lambda k, q: k[None, :] <= q[:, None] + 1),        # one key of the future
+    ("_visible", lambda k, q, s=None: k[None, :] < q[:, None]),       # diagonal dropped
+    ("_visible", lambda k, q, s=None: k[None, :] <= q[:, None] + 1),  # one key of the future
+    ("_visible", lambda k, q, s=None: k[None, :] <= q[:, None]),      # padding ignored
+    ("_visible", lambda k, q, s=None: (k[None, :] <= q[:, None]) &    # first valid key dropped
+     (True if s is None else k[None, :] > s[:, None])),
     ("_scale", lambda d: 1.0),                                      # scale dropped
     ("_scale", lambda d: 1.0 / d),                                  # wrong scale
     ("_kv_head_of", lambda h, N, G: h % G),                         # interleaved map
