@@ -199,22 +199,27 @@ size_t gqe_decode_workspace_size(const gqe_dims* dims);
  *  Kc, Vc   device bf16 [B, T, G, d]  caches; slot pos[b] must already hold
  *           the new token's K and V (the append is the caller's copy)
  *  pos      device int32 [B]          0 <= pos[b] < T, may differ per b
+ *  kv_start device int32 [B] or NULL: first valid cache slot of sequence b
+ *           (left padding; 工程实操 step 4: the causal condition is
+ *           intersected with key validity), 0 <= kv_start[b] <= pos[b];
+ *           sequence b then sees slots kv_start[b]..pos[b].  NULL = all 0.
  *  topk_idx device int32 [B, G, k]; w device fp32 [B, G, k]: gqe_route with
  *           dims S = 1 on the new tokens' x
  *  O_sel, o_bar, s_out, out_row_stride: as for gqe_attention_prefill, one
  *           output row per sequence b.
- * Output element type: float32 if dims->out_fp32 else bf16.  A position out
- * of range latches GQE_ERR_BAD_POSITION and that sequence's outputs are NaN;
- * an expert index out of range latches GQE_ERR_BAD_INDEX and its slot and
- * o_bar are NaN.  The cache is read once per step: each CTA serves every
+ * Output element type: float32 if dims->out_fp32 else bf16.  A position or
+ * first slot out of range latches GQE_ERR_BAD_POSITION and that sequence's
+ * outputs are NaN; an expert index out of range latches GQE_ERR_BAD_INDEX
+ * and its slot and o_bar are NaN.  The cache is read once per step: each CTA serves every
  * selected head of its KV head (and the shared head for KV head 0) over one
  * chunk of keys, and a second kernel merges the chunks.
  */
 gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void* Qs,
                                 const void* Kc, const void* Vc, const int32_t* pos,
-                                const int32_t* topk_idx, const float* w, void* O_sel,
-                                void* o_bar, void* s_out, int64_t out_row_stride, void* ws,
-                                size_t ws_bytes, void* stream);
+                                const int32_t* kv_start, const int32_t* topk_idx,
+                                const float* w, void* O_sel, void* o_bar, void* s_out,
+                                int64_t out_row_stride, void* ws, size_t ws_bytes,
+                                void* stream);
 
 /* Synchronises `stream`, then returns the status word latched in `ws`
  * (GQE_OK if no device-side error was recorded).  If `clear` is non-zero the

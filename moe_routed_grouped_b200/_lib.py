@@ -57,7 +57,7 @@ def _load() -> ctypes.CDLL:
         "gqe_attention_prefill_static": (I32, [S, P, P, P, P, P, P, P, P, P, I64, P]),
         "gqe_set_pair_threshold": (I64, [I64]),
         "gqe_decode_workspace_size": (SZ, [S]),
-        "gqe_attention_decode": (I32, [S, P, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
+        "gqe_attention_decode": (I32, [S, P, P, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -163,11 +163,12 @@ def gqe_decode_workspace_size(dm: GqeDims) -> int:
     return LIB.gqe_decode_workspace_size(ctypes.byref(dm))
 
 
-def gqe_attention_decode(dm, Q, Qs, Kc, Vc, pos, topk_idx, w, O_sel, o_bar, s_out,
+def gqe_attention_decode(dm, Q, Qs, Kc, Vc, pos, kv_start, topk_idx, w, O_sel, o_bar, s_out,
                          out_row_stride, ws, stream=None, check=True):
-    """One decode step; dm.S is the cache capacity T."""
+    """One decode step; dm.S is the cache capacity T; kv_start may be None."""
     r = LIB.gqe_attention_decode(ctypes.byref(dm), _ptr(Q), _ptr(Qs), _ptr(Kc), _ptr(Vc),
-                                 _ptr(pos), _ptr(topk_idx), _ptr(w), _ptr(O_sel), _ptr(o_bar),
+                                 _ptr(pos), _ptr(kv_start), _ptr(topk_idx), _ptr(w), _ptr(O_sel),
+                                 _ptr(o_bar),
                                  _ptr(s_out), int(out_row_stride), _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream))
     return _check(r, "gqe_attention_decode") if check else r

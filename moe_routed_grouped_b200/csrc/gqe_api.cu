@@ -300,14 +300,15 @@ size_t gqe_decode_workspace_size(const gqe_dims* dims) {
 
 gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void* Qs,
                                 const void* Kc, const void* Vc, const int32_t* pos,
-                                const int32_t* topk_idx, const float* w, void* O_sel,
-                                void* o_bar, void* s_out, int64_t out_row_stride, void* ws,
-                                size_t ws_bytes, void* stream) {
+                                const int32_t* kv_start, const int32_t* topk_idx,
+                                const float* w, void* O_sel, void* o_bar, void* s_out,
+                                int64_t out_row_stride, void* ws, size_t ws_bytes,
+                                void* stream) {
   gqe_status st = check_dims(dims, false);
   if (st != GQE_OK) return st;
   if (!aligned16(Q) || !aligned16(Qs) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(pos) ||
       !aligned16(topk_idx) || !aligned16(w) || !aligned16(O_sel) || !aligned16(o_bar) ||
-      !aligned16(s_out))
+      !aligned16(s_out) || (kv_start && !aligned16(kv_start)))
     return GQE_ERR_INVALID_ARG;
   if (out_row_stride < dims->d || out_row_stride % 8 != 0) return GQE_ERR_INVALID_ARG;
   const DecodePlan P = make_decode_plan(*dims);
@@ -319,6 +320,7 @@ gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void*
   a.Kc = static_cast<const uint16_t*>(Kc);
   a.Vc = static_cast<const uint16_t*>(Vc);
   a.pos = pos;
+  a.kv_start = kv_start;
   a.topk_idx = topk_idx;
   a.w = w;
   a.part_m = reinterpret_cast<float*>(wb + P.part_m);

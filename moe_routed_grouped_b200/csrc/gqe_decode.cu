@@ -1,6 +1,8 @@
 // Incremental decode step of GQE: one new token per sequence attends its
 // cached history ("AI 大模型之 GQA", 工程实操 非方形因果遮罩: query length 1,
-// key length the whole history, mask on the absolute position).
+// key length the whole history, mask on the absolute position; with padding
+// the mask is intersected with key validity, here a first valid slot per
+// sequence for left-padded caches).
 //
 // A decode step reads every cached K/V row of each KV head once and does
 // little arithmetic with it, so it is bound by HBM bandwidth, not by the
@@ -72,15 +74,18 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const De
   const int g = static_cast<int>(unit % a.G);
   const int b = static_cast<int>(unit / a.G);
 
+  // visible keys of sequence b: slots lo..pos (lo > 0 with left padding)
   const int pos = a.pos[b];
-  if (pos < 0 || pos >= a.T) {
+  const int lo = a.kv_start ? a.kv_start[b] : 0;
+  if (pos < 0 || pos >= a.T || lo < 0 || lo > pos) {
     if (threadIdx.x == 0 && c == 0 && pass == 0 && g == 0)
       latch_status(a.status, GQE_ERR_BAD_POSITION);
     return;
   }
-  const int64_t t0 = static_cast<int64_t>(c) * a.chunk;
-  if (t0 > pos) return;  // no visible key in this chunk; the merge stops before it
-  const int64_t t1 = min(t0 + a.chunk, static_cast<int64_t>(pos) + 1);
+  const int64_t c0 = static_cast<int64_t>(c) * a.chunk;
+  if (c0 > pos || c0 + a.chunk <= lo) return;  // no visible key here; the merge skips it
+  const int64_t t0 = max(c0, static_cast<int64_t>(lo));
+  const int64_t t1 = min(c0 + a.chunk, static_cast<int64_t>(pos) + 1);
 
   // this pass's head slots: j < k routed (head g*M + topk_idx), j == k the
   // shared head (KV head 0 only); a slot that is not live is skipped
@@ -213,7 +218,8 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const De
 }
 
 // Merge of the chunks of one (b, g): for each live head slot, rescale every
-// chunk that holds visible keys to the common maximum, add, normalise; then
+// chunk that holds visible keys (those the partial kernel wrote) to the
+// common maximum, add, normalise; then
 // o_bar = sum_j w_j * O_j in slot order (review §二 三个关键部件) and the
 // shared head for g = 0.  One thread per output element.
 template <int D>
@@ -223,8 +229,10 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
   const int g = static_cast<int>(bg % a.G);
   const int e = threadIdx.x;
   const int pos = a.pos[b];
-  const bool pos_ok = pos >= 0 && pos < a.T;
-  const int nc = pos_ok ? pos / a.chunk + 1 : 0;  // chunks with visible keys
+  const int lo = a.kv_start ? a.kv_start[b] : 0;
+  const bool pos_ok = pos >= 0 && pos < a.T && lo >= 0 && lo <= pos;
+  const int c_lo = pos_ok ? lo / a.chunk : 0;     // chunks c_lo .. nc-1 hold visible keys
+  const int nc = pos_ok ? pos / a.chunk + 1 : 0;
   const int nh = a.k + (g == 0 ? 1 : 0);
   const float nan = __int_as_float(0x7fc00000);
   const int64_t r = static_cast<int64_t>(b) * a.out_row_stride;
@@ -239,9 +247,9 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
     if (ok) {
       const int64_t p0 = (bg * a.heads + j) * a.nchunks;
       float mx = kNoKeyMax;
-      for (int c = 0; c < nc; ++c) mx = fmaxf(mx, a.part_m[p0 + c]);
+      for (int c = c_lo; c < nc; ++c) mx = fmaxf(mx, a.part_m[p0 + c]);
       float acc = 0.f, lsum = 0.f;
-      for (int c = 0; c < nc; ++c) {
+      for (int c = c_lo; c < nc; ++c) {
         const float sc = exp2f(a.part_m[p0 + c] - mx);
         acc = fmaf(a.part_o[(p0 + c) * D + e], sc, acc);
         lsum = fmaf(a.part_l[p0 + c], sc, lsum);

@@ -214,6 +214,7 @@ struct DecodeArgs {
   const uint16_t* Kc;   // bf16 [B, T, G, d]
   const uint16_t* Vc;   // bf16 [B, T, G, d]
   const int32_t* pos;   // [B]
+  const int32_t* kv_start;  // [B] first valid slot, or null (0)
   const int32_t* topk_idx;  // [B, G, k]
   const float* w;           // [B, G, k]
   float* part_m;        // [B, G, heads, nchunks]: running max (log2 units)

@@ -127,18 +127,19 @@ class GqeDecode:
                        stream)
         return self.topk_idx, self.p, self.w
 
-    def attention(self, Q, Qs, Kc, Vc, pos, stream=None):
-        """Q [B, N, d], Qs [B, d], caches [B, T, G, d] (bf16), pos int32 [B]."""
+    def attention(self, Q, Qs, Kc, Vc, pos, kv_start=None, stream=None):
+        """Q [B, N, d], Qs [B, d], caches [B, T, G, d] (bf16), pos int32 [B];
+        kv_start int32 [B] (first valid slot, left padding) or None."""
         a = self.G * self.k * self.d
         flat = self.concat.view(-1)
-        _lib.gqe_attention_decode(self.dims, Q, Qs, Kc, Vc, pos, self.topk_idx, self.w,
-                                  self.concat, flat[a:], flat[a + self.G * self.d:], self.row,
-                                  self.ws, stream)
+        _lib.gqe_attention_decode(self.dims, Q, Qs, Kc, Vc, pos, kv_start, self.topk_idx,
+                                  self.w, self.concat, flat[a:], flat[a + self.G * self.d:],
+                                  self.row, self.ws, stream)
         return self.concat
 
-    def forward(self, x, W_r, bias, Q, Qs, Kc, Vc, pos, stream=None):
+    def forward(self, x, W_r, bias, Q, Qs, Kc, Vc, pos, kv_start=None, stream=None):
         self.route(x, W_r, bias, stream)
-        return self.attention(Q, Qs, Kc, Vc, pos, stream)
+        return self.attention(Q, Qs, Kc, Vc, pos, kv_start, stream)
 
     def device_status(self, clear=True, stream=None) -> int:
         return _lib.gqe_get_device_status(self.ws, 1 if clear else 0, stream)

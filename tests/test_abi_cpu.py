@@ -120,12 +120,13 @@ def test_decode_rejects_bad_arguments():
     need = _lib.gqe_decode_workspace_size(dm)
     assert need > 512
 
-    def call(stride=17 * 64, ws_bytes=1 << 40, pos=FAKE, d=dm):
-        return L.gqe_attention_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, pos, FAKE, FAKE,
-                                      FAKE, FAKE, FAKE, stride, FAKE, ws_bytes, None)
+    def call(stride=17 * 64, ws_bytes=1 << 40, pos=FAKE, d=dm, start=None):
+        return L.gqe_attention_decode(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, pos, start, FAKE,
+                                      FAKE, FAKE, FAKE, FAKE, stride, FAKE, ws_bytes, None)
     assert call(stride=60) == 1                      # not a multiple of 8
     assert call(pos=None) == 1                       # positions are required
     assert call(pos=ctypes.c_void_p(0x10004)) == 1   # misaligned
+    assert call(start=ctypes.c_void_p(0x10004)) == 1  # misaligned first-slot array
     assert call(ws_bytes=need - 1) == 5
     assert call(d=_lib.dims(2, 4096, 16, 8, 3, 64)) == 1   # k > M
     assert call(d=_lib.dims(2, 4096, 16, 8, 1, 96)) == 2   # head dim outside {64, 128}

@@ -41,21 +41,23 @@ def _case(B, T, N, G, k, d, dm, seed, bias0=0.0):
     return c
 
 
-def _run(shape, pos, seed, out_fp32=True, bias0=0.0):
+def _run(shape, pos, seed, out_fp32=True, bias0=0.0, kv_start=None):
     B, T, N, G, k, d, dm = shape
     c = _case(B, T, N, G, k, d, dm, seed, bias0)
     L = GqeDecode(B, T, N, G, k, d, dm, out_fp32=out_fp32)
     bias = None if c["bias"] is None else torch.from_numpy(c["bias"]).cuda()
     pos_d = torch.tensor(pos, dtype=torch.int32, device="cuda")
+    ks_d = None if kv_start is None else torch.tensor(kv_start, dtype=torch.int32, device="cuda")
     L.forward(dev_bf16(c["x"]), dev_bf16(c["W_r"]), bias, dev_bf16(c["Q"]), dev_bf16(c["Qs"]),
-              dev_bf16(c["Kc"]), dev_bf16(c["Vc"]), pos_d)
+              dev_bf16(c["Kc"]), dev_bf16(c["Vc"]), pos_d, ks_d)
     torch.cuda.synchronize()
     return c, L
 
 
-def _oracle(c, pos, k):
+def _oracle(c, pos, k, kv_start=None):
     return oracle.gqe_decode_step(c["x"], c["W_r"], c["bias"], c["Q"], c["Qs"], c["Kc"], c["Vc"],
-                                  np.asarray(pos), k)
+                                  np.asarray(pos), k,
+                                  kv_start=None if kv_start is None else np.asarray(kv_start))
 
 
 # (B, T, N, G, k, d, d_model), positions.  With a short cache the chunk is
@@ -96,6 +98,29 @@ def test_decode_long_cache_many_chunks():
     c, L = _run(shape, pos, seed=31000, bias0=1.5)
     assert L.device_status() == 0
     idx, p, w, O_sel, o_bar, s = _oracle(c, pos, 1)
+    assert np.array_equal(L.topk_idx.cpu().numpy(), idx)
+    check_close(L.O_sel().cpu().numpy(), O_sel, "O_sel")
+    check_close(L.o_bar().cpu().numpy(), o_bar, "o_bar")
+    check_close(L.s_out().cpu().numpy(), s, "shared head")
+
+
+# left padding: (shape, positions, first valid slots); the first slot falls
+# inside a chunk, on a chunk edge (256), at 0, and equal to the position
+PADDED = [
+    ((4, 700, 16, 8, 1, 64, 256), [699, 300, 40, 600], [200, 0, 40, 256]),
+    ((2, 1000, 32, 8, 2, 128, 512), [999, 517], [255, 1]),
+    ((3, 600, 32, 4, 5, 64, 128), [599, 300, 512], [511, 299, 512]),
+]
+
+
+@pytest.mark.parametrize("shape,pos,kv_start", PADDED, ids=lambda v: "x".join(map(str, v)))
+def test_decode_left_padding_parity(shape, pos, kv_start):
+    """The causal condition intersected with key validity: sequence b sees
+    slots kv_start[b]..pos[b] only."""
+    B, T, N, G, k, d, dm = shape
+    c, L = _run(shape, pos, seed=35000 + B + T, kv_start=kv_start)
+    assert L.device_status() == 0
+    idx, p, w, O_sel, o_bar, s = _oracle(c, pos, k, kv_start)
     assert np.array_equal(L.topk_idx.cpu().numpy(), idx)
     check_close(L.O_sel().cpu().numpy(), O_sel, "O_sel")
     check_close(L.o_bar().cpu().numpy(), o_bar, "o_bar")
@@ -168,6 +193,15 @@ def test_decode_rejects_bad_position_and_index_on_device():
     assert torch.isfinite(out[1]).all()
     ref = _oracle(c, [0, 5, 0], k)
     check_close(L.O_sel()[1].cpu().numpy(), ref[3][1], "O_sel of the valid sequence")
+
+    # a first valid slot after the position is rejected the same way
+    L.attention(dev["Q"], dev["Qs"], dev["Kc"], dev["Vc"],
+                torch.tensor([7, 5, 9], dtype=torch.int32, device="cuda"),
+                torch.tensor([0, 6, 0], dtype=torch.int32, device="cuda"))
+    assert L.device_status(clear=True) == 8
+    out = L.concat.cpu()
+    assert torch.isnan(out[1]).all() and torch.isfinite(out[0]).all()
+    assert torch.isfinite(out[2]).all()
 
     good = torch.tensor([7, 5, 299], dtype=torch.int32, device="cuda")
     L.topk_idx[1, 3, 0] = N // G                     # expert index == M
