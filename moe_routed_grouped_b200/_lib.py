@@ -74,8 +74,13 @@ def _ptr(t):
 
 
 def _stream(stream):
-    return ctypes.c_void_p(stream if isinstance(stream, int) else
-                           (0 if stream is None else stream.cuda_stream))
+    """A cudaStream_t: an int handle, a torch.cuda.Stream, or None for torch's
+    current stream on the current device (so calls order with the caller's
+    torch work and can be captured into a CUDA graph)."""
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return ctypes.c_void_p(stream if isinstance(stream, int) else stream.cuda_stream)
 
 
 def _check(code: int, where: str) -> int:

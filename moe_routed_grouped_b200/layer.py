@@ -141,5 +141,23 @@ class GqeDecode:
         self.route(x, W_r, bias, stream)
         return self.attention(Q, Qs, Kc, Vc, pos, kv_start, stream)
 
+    def graph(self, x, W_r, bias, Q, Qs, Kc, Vc, pos, kv_start=None, warmup=2):
+        """Capture one decode step (router + attention: four kernel launches)
+        on these tensors into a torch.cuda.CUDAGraph.  Each replay re-runs the
+        step on what the tensors then hold: copy the next tokens' x, Q, Qs and
+        positions (and the new cache rows) into them, then replay.  Outputs
+        land in this object's buffers (``concat``, ``topk_idx``, ``p``, ``w``)."""
+        cur = torch.cuda.current_stream(self.device)
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(cur)
+        with torch.cuda.stream(side):  # warm-up outside the capture (one-time setup)
+            for _ in range(warmup):
+                self.forward(x, W_r, bias, Q, Qs, Kc, Vc, pos, kv_start)
+        cur.wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.forward(x, W_r, bias, Q, Qs, Kc, Vc, pos, kv_start)
+        return g
+
     def device_status(self, clear=True, stream=None) -> int:
         return _lib.gqe_get_device_status(self.ws, 1 if clear else 0, stream)

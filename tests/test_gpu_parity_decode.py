@@ -211,3 +211,29 @@ def test_decode_rejects_bad_position_and_index_on_device():
     assert torch.isfinite(L.O_sel()[1, :3]).all() and torch.isfinite(L.s_out()).all()
     assert torch.isfinite(L.O_sel()[0]).all() and torch.isfinite(L.O_sel()[2]).all()
     assert L.device_status() == 0
+
+
+def test_decode_step_replays_as_a_cuda_graph():
+    """A captured decode step (router + attention) replayed on new tokens and
+    positions gives the same bits as the eager calls on the same inputs."""
+    B, T, N, G, k, d, dm = 2, 600, 16, 8, 2, 64, 128
+    c = _case(B, T, N, G, k, d, dm, 36000)
+    st = {n: dev_bf16(c[n]) for n in ("x", "W_r", "Q", "Qs", "Kc", "Vc")}
+    pos = torch.tensor([599, 0], dtype=torch.int32, device="cuda")
+    L = GqeDecode(B, T, N, G, k, d, dm)
+    g = L.graph(st["x"], st["W_r"], None, st["Q"], st["Qs"], st["Kc"], st["Vc"], pos)
+    E = GqeDecode(B, T, N, G, k, d, dm)
+    for i, p_ in enumerate(([10, 599], [300, 3], [599, 599])):
+        nxt = _case(B, T, N, G, k, d, dm, 36100 + 10 * i)
+        for n in ("x", "Q", "Qs"):
+            st[n].copy_(dev_bf16(nxt[n]))
+        pos.copy_(torch.tensor(p_, dtype=torch.int32))
+        g.replay()
+        E.forward(st["x"], st["W_r"], None, st["Q"], st["Qs"], st["Kc"], st["Vc"], pos)
+        torch.cuda.synchronize()
+        assert torch.equal(L.topk_idx, E.topk_idx)
+        assert torch.equal(L.concat, E.concat), p_
+        ref = oracle.gqe_decode_step(nxt["x"], c["W_r"], None, nxt["Q"], nxt["Qs"], c["Kc"],
+                                     c["Vc"], np.asarray(p_), k)
+        check_close(L.O_sel().cpu().numpy(), ref[3], "O_sel (graph)")
+    assert L.device_status() == 0 and E.device_status() == 0
