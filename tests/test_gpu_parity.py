@@ -231,3 +231,25 @@ def test_bf16_output_mode_d128():
                            (L.s_out(), s, "s")):
         g = got.float().cpu().numpy()
         assert (np.abs(g - ref) <= 1e-2 + 2 ** -8 * np.abs(ref)).all(), what
+
+
+def test_right_padded_batch_rows_are_exact():
+    """Right padding ([GQA article] 工程实操 step 4): a valid row i < len_b
+    sees keys t <= i < len_b only, so the causal mask already implies key
+    validity and the padded tail (garbage tokens, routed like any other)
+    cannot reach it.  Each sequence's valid rows equal the oracle on that
+    sequence cut to its length."""
+    shape = (3, 300, 16, 8, 2, 64, 64)
+    B, S, N, G, k, d, dm = shape
+    lens = [300, 177, 1]
+    inp, L = _run(shape, seed=18500)
+    go, gb, gs = L.O_sel().cpu().numpy(), L.o_bar().cpu().numpy(), L.s_out().cpu().numpy()
+    gi = L.topk_idx.cpu().numpy()
+    for b, n in enumerate(lens):
+        cut = {key: inp[key][b:b + 1, :n] for key in ("x", "Q", "Qs", "K", "V")}
+        idx, p, w, _ = oracle.route(cut["x"], inp["W_r"], None, k)
+        assert np.array_equal(gi[b:b + 1, :n], idx)
+        O_sel, o_bar, s = oracle.gqe_prefill(cut["Q"], cut["Qs"], cut["K"], cut["V"], idx, w)
+        check_close(go[b:b + 1, :n], O_sel, f"O_sel b={b}")
+        check_close(gb[b:b + 1, :n], o_bar, f"o_bar b={b}")
+        check_close(gs[b:b + 1, :n], s, f"s b={b}")
