@@ -1,4 +1,4 @@
-"""CPU oracle for GQE prefill and decode (test infrastructure, not product code).
+"""CPU oracle for GQE prefill, decode and the attention layer around them (test infrastructure, not product code).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The library under
@@ -6,6 +6,7 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 """
 from .gqe_oracle import (  # noqa: F401
     bf16_to_f64,
+    f64_to_bf16_bits,
     router_logits,
     route,
     topk_exact_order,
@@ -18,4 +19,5 @@ from .gqe_oracle import (  # noqa: F401
     dense_gqa,
     dense_gqa_repeat,
     kv_cache_bytes,
+    gqe_layer_prefill,
 )

@@ -53,6 +53,16 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
 
 
+def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    """Round float64 values (finite, in bf16's normal range) to the nearest
+    bf16, ties to even, in one step; returns the bit patterns.  bf16 keeps 8
+    significant bits: with v = m * 2^e, 1/2 <= |m| < 1, the result is
+    round_half_even(m * 2^8) * 2^(e - 8)."""
+    m, e = np.frexp(np.asarray(v, dtype=np.float64))
+    q = np.ldexp(np.round(m * 256.0), e - 8)  # np.round: halves to even
+    return (q.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
 # ---------------------------------------------------------------------------
 # small helpers kept separate so the pin tests can plant mistakes in them
 # ---------------------------------------------------------------------------
@@ -405,3 +415,48 @@ def dense_gqa_repeat(Q_bits, K_bits, V_bits, dtype=np.float64):
 def kv_cache_bytes(L: int, G: int, S: int, d: int, b: int, B: int = 1) -> int:
     """[GQA article] §4.1: KV bytes per sequence = 2 * L * G * d * S * b (times B)."""
     return 2 * L * G * d * S * b * B
+
+
+# ---------------------------------------------------------------------------
+# the whole attention layer around the path (projections and W_O)
+# ---------------------------------------------------------------------------
+
+def gqe_layer_prefill(x_bits, Wq_bits, Wk_bits, Wv_bits, Ws_bits, Wr_bits, Wo_bits, bias, k):
+    """GQE attention layer, causal prefill, from x to y.
+
+    [GQE review] §二: the router picks k query heads per (token, group); only
+    the selected query heads are computed at all, so their query projection
+    runs for the selected (token, head) pairs only; the layer output is
+    y_i = Concat(O_i, ō_i, s(x_i)) W_O.  The projections themselves are
+    plain linear maps (the pages give them no special form):
+      q_{i,h} = x_i W_Q[h] (selected h only), K_{i,g} = x_i W_K[g],
+      V_{i,g} = x_i W_V[g], and the shared head's query x_i W_s.
+    They are rounded to bf16, the element type the attention takes.
+    Shapes: x [B,S,dm]; W_Q [N,dm,d]; W_K, W_V [G,dm,d]; W_s [dm,d];
+    W_r [G,dm,M]; W_O [(G*k + G + 1)*d, dm], rows in concat order; all bf16
+    bits.  Returns a dict with y [B,S,dm] (float64) and the intermediates
+    (Q bits with unselected heads left zero, K, V, Qs bits, topk_idx, w,
+    concat).
+    """
+    x = bf16_to_f64(x_bits)
+    Wq, Wk, Wv = bf16_to_f64(Wq_bits), bf16_to_f64(Wk_bits), bf16_to_f64(Wv_bits)
+    Ws, Wo = bf16_to_f64(Ws_bits), bf16_to_f64(Wo_bits)
+    B, S, dm = x.shape
+    N, _, d = Wq.shape
+    G = Wk.shape[0]
+    M = N // G
+    idx, p, w, _ = route(x_bits, Wr_bits, bias, k)
+    Q_bits = np.zeros((B, S, N, d), dtype=np.uint16)
+    for g in range(G):
+        for m in range(M):
+            h = _expert_head(g, m, M)
+            rows = np.nonzero((idx[:, :, g, :] == m).any(axis=-1))  # (b, i) that selected m
+            if rows[0].size:
+                Q_bits[rows[0], rows[1], h] = f64_to_bf16_bits(x[rows] @ Wq[h])
+    K_bits = f64_to_bf16_bits(np.einsum("bsc,gcd->bsgd", x, Wk))
+    V_bits = f64_to_bf16_bits(np.einsum("bsc,gcd->bsgd", x, Wv))
+    Qs_bits = f64_to_bf16_bits(x @ Ws)
+    O_sel, o_bar, s_out = gqe_prefill(Q_bits, Qs_bits, K_bits, V_bits, idx, w)
+    concat = np.concatenate([O_sel.reshape(B, S, -1), o_bar.reshape(B, S, -1), s_out], axis=-1)
+    return dict(y=concat @ Wo, Q=Q_bits, K=K_bits, V=V_bits, Qs=Qs_bits, topk_idx=idx, p=p,
+                w=w, concat=concat)

@@ -613,3 +613,109 @@ def test_planted_kv_bytes_mistake(monkeypatch):
     monkeypatch.setattr(oracle, "kv_cache_bytes", lambda L, G, S, d, b, B=1: L * G * d * S * b * B)
     with pytest.raises(AssertionError):
         check_kv_bytes()
+
+
+# --------------------------------------------------------------------------
+# the attention layer around the path: projections and W_O
+# --------------------------------------------------------------------------
+
+def test_f64_to_bf16_rounding():
+    """Nearest bf16, ties to even: agrees with the input generator's float32
+    rounding on float32 values, lands on a neighbour within half an ulp, and
+    sends exact midpoints to the even significand."""
+    rng = np.random.default_rng(3)
+    v32 = (rng.standard_normal(4000) * np.exp(rng.uniform(-20, 20, 4000))).astype(np.float32)
+    assert np.array_equal(og.f64_to_bf16_bits(v32.astype(np.float64)), f32_to_bf16_bits(v32))
+    v = rng.standard_normal(4000) * 7.0
+    q = og.bf16_to_f64(og.f64_to_bf16_bits(v))
+    ulp = 2.0 ** (np.floor(np.log2(np.abs(v))) - 7)
+    assert (np.abs(q - v) <= ulp / 2).all()
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: even significand is 1
+    # 1 + 3*2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6: even is 1 + 2^-6
+    mids = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8)])
+    assert og.bf16_to_f64(og.f64_to_bf16_bits(mids)).tolist() == [1.0, 1 + 2.0 ** -6, -1.0]
+
+
+def _layer_case(seed, B=1, S=6, N=4, G=2, d=2, dm=10):
+    M = N // G
+    return dict(
+        x=normal_bf16((B, S, dm), seed), Wq=normal_bf16((N, dm, d), seed + 1, std=0.5),
+        Wk=normal_bf16((G, dm, d), seed + 2, std=0.5), Wv=normal_bf16((G, dm, d), seed + 3),
+        Ws=normal_bf16((dm, d), seed + 4, std=0.5),
+        Wr=normal_bf16((G, dm, M), seed + 5, std=dm ** -0.5))
+
+
+def check_layer_bruteforce():
+    """Every step of the layer written out with loops on a tiny case: routed
+    query projection for the selected heads only, K/V/shared projections,
+    causal softmax attention per selected head, ō, concat, W_O."""
+    k = 1
+    c = _layer_case(19300)
+    B, S, dm = c["x"].shape
+    N, _, d = c["Wq"].shape
+    G = c["Wk"].shape[0]
+    M = N // G
+    width = (G * k + G + 1) * d
+    Wo = normal_bf16((width, dm), 19306, std=0.3)
+    out = oracle.gqe_layer_prefill(c["x"], c["Wq"], c["Wk"], c["Wv"], c["Ws"], c["Wr"], Wo,
+                                   None, k)
+    X, f = og.bf16_to_f64(c["x"]), og.bf16_to_f64
+    rb = lambda v: float(f(og.f64_to_bf16_bits(np.array([v])))[0])  # noqa: E731
+
+    def proj(row, W):  # W [dm, d]
+        return [rb(math.fsum(row[c_] * W[c_, e] for c_ in range(dm))) for e in range(d)]
+
+    idx = out["topk_idx"]
+    for b in range(B):
+        K = [[proj(X[b, t], f(c["Wk"][g])) for g in range(G)] for t in range(S)]
+        V = [[proj(X[b, t], f(c["Wv"][g])) for g in range(G)] for t in range(S)]
+        for i in range(S):
+            def attend(q, g):
+                sc = [math.fsum(q[e] * K[t][g][e] for e in range(d)) / math.sqrt(d)
+                      for t in range(i + 1)]
+                mx = max(sc)
+                ex = [math.exp(s_ - mx) for s_ in sc]
+                z = math.fsum(ex)
+                return [math.fsum(ex[t] * V[t][g][e] for t in range(i + 1)) / z for e in range(d)]
+            row = []
+            obar = []
+            for g in range(G):
+                m = int(idx[b, i, g, 0])
+                q = proj(X[b, i], f(c["Wq"][g * M + m]))
+                assert np.array_equal(out["Q"][b, i, g * M + m],
+                                      og.f64_to_bf16_bits(np.array(q)))
+                o = attend(q, g)
+                row += o
+                obar += o                           # k = 1: w = 1
+            row += obar + attend(proj(X[b, i], f(c["Ws"])), 0)
+            y = [math.fsum(row[r] * f(Wo)[r, c_] for r in range(width)) for c_ in range(dm)]
+            assert np.allclose(out["y"][b, i], y, rtol=1e-12, atol=1e-12), (b, i)
+            # unselected heads are never projected
+            for g in range(G):
+                for m in range(M):
+                    if m != idx[b, i, g, 0]:
+                        assert not out["Q"][b, i, g * M + m].any()
+
+
+def test_layer_bruteforce():
+    check_layer_bruteforce()
+
+
+ALL_CHECKS.append(check_layer_bruteforce)  # planted mistakes must show here too
+
+
+def test_layer_with_identity_output_projection_is_the_concat():
+    """W_O = I (d_model equal to the concat width) returns the concat buffer,
+    which is the path's output on the projected inputs."""
+    k = 2
+    c = _layer_case(19400, B=2, S=9, N=8, G=2, d=2, dm=(2 * 2 + 2 + 1) * 2)
+    dm = c["x"].shape[2]
+    eye = og.f64_to_bf16_bits(np.eye(dm))
+    out = oracle.gqe_layer_prefill(c["x"], c["Wq"], c["Wk"], c["Wv"], c["Ws"], c["Wr"], eye,
+                                   None, k)
+    assert np.array_equal(out["y"], out["concat"])
+    O_sel, o_bar, s = oracle.gqe_prefill(out["Q"], out["Qs"], out["K"], out["V"],
+                                         out["topk_idx"], out["w"])
+    B, S = O_sel.shape[:2]
+    assert np.array_equal(out["concat"], np.concatenate(
+        [O_sel.reshape(B, S, -1), o_bar.reshape(B, S, -1), s], axis=-1))
