@@ -15,6 +15,7 @@ from .gqe_oracle import (  # noqa: F401
     gqe_prefill,
     gqe_prefill_rows,
     gqe_decode_step,
+    gqe_append_step,
     exact_logits,
     dense_gqa,
     dense_gqa_repeat,

@@ -367,6 +367,24 @@ def gqe_decode_step(x_bits, Wr_bits, bias, Q_bits, Qs_bits, Kc_bits, Vc_bits, po
     return idx, p, w, O_sel, o_bar, s_out
 
 
+def gqe_append_step(x_bits, Wr_bits, bias, Q_bits, Qs_bits, Kc_bits, Vc_bits, pos, k,
+                    dtype=np.float64, kv_start=None):
+    """n new tokens per sequence over a cache (short chunked prefill).
+
+    [GQA article] 工程实操 非方形因果遮罩: Sq queries at the end of Sk keys;
+    the mask is taken on absolute positions, so new token r of sequence b,
+    at slot pos[b] + r, sees slots kv_start[b]..pos[b] + r (its own K/V and
+    those of the earlier new tokens are already in the cache).  Each row is
+    the decode step of its own token.  x [B, n, dm], Q [B, n, N, d],
+    Qs [B, n, d]; returns the decode step's arrays with an n axis after B.
+    """
+    n = np.asarray(x_bits).shape[1]
+    rows = [gqe_decode_step(x_bits[:, r], Wr_bits, bias, Q_bits[:, r], Qs_bits[:, r], Kc_bits,
+                            Vc_bits, np.asarray(pos) + r, k, dtype=dtype, kv_start=kv_start)
+            for r in range(n)]
+    return tuple(np.stack([row[i] for row in rows], axis=1) for i in range(6))
+
+
 def dense_gqa(Q_bits, K_bits, V_bits, dtype=np.float64, rows=None):
     """Dense GQA (every query head active), explicit head -> KV-head map.
 

@@ -719,3 +719,20 @@ def test_layer_with_identity_output_projection_is_the_concat():
     B, S = O_sel.shape[:2]
     assert np.array_equal(out["concat"], np.concatenate(
         [O_sel.reshape(B, S, -1), o_bar.reshape(B, S, -1), s], axis=-1))
+
+
+def test_append_step_equals_prefill_rows():
+    """n new tokens appended at slots t..t+n-1 of the full sequence's cache
+    are prefill's rows t..t+n-1 (the non-square causal case Sq = n over
+    Sk = t + n keys)."""
+    (B, S, N, G, k, d, dm), c = _decode_case(19500)
+    idx, p, w, _ = oracle.route(c["x"], c["W_r"], None, k)
+    O_sel, o_bar, s = oracle.gqe_prefill(c["Q"], c["Qs"], c["K"], c["V"], idx, w)
+    for t, n in ((5, 2), (0, 3), (30, 10)):
+        sl = slice(t, t + n)
+        got = oracle.gqe_append_step(c["x"][:, sl], c["W_r"], None, c["Q"][:, sl],
+                                     c["Qs"][:, sl], c["K"], c["V"], np.array([t] * B), k)
+        assert np.array_equal(got[0], idx[:, sl])
+        assert np.allclose(got[3], O_sel[:, sl], rtol=1e-12, atol=1e-12)
+        assert np.allclose(got[4], o_bar[:, sl], rtol=1e-12, atol=1e-12)
+        assert np.allclose(got[5], s[:, sl], rtol=1e-12, atol=1e-12)
