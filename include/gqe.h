@@ -221,6 +221,29 @@ gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void*
                                 int64_t out_row_stride, void* ws, size_t ws_bytes,
                                 void* stream);
 
+/*
+ * gqe_attention_append - n_new new tokens per sequence over the caches: a
+ * short chunked prefill, or checking n_new drafted tokens at once.
+ * "AI 大模型之 GQA", 工程实操 非方形因果遮罩: Sq queries at the end of Sk keys,
+ * masked on absolute positions.  New token r of sequence b sits at cache
+ * slot pos[b] + r and sees slots kv_start[b]..pos[b] + r; slots pos[b] ..
+ * pos[b] + n_new - 1 must already hold the new tokens' K and V.  Everything
+ * else is gqe_attention_decode with an n_new axis after B:
+ *  Q bf16 [B, n_new, N, d]; Qs bf16 [B, n_new, d];
+ *  topk_idx int32 / w fp32 [B, n_new, G, k] (gqe_route with dims S = n_new);
+ *  output row b * n_new + r of O_sel / o_bar / s_out (stride as before).
+ * 1 <= n_new <= 64 and n_new <= T (longer chunks belong to the prefill
+ * kernels); pos[b] + n_new - 1 < T is checked on the device
+ * (GQE_ERR_BAD_POSITION).  gqe_attention_decode is the n_new = 1 case.
+ */
+size_t gqe_append_workspace_size(const gqe_dims* dims, int32_t n_new);
+gqe_status gqe_attention_append(const gqe_dims* dims, int32_t n_new, const void* Q,
+                                const void* Qs, const void* Kc, const void* Vc,
+                                const int32_t* pos, const int32_t* kv_start,
+                                const int32_t* topk_idx, const float* w, void* O_sel,
+                                void* o_bar, void* s_out, int64_t out_row_stride, void* ws,
+                                size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then returns the status word latched in `ws`
  * (GQE_OK if no device-side error was recorded).  If `clear` is non-zero the
  * word is reset to GQE_OK afterwards. */

@@ -5,8 +5,8 @@ The compute lives in ``libgqe.so`` (CUDA kernels behind the C ABI of
 torch-facing layer (``layer``) that allocates device buffers and calls the ABI.
 """
 from ._lib import (  # noqa: F401
-    EXPORTS, GqeDims, GqeError, LIB, LIB_PATH, STATUS, dims, gqe_attention_decode,
-    gqe_attention_prefill, gqe_decode_workspace_size,
+    EXPORTS, GqeDims, GqeError, LIB, LIB_PATH, STATUS, dims, gqe_append_workspace_size,
+    gqe_attention_append, gqe_attention_decode, gqe_attention_prefill, gqe_decode_workspace_size,
     gqe_attention_prefill_static, gqe_bucket,
     gqe_dense_gqa_prefill, gqe_get_device_status, gqe_kv_cache_bytes, gqe_route,
     gqe_selftest_bounded_wait, gqe_set_pair_threshold, gqe_set_profile_events, gqe_status_string,

@@ -18,7 +18,7 @@ EXPORTS = (
     "gqe_dense_gqa_prefill", "gqe_get_device_status", "gqe_kv_cache_bytes",
     "gqe_status_string", "gqe_selftest_bounded_wait", "gqe_set_profile_events",
     "gqe_attention_prefill_static", "gqe_set_pair_threshold", "gqe_decode_workspace_size",
-    "gqe_attention_decode",
+    "gqe_attention_decode", "gqe_append_workspace_size", "gqe_attention_append",
 )
 
 STATUS = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED", 3: "GQE_ERR_CUDA",
@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
         "gqe_set_pair_threshold": (I64, [I64]),
         "gqe_decode_workspace_size": (SZ, [S]),
         "gqe_attention_decode": (I32, [S, P, P, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
+        "gqe_append_workspace_size": (SZ, [S, I32]),
+        "gqe_attention_append": (I32, [S, I32, P, P, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -177,3 +179,17 @@ def gqe_attention_decode(dm, Q, Qs, Kc, Vc, pos, kv_start, topk_idx, w, O_sel, o
                                  _ptr(s_out), int(out_row_stride), _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream))
     return _check(r, "gqe_attention_decode") if check else r
+
+
+def gqe_append_workspace_size(dm: GqeDims, n_new: int) -> int:
+    return LIB.gqe_append_workspace_size(ctypes.byref(dm), int(n_new))
+
+
+def gqe_attention_append(dm, n_new, Q, Qs, Kc, Vc, pos, kv_start, topk_idx, w, O_sel, o_bar,
+                         s_out, out_row_stride, ws, stream=None, check=True):
+    """n_new new tokens per sequence over the caches; dm.S is the capacity T."""
+    r = LIB.gqe_attention_append(ctypes.byref(dm), int(n_new), _ptr(Q), _ptr(Qs), _ptr(Kc),
+                                 _ptr(Vc), _ptr(pos), _ptr(kv_start), _ptr(topk_idx), _ptr(w),
+                                 _ptr(O_sel), _ptr(o_bar), _ptr(s_out), int(out_row_stride),
+                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_attention_append") if check else r

@@ -298,20 +298,30 @@ size_t gqe_decode_workspace_size(const gqe_dims* dims) {
   return make_decode_plan(*dims).total;
 }
 
-gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void* Qs,
-                                const void* Kc, const void* Vc, const int32_t* pos,
-                                const int32_t* kv_start, const int32_t* topk_idx,
-                                const float* w, void* O_sel, void* o_bar, void* s_out,
-                                int64_t out_row_stride, void* ws, size_t ws_bytes,
-                                void* stream) {
+size_t gqe_append_workspace_size(const gqe_dims* dims, int32_t n_new) {
+  if (check_dims(dims, false) != GQE_OK || n_new < 1 || n_new > kMaxAppend ||
+      n_new > dims->S)
+    return 0;
+  return make_decode_plan(*dims, n_new).total;
+}
+
+gqe_status gqe_attention_append(const gqe_dims* dims, int32_t n_new, const void* Q,
+                                const void* Qs, const void* Kc, const void* Vc,
+                                const int32_t* pos, const int32_t* kv_start,
+                                const int32_t* topk_idx, const float* w, void* O_sel,
+                                void* o_bar, void* s_out, int64_t out_row_stride, void* ws,
+                                size_t ws_bytes, void* stream) {
   gqe_status st = check_dims(dims, false);
   if (st != GQE_OK) return st;
+  if (n_new < 1 || n_new > kMaxAppend || n_new > dims->S) return GQE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(dims->B) * n_new * dims->N >= (int64_t(1) << 31))
+    return GQE_ERR_UNSUPPORTED;
   if (!aligned16(Q) || !aligned16(Qs) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(pos) ||
       !aligned16(topk_idx) || !aligned16(w) || !aligned16(O_sel) || !aligned16(o_bar) ||
       !aligned16(s_out) || (kv_start && !aligned16(kv_start)))
     return GQE_ERR_INVALID_ARG;
   if (out_row_stride < dims->d || out_row_stride % 8 != 0) return GQE_ERR_INVALID_ARG;
-  const DecodePlan P = make_decode_plan(*dims);
+  const DecodePlan P = make_decode_plan(*dims, n_new);
   if (!aligned16(ws) || ws_bytes < P.total) return GQE_ERR_WORKSPACE;
   uint8_t* wb = static_cast<uint8_t*>(ws);
   DecodeArgs a{};
@@ -338,6 +348,7 @@ gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void*
   a.M = dims->N / dims->G;
   a.k = dims->k;
   a.d = dims->d;
+  a.n_new = n_new;
   a.heads = static_cast<int>(P.heads);
   a.passes = static_cast<int>(P.passes);
   a.nchunks = static_cast<int>(P.nchunks);
@@ -345,6 +356,16 @@ gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void*
   a.out_fp32 = dims->out_fp32;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dims->d)));
   return from_cuda(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void* Qs,
+                                const void* Kc, const void* Vc, const int32_t* pos,
+                                const int32_t* kv_start, const int32_t* topk_idx,
+                                const float* w, void* O_sel, void* o_bar, void* s_out,
+                                int64_t out_row_stride, void* ws, size_t ws_bytes,
+                                void* stream) {
+  return gqe_attention_append(dims, 1, Q, Qs, Kc, Vc, pos, kv_start, topk_idx, w, O_sel, o_bar,
+                              s_out, out_row_stride, ws, ws_bytes, stream);
 }
 
 gqe_status gqe_get_device_status(void* ws, int32_t clear, void* stream) {

@@ -44,6 +44,10 @@ __device__ __forceinline__ void store_out(void* base, int64_t off, float v, int 
 }
 
 // Partial attention of one (b, g, chunk) for head slots pass*HB .. pass*HB+HB-1.
+// MULTI (n_new > 1): slot r*(k+1) + j belongs to new token r, whose query sits
+// at slot pos + r and sees keys up to there; each head slot then carries its
+// own causal bound.  Without MULTI every slot is token 0's and the chunk's end
+// is its bound.
 //
 // Lanes: a key row of D bf16 is read by L = D/8 lanes, 16 bytes each, so a
 // warp reads 32/L consecutive rows per load; the key slots of the CTA are
@@ -52,7 +56,7 @@ __device__ __forceinline__ void store_out(void* base, int64_t off, float v, int 
 // the group ends with the same sum), then each slot keeps its own online
 // softmax state per head; the slots are merged through shared memory at the
 // end of the chunk.
-template <int D, int HB>
+template <int D, int HB, bool MULTI>
 __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const DecodeArgs a) {
   constexpr int L = D / 8;
   constexpr int SPW = 32 / L;
@@ -74,36 +78,45 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const De
   const int g = static_cast<int>(unit % a.G);
   const int b = static_cast<int>(unit / a.G);
 
-  // visible keys of sequence b: slots lo..pos (lo > 0 with left padding)
+  // visible keys of sequence b: slots lo..pos + r for new token r (lo > 0
+  // with left padding); `last` is the last new token's slot
   const int pos = a.pos[b];
   const int lo = a.kv_start ? a.kv_start[b] : 0;
-  if (pos < 0 || pos >= a.T || lo < 0 || lo > pos) {
+  const int64_t last = static_cast<int64_t>(pos) + a.n_new - 1;
+  if (pos < 0 || last >= a.T || lo < 0 || lo > pos) {
     if (threadIdx.x == 0 && c == 0 && pass == 0 && g == 0)
       latch_status(a.status, GQE_ERR_BAD_POSITION);
     return;
   }
   const int64_t c0 = static_cast<int64_t>(c) * a.chunk;
-  if (c0 > pos || c0 + a.chunk <= lo) return;  // no visible key here; the merge skips it
+  if (c0 > last || c0 + a.chunk <= lo) return;  // no visible key here; the merge skips it
   const int64_t t0 = max(c0, static_cast<int64_t>(lo));
-  const int64_t t1 = min(c0 + a.chunk, static_cast<int64_t>(pos) + 1);
+  const int64_t t1 = min(c0 + a.chunk, last + 1);
 
   // this pass's head slots: j < k routed (head g*M + topk_idx), j == k the
   // shared head (KV head 0 only); a slot that is not live is skipped
   const int64_t bg = static_cast<int64_t>(b) * a.G + g;
   float q[HB][8];
   bool live[HB];
+  int qpos[HB];  // causal bound of each slot (MULTI)
 #pragma unroll
   for (int h = 0; h < HB; ++h) {
-    const int j = pass * HB + h;
+    int r = 0, j = pass * HB + h;
+    if (MULTI) {
+      r = j / (a.k + 1);
+      j -= r * (a.k + 1);
+    }
+    qpos[h] = pos + r;
+    const int64_t tr = static_cast<int64_t>(b) * a.n_new + r;  // the token's row
     const uint16_t* qrow = nullptr;
-    if (j < a.k) {
-      const int m = a.topk_idx[bg * a.k + j];
+    if (r < a.n_new && j < a.k) {
+      const int m = a.topk_idx[(tr * a.G + g) * a.k + j];
       if (m >= 0 && m < a.M)
-        qrow = a.Q + (static_cast<int64_t>(b) * a.N + static_cast<int64_t>(g) * a.M + m) * D;
+        qrow = a.Q + (tr * a.N + static_cast<int64_t>(g) * a.M + m) * D;
       else if (threadIdx.x == 0)
         latch_status(a.status, GQE_ERR_BAD_INDEX);
-    } else if (j == a.k && g == 0) {
-      qrow = a.Qs + static_cast<int64_t>(b) * D;
+    } else if (r < a.n_new && j == a.k && g == 0) {
+      qrow = a.Qs + tr * D;
     }
     live[h] = qrow != nullptr;
     if (live[h]) {
@@ -153,7 +166,9 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const De
         for (int e = 0; e < 8; ++e) acc = fmaf(q[h][e], kf[e], acc);
 #pragma unroll
         for (int off = L / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        s[u] = ok[u] ? acc : -INFINITY;
+        bool vis = ok[u];
+        if (MULTI) vis = vis && tb + u * NS + slot <= qpos[h];
+        s[u] = vis ? acc : -INFINITY;
       }
       float mx = m_run[h];
 #pragma unroll
@@ -217,35 +232,40 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const De
   }
 }
 
-// Merge of the chunks of one (b, g): for each live head slot, rescale every
-// chunk that holds visible keys (those the partial kernel wrote) to the
-// common maximum, add, normalise; then
+// Merge of the chunks of one (new token, g): for each live head slot of that
+// token, rescale every chunk that holds keys it sees (the partial kernel
+// wrote those) to the common maximum, add, normalise; then
 // o_bar = sum_j w_j * O_j in slot order (review §二 三个关键部件) and the
 // shared head for g = 0.  One thread per output element.
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
-  const int64_t bg = blockIdx.x;
-  const int b = static_cast<int>(bg / a.G);
-  const int g = static_cast<int>(bg % a.G);
+  // one CTA per (new token row, g); row tr = b * n_new + r
+  const int g = static_cast<int>(blockIdx.x % a.G);
+  const int64_t tr = blockIdx.x / a.G;
+  const int b = static_cast<int>(tr / a.n_new);
+  const int r = static_cast<int>(tr % a.n_new);
+  const int64_t bg = static_cast<int64_t>(b) * a.G + g;  // partials are per (b, g)
+  const int64_t rg = tr * a.G + g;                       // router outputs per (row, g)
   const int e = threadIdx.x;
   const int pos = a.pos[b];
   const int lo = a.kv_start ? a.kv_start[b] : 0;
-  const bool pos_ok = pos >= 0 && pos < a.T && lo >= 0 && lo <= pos;
-  const int c_lo = pos_ok ? lo / a.chunk : 0;     // chunks c_lo .. nc-1 hold visible keys
-  const int nc = pos_ok ? pos / a.chunk + 1 : 0;
+  const bool pos_ok = pos >= 0 && static_cast<int64_t>(pos) + a.n_new - 1 < a.T && lo >= 0 &&
+                      lo <= pos;
+  const int c_lo = pos_ok ? lo / a.chunk : 0;  // chunks c_lo .. nc-1 hold visible keys
+  const int nc = pos_ok ? (pos + r) / a.chunk + 1 : 0;
   const int nh = a.k + (g == 0 ? 1 : 0);
   const float nan = __int_as_float(0x7fc00000);
-  const int64_t r = static_cast<int64_t>(b) * a.out_row_stride;
+  const int64_t row = tr * a.out_row_stride;
   float obar = 0.f;
   for (int j = 0; j < nh; ++j) {
     bool ok = pos_ok;
     if (j < a.k) {
-      const int m = a.topk_idx[bg * a.k + j];
+      const int m = a.topk_idx[rg * a.k + j];
       ok = ok && m >= 0 && m < a.M;
     }
     float out = nan;  // a rejected position or expert index yields NaN
     if (ok) {
-      const int64_t p0 = (bg * a.heads + j) * a.nchunks;
+      const int64_t p0 = (bg * a.heads + static_cast<int64_t>(r) * (a.k + 1) + j) * a.nchunks;
       float mx = kNoKeyMax;
       for (int c = c_lo; c < nc; ++c) mx = fmaxf(mx, a.part_m[p0 + c]);
       float acc = 0.f, lsum = 0.f;
@@ -257,33 +277,42 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
       out = acc / lsum;
     }
     if (j < a.k) {
-      store_out(a.O_sel, r + (static_cast<int64_t>(g) * a.k + j) * D + e, out, a.out_fp32);
-      obar = fmaf(a.w[bg * a.k + j], out, obar);
+      store_out(a.O_sel, row + (static_cast<int64_t>(g) * a.k + j) * D + e, out, a.out_fp32);
+      obar = fmaf(a.w[rg * a.k + j], out, obar);
     } else {
-      store_out(a.s_out, r + e, out, a.out_fp32);
+      store_out(a.s_out, row + e, out, a.out_fp32);
     }
   }
-  store_out(a.o_bar, r + static_cast<int64_t>(g) * D + e, obar, a.out_fp32);
+  store_out(a.o_bar, row + static_cast<int64_t>(g) * D + e, obar, a.out_fp32);
 }
 
-template <int D, int HB>
+template <int D, int HB, bool MULTI>
 cudaError_t launch_decode_dh(const DecodeArgs& a, cudaStream_t st) {
   const int64_t ctas = static_cast<int64_t>(a.B) * a.G * a.passes * a.nchunks;
-  decode_partial_kernel<D, HB><<<static_cast<unsigned>(ctas), kDecThreads, 0, st>>>(a);
+  decode_partial_kernel<D, HB, MULTI><<<static_cast<unsigned>(ctas), kDecThreads, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_merge_kernel<D><<<static_cast<unsigned>(static_cast<int64_t>(a.B) * a.G), D, 0, st>>>(a);
+  const int64_t rows = static_cast<int64_t>(a.B) * a.n_new * a.G;
+  decode_merge_kernel<D><<<static_cast<unsigned>(rows), D, 0, st>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
+  if (a.n_new > 1) {  // several new tokens: per-slot causal bounds
+    if (a.d == 64) return launch_decode_dh<64, kDecHeads, true>(a, st);
+    if (a.d == 128) return launch_decode_dh<128, kDecHeads, true>(a, st);
+    return cudaErrorInvalidValue;
+  }
   // two head slots cover k = 1 (a routed head, plus the shared one for g = 0)
   const bool narrow = a.heads <= 2;
-  if (a.d == 64) return narrow ? launch_decode_dh<64, 2>(a, st) : launch_decode_dh<64, kDecHeads>(a, st);
+  if (a.d == 64)
+    return narrow ? launch_decode_dh<64, 2, false>(a, st)
+                  : launch_decode_dh<64, kDecHeads, false>(a, st);
   if (a.d == 128)
-    return narrow ? launch_decode_dh<128, 2>(a, st) : launch_decode_dh<128, kDecHeads>(a, st);
+    return narrow ? launch_decode_dh<128, 2, false>(a, st)
+                  : launch_decode_dh<128, kDecHeads, false>(a, st);
   return cudaErrorInvalidValue;
 }
 

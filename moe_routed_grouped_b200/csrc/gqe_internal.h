@@ -168,29 +168,30 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 cudaError_t launch_selftest_wait(int* status, uint64_t limit_ns, cudaStream_t st);
 
 // ------------------------------------------------------------ decode step
-// Split-KV plan of gqe_attention_decode.  A CTA takes one chunk of keys of
-// one (b, g) and up to kDecHeads of that group's head slots (slots 0..k-1 the
-// routed heads, slot k the shared head, live only for g = 0); a second
-// kernel merges the chunks.  The plan depends on dims only, so the workspace
-// size does too.
+// Split-KV plan of gqe_attention_decode / gqe_attention_append.  A CTA takes
+// one chunk of keys of one (b, g) and up to kDecHeads of that group's head
+// slots; slot r*(k+1) + j is new token r's routed head j (j < k) or its shared
+// head (j = k, live only for g = 0).  A second kernel merges the chunks.  The
+// plan depends on dims and n_new only, so the workspace size does too.
 constexpr int kDecThreads = 128;     // 4 warps per partial-attention CTA
 constexpr int kDecHeads = 4;         // head slots per CTA (registers bound it)
 constexpr int kDecUnroll = 4;        // keys in flight per key slot
 constexpr int64_t kDecTargetCtas = 4 * 148;
 constexpr int64_t kDecMinChunk = 256;
+constexpr int kMaxAppend = 64;       // new tokens per sequence in one append call
 
 struct DecodePlan {
-  int64_t heads;    // head slots per (b, g): k + 1
+  int64_t heads;    // head slots per (b, g): (k + 1) * n_new
   int64_t passes;   // ceil(heads / kDecHeads)
   int64_t chunk;    // keys per CTA (multiple of 64)
   int64_t nchunks;  // ceil(T / chunk)
   size_t status, part_m, part_l, part_o, total;  // workspace byte offsets
 };
 
-inline DecodePlan make_decode_plan(const gqe_dims& d) {
+inline DecodePlan make_decode_plan(const gqe_dims& d, int64_t n_new = 1) {
   DecodePlan P{};
   const int64_t B = d.B, T = d.S, G = d.G, hd = d.d;
-  P.heads = d.k + 1;
+  P.heads = (d.k + 1) * n_new;
   P.passes = (P.heads + kDecHeads - 1) / kDecHeads;
   const int64_t groups = B * G * P.passes;
   const int64_t want = groups >= kDecTargetCtas ? 1 : (kDecTargetCtas + groups - 1) / groups;
@@ -209,14 +210,14 @@ inline DecodePlan make_decode_plan(const gqe_dims& d) {
 }
 
 struct DecodeArgs {
-  const uint16_t* Q;    // bf16 [B, N, d]
-  const uint16_t* Qs;   // bf16 [B, d]
+  const uint16_t* Q;    // bf16 [B, n_new, N, d]
+  const uint16_t* Qs;   // bf16 [B, n_new, d]
   const uint16_t* Kc;   // bf16 [B, T, G, d]
   const uint16_t* Vc;   // bf16 [B, T, G, d]
-  const int32_t* pos;   // [B]
+  const int32_t* pos;   // [B]: slot of new token 0 (token r at pos + r)
   const int32_t* kv_start;  // [B] first valid slot, or null (0)
-  const int32_t* topk_idx;  // [B, G, k]
-  const float* w;           // [B, G, k]
+  const int32_t* topk_idx;  // [B, n_new, G, k]
+  const float* w;           // [B, n_new, G, k]
   float* part_m;        // [B, G, heads, nchunks]: running max (log2 units)
   float* part_l;        // [B, G, heads, nchunks]: sum of exponentials
   float* part_o;        // [B, G, heads, nchunks, d]: unnormalised output
@@ -226,6 +227,7 @@ struct DecodeArgs {
   int64_t out_row_stride;
   int* status;
   int B, T, N, G, M, k, d;
+  int n_new;            // new tokens per sequence (1: decode)
   int heads, passes, nchunks, chunk;
   int out_fp32;
   float scale_log2;     // log2(e) / sqrt(d)

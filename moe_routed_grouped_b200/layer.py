@@ -82,59 +82,71 @@ class GqePrefill:
 
 class GqeDecode:
     """Buffers and calls for one decode step of B sequences over KV caches of
-    capacity T (shape [B, T, G, d]).
+    capacity T (shape [B, T, G, d]); with ``n_new`` > 1, n_new new tokens per
+    sequence in one call (gqe_attention_append).
 
-    ``concat`` has one W_O input row per sequence, laid out as in
-    :class:`GqePrefill`.  One workspace serves the router (run on the new
-    tokens, S = 1) and the decode attention, in stream order.
+    ``concat`` has one W_O input row per new token (row b * n_new + r), laid
+    out as in :class:`GqePrefill`.  Per-token tensors have an n_new axis after
+    B when n_new > 1 (x [B, n_new, d_model], Q [B, n_new, N, d] ...) and none
+    when n_new = 1.  One workspace serves the router (run on the new tokens,
+    S = n_new) and the attention, in stream order.
     """
 
-    def __init__(self, B, T, N, G, k, d, d_model, out_fp32=True, device="cuda"):
+    def __init__(self, B, T, N, G, k, d, d_model, out_fp32=True, device="cuda", n_new=1):
         if N % G:
             raise ValueError("N must be a multiple of G")
         self.B, self.T, self.N, self.G, self.k, self.d, self.d_model = B, T, N, G, k, d, d_model
         self.M = N // G
+        self.n_new = n_new
         of = 1 if out_fp32 else 0
-        self.route_dims = _lib.dims(B, 1, N, G, k, d, d_model, of)
+        self.route_dims = _lib.dims(B, n_new, N, G, k, d, d_model, of)
         self.dims = _lib.dims(B, T, N, G, k, d, d_model, of)
         a = _lib.gqe_workspace_size(self.route_dims)
-        b = _lib.gqe_decode_workspace_size(self.dims)
+        b = _lib.gqe_append_workspace_size(self.dims, n_new)
         if a == 0 or b == 0:
-            raise _lib.GqeError(2, "gqe_decode_workspace_size")
+            raise _lib.GqeError(2, "gqe_append_workspace_size")
         dev = torch.device(device)
         self.device = dev
         self.ws = torch.zeros(max(a, b), dtype=torch.uint8, device=dev)
         self.out_dtype = torch.float32 if out_fp32 else torch.bfloat16
         self.row = (G * k + G + 1) * d
-        self.concat = torch.empty(B, self.row, dtype=self.out_dtype, device=dev)
-        self.topk_idx = torch.empty(B, G, k, dtype=torch.int32, device=dev)
-        self.p = torch.empty(B, G, self.M, dtype=torch.float32, device=dev)
-        self.w = torch.empty(B, G, k, dtype=torch.float32, device=dev)
+        self.concat = torch.empty(B * n_new, self.row, dtype=self.out_dtype, device=dev)
+        lead = (B,) if n_new == 1 else (B, n_new)
+        self._lead = lead
+        self.topk_idx = torch.empty(*lead, G, k, dtype=torch.int32, device=dev)
+        self.p = torch.empty(*lead, G, self.M, dtype=torch.float32, device=dev)
+        self.w = torch.empty(*lead, G, k, dtype=torch.float32, device=dev)
 
     def O_sel(self):
-        return self.concat[:, : self.G * self.k * self.d].view(self.B, self.G, self.k, self.d)
+        return self.concat[:, : self.G * self.k * self.d].view(*self._lead, self.G, self.k, self.d)
 
     def o_bar(self):
         a = self.G * self.k * self.d
-        return self.concat[:, a: a + self.G * self.d].view(self.B, self.G, self.d)
+        return self.concat[:, a: a + self.G * self.d].view(*self._lead, self.G, self.d)
 
     def s_out(self):
-        return self.concat[:, (self.G * self.k + self.G) * self.d:]
+        return self.concat[:, (self.G * self.k + self.G) * self.d:].view(*self._lead, self.d)
 
     def route(self, x, W_r, bias=None, stream=None):
-        """x: bf16 [B, d_model] (the new tokens)."""
+        """x: bf16 [B, d_model] (the new tokens; [B, n_new, d_model] if n_new > 1)."""
         _lib.gqe_route(self.route_dims, x, W_r, bias, self.topk_idx, self.p, self.w, self.ws,
                        stream)
         return self.topk_idx, self.p, self.w
 
     def attention(self, Q, Qs, Kc, Vc, pos, kv_start=None, stream=None):
-        """Q [B, N, d], Qs [B, d], caches [B, T, G, d] (bf16), pos int32 [B];
+        """Q [B, N, d], Qs [B, d] (n_new axis after B if n_new > 1), caches
+        [B, T, G, d] (bf16), pos int32 [B] (slot of the first new token);
         kv_start int32 [B] (first valid slot, left padding) or None."""
         a = self.G * self.k * self.d
         flat = self.concat.view(-1)
-        _lib.gqe_attention_decode(self.dims, Q, Qs, Kc, Vc, pos, kv_start, self.topk_idx,
-                                  self.w, self.concat, flat[a:], flat[a + self.G * self.d:],
-                                  self.row, self.ws, stream)
+        if self.n_new == 1:
+            _lib.gqe_attention_decode(self.dims, Q, Qs, Kc, Vc, pos, kv_start, self.topk_idx,
+                                      self.w, self.concat, flat[a:], flat[a + self.G * self.d:],
+                                      self.row, self.ws, stream)
+        else:
+            _lib.gqe_attention_append(self.dims, self.n_new, Q, Qs, Kc, Vc, pos, kv_start,
+                                      self.topk_idx, self.w, self.concat, flat[a:],
+                                      flat[a + self.G * self.d:], self.row, self.ws, stream)
         return self.concat
 
     def forward(self, x, W_r, bias, Q, Qs, Kc, Vc, pos, kv_start=None, stream=None):

@@ -146,3 +146,20 @@ def test_decode_workspace_scales_with_the_split():
     assert one < long < wide
     # the scratch does not grow past the CTA target once chunks are long
     assert _lib.gqe_decode_workspace_size(_lib.dims(1, 1 << 20, 16, 8, 1, 64)) <= 2 * long
+
+
+def test_append_rejects_bad_token_counts():
+    dm = _lib.dims(2, 100, 16, 8, 1, 64)
+    L = _lib.LIB
+
+    def call(n, ws_bytes=1 << 40):
+        return L.gqe_attention_append(ctypes.byref(dm), n, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                      FAKE, FAKE, FAKE, FAKE, FAKE, 17 * 64, FAKE, ws_bytes, None)
+    assert call(0) == 1 and call(65) == 1          # 1 <= n_new <= 64
+    assert _lib.gqe_append_workspace_size(dm, 0) == 0
+    assert _lib.gqe_append_workspace_size(dm, 65) == 0
+    small = _lib.dims(2, 10, 16, 8, 1, 64)
+    assert _lib.gqe_append_workspace_size(small, 11) == 0   # more new tokens than slots
+    need = _lib.gqe_append_workspace_size(dm, 5)
+    assert need > _lib.gqe_append_workspace_size(dm, 1) == _lib.gqe_decode_workspace_size(dm)
+    assert call(5, ws_bytes=need - 1) == 5

@@ -237,3 +237,74 @@ def test_decode_step_replays_as_a_cuda_graph():
                                      c["Vc"], np.asarray(p_), k)
         check_close(L.O_sel().cpu().numpy(), ref[3], "O_sel (graph)")
     assert L.device_status() == 0 and E.device_status() == 0
+
+
+# several new tokens per sequence (gqe_attention_append): (shape, n_new,
+# slot of the first new token, first valid slot or None).  Chunk edges at 256;
+# the last case is a whole 64-slot cache written by one call.
+APPEND = [
+    ((3, 700, 16, 8, 1, 64, 256), 2, [0, 254, 600], None),
+    ((2, 1000, 32, 8, 2, 128, 512), 3, [997, 255], [200, 0]),
+    ((2, 600, 16, 8, 1, 64, 64), 7, [250, 593], [250, 256]),
+    ((1, 300, 32, 4, 5, 64, 128), 2, [298], None),
+    ((2, 64, 8, 4, 2, 64, 64), 64, [0, 0], None),
+]
+
+
+@pytest.mark.parametrize("shape,n_new,pos,kv_start", APPEND,
+                         ids=lambda v: "x".join(map(str, v)) if isinstance(v, (tuple, list))
+                         else str(v))
+def test_append_parity(shape, n_new, pos, kv_start):
+    """New token r of sequence b at slot pos[b] + r sees slots
+    kv_start[b]..pos[b] + r: Sq queries at the end of Sk keys."""
+    B, T, N, G, k, d, dm = shape
+    M = N // G
+    seed = 37000 + B + T + n_new
+    c = dict(x=normal_bf16((B, n_new, dm), seed),
+             W_r=normal_bf16((G, dm, M), seed + 1, std=dm ** -0.5),
+             Q=normal_bf16((B, n_new, N, d), seed + 2), Qs=normal_bf16((B, n_new, d), seed + 3),
+             Kc=normal_bf16((B, T, G, d), seed + 4), Vc=normal_bf16((B, T, G, d), seed + 5))
+    L = GqeDecode(B, T, N, G, k, d, dm, n_new=n_new)
+    ks = None if kv_start is None else torch.tensor(kv_start, dtype=torch.int32, device="cuda")
+    L.forward(dev_bf16(c["x"]), dev_bf16(c["W_r"]), None, dev_bf16(c["Q"]), dev_bf16(c["Qs"]),
+              dev_bf16(c["Kc"]), dev_bf16(c["Vc"]),
+              torch.tensor(pos, dtype=torch.int32, device="cuda"), ks)
+    torch.cuda.synchronize()
+    assert L.device_status() == 0
+    idx, p, w, O_sel, o_bar, s = oracle.gqe_append_step(
+        c["x"], c["W_r"], None, c["Q"], c["Qs"], c["Kc"], c["Vc"], np.asarray(pos), k,
+        kv_start=None if kv_start is None else np.asarray(kv_start))
+    assert np.array_equal(L.topk_idx.cpu().numpy(), idx)
+    check_close(L.O_sel().cpu().numpy(), O_sel, "O_sel")
+    check_close(L.o_bar().cpu().numpy(), o_bar, "o_bar")
+    check_close(L.s_out().cpu().numpy(), s, "shared head")
+
+
+def test_append_matches_decode_steps_and_checks_the_last_slot():
+    """An append of n tokens equals n decode steps at the successive slots,
+    and a call whose last new token would fall beyond the cache is refused on
+    the device."""
+    B, T, N, G, k, d, dm, n = 2, 520, 16, 8, 2, 64, 128, 4
+    c = dict(x=normal_bf16((B, n, dm), 38000), W_r=normal_bf16((G, dm, 2), 38001, std=dm ** -0.5),
+             Q=normal_bf16((B, n, N, d), 38002), Qs=normal_bf16((B, n, d), 38003),
+             Kc=normal_bf16((B, T, G, d), 38004), Vc=normal_bf16((B, T, G, d), 38005))
+    dv = {key: dev_bf16(v) for key, v in c.items()}
+    A = GqeDecode(B, T, N, G, k, d, dm, n_new=n)
+    pos = [100, 516]
+    A.forward(dv["x"], dv["W_r"], None, dv["Q"], dv["Qs"], dv["Kc"], dv["Vc"],
+              torch.tensor(pos, dtype=torch.int32, device="cuda"))
+    D = GqeDecode(B, T, N, G, k, d, dm)
+    for r in range(n):
+        D.forward(dv["x"][:, r].contiguous(), dv["W_r"], None, dv["Q"][:, r].contiguous(),
+                  dv["Qs"][:, r].contiguous(), dv["Kc"], dv["Vc"],
+                  torch.tensor([p_ + r for p_ in pos], dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+        assert torch.equal(D.topk_idx, A.topk_idx[:, r])
+        assert (D.O_sel() - A.O_sel()[:, r]).abs().max().item() <= 1e-5
+        assert (D.s_out() - A.s_out()[:, r]).abs().max().item() <= 1e-5
+    assert A.device_status() == 0 and D.device_status() == 0
+    A.attention(dv["Q"], dv["Qs"], dv["Kc"], dv["Vc"],
+                torch.tensor([100, 517], dtype=torch.int32, device="cuda"))  # 517 + 3 = T
+    assert A.device_status(clear=True) == 8
+    out = A.concat.view(B, n, -1).cpu()
+    assert torch.isnan(out[1]).all() and torch.isfinite(out[0]).all()
