@@ -163,3 +163,27 @@ def test_append_rejects_bad_token_counts():
     need = _lib.gqe_append_workspace_size(dm, 5)
     assert need > _lib.gqe_append_workspace_size(dm, 1) == _lib.gqe_decode_workspace_size(dm)
     assert call(5, ws_bytes=need - 1) == 5
+
+
+def test_decode_wrapper_buffer_views_on_host():
+    """The torch wrapper's buffers and concat views (allocated on the host
+    here; nothing is launched): one W_O row per new token, laid out as
+    [O_sel | o_bar | shared head]."""
+    from moe_routed_grouped_b200.layer import GqeDecode
+    B, T, N, G, k, d, dm = 3, 600, 16, 8, 2, 64, 128
+    one = GqeDecode(B, T, N, G, k, d, dm, device="cpu")
+    assert one.concat.shape == (B, (G * k + G + 1) * d)
+    assert one.O_sel().shape == (B, G, k, d) and one.o_bar().shape == (B, G, d)
+    assert one.s_out().shape == (B, d) and one.topk_idx.shape == (B, G, k)
+    many = GqeDecode(B, T, N, G, k, d, dm, device="cpu", n_new=5)
+    assert many.concat.shape == (B * 5, (G * k + G + 1) * d)
+    assert many.O_sel().shape == (B, 5, G, k, d) and many.s_out().shape == (B, 5, d)
+    assert many.topk_idx.shape == (B, 5, G, k) and many.p.shape == (B, 5, G, N // G)
+    # the views alias the concat buffer in its column order
+    many.concat.zero_()
+    many.o_bar()[1, 2, 3] = 1.0
+    row = many.concat[1 * 5 + 2]
+    assert row[G * k * d + 3 * d: G * k * d + 4 * d].eq(1).all() and row.sum() == d
+    assert many.ws.numel() >= gqe.gqe_append_workspace_size(many.dims, 5)
+    with pytest.raises(gqe.GqeError):
+        GqeDecode(B, T, N, G, k, d, dm, device="cpu", n_new=65)
