@@ -187,3 +187,22 @@ def test_decode_wrapper_buffer_views_on_host():
     assert many.ws.numel() >= gqe.gqe_append_workspace_size(many.dims, 5)
     with pytest.raises(gqe.GqeError):
         GqeDecode(B, T, N, G, k, d, dm, device="cpu", n_new=65)
+
+
+def test_prefill_wrapper_buffer_views_on_host():
+    """GqePrefill's concat buffer (host allocation, nothing launched): slot j
+    of group g at (g*k + j)*d, then o_bar per group, then the shared head."""
+    from moe_routed_grouped_b200.layer import GqePrefill
+    B, S, N, G, k, d, dm = 2, 130, 16, 4, 3, 64, 64
+    L = GqePrefill(B, S, N, G, k, d, dm, device="cpu")
+    width = (G * k + G + 1) * d
+    assert L.concat.shape == (B * S, width)
+    assert L.O_sel().shape == (B, S, G, k, d) and L.o_bar().shape == (B, S, G, d)
+    assert L.s_out().shape == (B, S, d)
+    L.concat.zero_()
+    L.O_sel()[1, 7, 2, 1] = 2.0
+    L.s_out()[1, 7] = 3.0
+    row = L.concat[1 * S + 7]
+    assert row[(2 * k + 1) * d:(2 * k + 2) * d].eq(2).all()
+    assert row[width - d:].eq(3).all() and row.sum() == 5 * d
+    assert L.ws.numel() == gqe.gqe_workspace_size(L.dims)
