@@ -16,7 +16,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgqe.so")
 SOURCES = ["gqe_route.cu", "gqe_bucket.cu", "gqe_attn.cu", "gqe_decode.cu", "gqe_api.cu",
            "gqe_static.cu"]
-HEADERS = ["gqe_device.cuh", "gqe_internal.h"]
+HEADERS = ["gqe_device.cuh", "gqe_internal.h", "gqe_decode.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xptxas", "-v"]

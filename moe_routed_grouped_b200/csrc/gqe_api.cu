@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "gqe_decode.h"
 #include "gqe_internal.h"
 
 using namespace gqe;

@@ -15,8 +15,8 @@
 // adds the chunks, then writes the routed slots, o_bar and the shared head.
 #include <cuda_bf16.h>
 
+#include "gqe_decode.h"
 #include "gqe_device.cuh"
-#include "gqe_internal.h"
 
 namespace gqe {
 namespace {
