@@ -21,4 +21,10 @@ from .gqe_oracle import (  # noqa: F401
     dense_gqa_repeat,
     kv_cache_bytes,
     gqe_layer_prefill,
+    causal_attention_backward,
+    gqe_prefill_values,
+    gqe_prefill_backward,
+    router_values,
+    router_backward,
+    load_balance_loss,
 )

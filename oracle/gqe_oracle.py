@@ -478,3 +478,156 @@ def gqe_layer_prefill(x_bits, Wq_bits, Wk_bits, Wv_bits, Ws_bits, Wr_bits, Wo_bi
     concat = np.concatenate([O_sel.reshape(B, S, -1), o_bar.reshape(B, S, -1), s_out], axis=-1)
     return dict(y=concat @ Wo, Q=Q_bits, K=K_bits, V=V_bits, Qs=Qs_bits, topk_idx=idx, p=p,
                 w=w, concat=concat)
+
+
+# ---------------------------------------------------------------------------
+# backward pass (gradients of the path's outputs), on float64 values
+# ---------------------------------------------------------------------------
+
+def causal_attention_backward(q, pos, K, V, dO):
+    """Gradients of o_r = softmax_t(q_r . K_t / sqrt(d), t <= pos_r) V for one
+    query head: returns (dq, dK, dV) for the upstream gradient dO.
+
+    With S = q K^T / sqrt(d) (masked), P = softmax_rows(S), O = P V:
+    dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(dO * O)),
+    dq = dS K / sqrt(d), dK = dS^T q / sqrt(d).  Rows of dS outside the mask
+    are zero because P is.
+    """
+    q, K, V, dO = (np.asarray(a, dtype=np.float64) for a in (q, K, V, dO))
+    pos = np.asarray(pos, dtype=np.int64)
+    d = q.shape[1]
+    sc = _scale(d)
+    keys = np.arange(K.shape[0])
+    s = np.where(_visible(keys, pos), (q @ K.T) * sc, -np.inf)
+    P = np.exp(s - s.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    O = P @ V
+    dV = P.T @ dO
+    dP = dO @ V.T
+    dS = P * (dP - (dO * O).sum(axis=1, keepdims=True))
+    return (dS @ K) * sc, (dS.T @ q) * sc, dV
+
+
+def gqe_prefill_values(Q, Qs, K, V, topk_idx, w):
+    """:func:`gqe_prefill` on float64 values instead of bf16 bits (for
+    finite-difference checks of the backward pass)."""
+    Q, Qs, K, V, w = (np.asarray(a, dtype=np.float64) for a in (Q, Qs, K, V, w))
+    B, S, N, d = Q.shape
+    G = K.shape[2]
+    M = N // G
+    k = topk_idx.shape[-1]
+    r = np.arange(S)
+    O_sel = np.zeros((B, S, G, k, d))
+    s_out = np.zeros((B, S, d))
+    for b in range(B):
+        for g in range(G):
+            for j in range(k):
+                heads = _expert_head(g, topk_idx[b, :, g, j].astype(np.int64), M)
+                O_sel[b, :, g, j] = causal_attention(Q[b, r, heads], r, K[b, :, g], V[b, :, g])
+        s_out[b] = causal_attention(Qs[b], r, K[b, :, 0], V[b, :, 0])
+    o_bar = np.zeros((B, S, G, d))
+    for j in range(k):
+        o_bar = o_bar + w[:, :, :, j, None] * O_sel[:, :, :, j]
+    return O_sel, o_bar, s_out
+
+
+def gqe_prefill_backward(Q, Qs, K, V, topk_idx, w, dO_sel, do_bar, ds):
+    """Gradients of the path's outputs (O_sel, ō, s) with respect to its
+    inputs, for upstream gradients dO_sel [B,S,G,k,d], do_bar [B,S,G,d],
+    ds [B,S,d].  Returns dict(dQ [B,S,N,d] (zero for heads a token did not
+    select), dQs, dK, dV [B,S,G,d], dw [B,S,G,k]).
+
+    [GQA article] 训练与部署 共享键值的梯度归约: each query head's attention
+    backward is computed on its own, and dK, dV of a shared KV head are the
+    SUM of the contributions of every head that reads it (here the selected
+    routed heads of the group, plus the shared head for KV head 0); query
+    gradients stay with their own head.  [GQE review] 三个关键部件: ō =
+    sum_j w_j o_j, so slot j's output receives dO_sel_j + w_j dō and
+    dw_j = <dō, o_j> -- the differentiable signal the weighted-sum slot
+    gives the router.
+    """
+    Q, Qs, K, V, w = (np.asarray(a, dtype=np.float64) for a in (Q, Qs, K, V, w))
+    B, S, N, d = Q.shape
+    G = K.shape[2]
+    M = N // G
+    k = topk_idx.shape[-1]
+    r = np.arange(S)
+    dQ, dQs = np.zeros_like(Q), np.zeros_like(Qs)
+    dK, dV = np.zeros_like(K), np.zeros_like(V)
+    dw = np.zeros((B, S, G, k))
+    for b in range(B):
+        for g in range(G):
+            for j in range(k):
+                heads = _expert_head(g, topk_idx[b, :, g, j].astype(np.int64), M)
+                q = Q[b, r, heads]
+                o = causal_attention(q, r, K[b, :, g], V[b, :, g])
+                dw[b, :, g, j] = (do_bar[b, :, g] * o).sum(axis=1)
+                dO = dO_sel[b, :, g, j] + w[b, :, g, j, None] * do_bar[b, :, g]
+                dq, dk, dv = causal_attention_backward(q, r, K[b, :, g], V[b, :, g], dO)
+                dQ[b, r, heads] += dq
+                dK[b, :, g] += dk
+                dV[b, :, g] += dv
+        dq, dk, dv = causal_attention_backward(Qs[b], r, K[b, :, 0], V[b, :, 0], ds[b])
+        dQs[b] = dq
+        dK[b, :, 0] += dk
+        dV[b, :, 0] += dv
+    return dict(dQ=dQ, dQs=dQs, dK=dK, dV=dV, dw=dw)
+
+
+def router_values(x, Wr, bias, topk_idx):
+    """Router p and w on float64 values for a FIXED selection topk_idx
+    (the selection is discrete; gradients are taken with it held)."""
+    x, Wr = np.asarray(x, dtype=np.float64), np.asarray(Wr, dtype=np.float64)
+    l = np.einsum("bsc,gcm->bsgm", x, Wr)
+    if bias is not None:
+        l = l + np.asarray(bias, dtype=np.float64)
+    p = np.exp(l - l.max(axis=-1, keepdims=True))
+    p /= p.sum(axis=-1, keepdims=True)
+    ps = np.take_along_axis(p, topk_idx.astype(np.int64), axis=-1)
+    return p, ps / ps.sum(axis=-1, keepdims=True)
+
+
+def router_backward(x, Wr, bias, topk_idx, dw, dp_extra=None):
+    """Gradients through the router for upstream dw [B,S,G,k] (and an optional
+    direct dp [B,S,G,M], e.g. from an auxiliary loss).  [GQE review] 路由器
+    and 三个关键部件: w_j = p_{m_j} / sum_{j'} p_{m_j'} over the selected m_j,
+    p = softmax(l), l = x W_r[g] (+ bias).  Returns dict(dlogits, dx, dWr,
+    dbias).  At k = 1, w = 1 for any p, so dw carries no gradient.
+    """
+    x, Wr = np.asarray(x, dtype=np.float64), np.asarray(Wr, dtype=np.float64)
+    p, w = router_values(x, Wr, bias, topk_idx)
+    idx = topk_idx.astype(np.int64)
+    ps_sum = np.take_along_axis(p, idx, axis=-1).sum(axis=-1, keepdims=True)
+    dps = (dw - (dw * w).sum(axis=-1, keepdims=True)) / ps_sum  # d/dp of the selected ones
+    dp = np.zeros_like(p)
+    np.put_along_axis(dp, idx, dps, axis=-1)
+    if dp_extra is not None:
+        dp = dp + dp_extra
+    dl = p * (dp - (dp * p).sum(axis=-1, keepdims=True))
+    return dict(dlogits=dl, dx=np.einsum("bsgm,gcm->bsc", dl, Wr),
+                dWr=np.einsum("bsc,bsgm->gcm", x, dl), dbias=dl.sum(axis=(0, 1)))
+
+
+def load_balance_loss(p, topk_idx, alpha=1.0):
+    """Auxiliary load-balancing loss and its gradient with respect to p.
+
+    [GQE review] 为什么需要这些设计: training adds the standard MoE
+    load-balancing loss against routing collapse; the pages give no formula.
+    Reading: the Switch-Transformer form applied per group and averaged over
+    groups, L = alpha * mean_g M * sum_m f_{g,m} * P_{g,m}, with f the share of
+    the group's k*T selections that went to expert m (not differentiable) and
+    P the mean router probability of m over the T = B*S tokens.  Returns
+    (L, dL/dp [B,S,G,M]).
+    """
+    p = np.asarray(p, dtype=np.float64)
+    B, S, G, M = p.shape
+    T = B * S
+    k = topk_idx.shape[-1]
+    f = np.zeros((G, M))
+    for g in range(G):
+        f[g] = np.bincount(topk_idx[:, :, g, :].reshape(-1).astype(np.int64),
+                           minlength=M)[:M] / (T * k)
+    P = p.reshape(T, G, M).mean(axis=0)
+    L = alpha * M * (f * P).sum(axis=1).mean()
+    dp = np.broadcast_to(alpha * M * f / (G * T), p.shape).copy()
+    return L, dp

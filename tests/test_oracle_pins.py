@@ -736,3 +736,154 @@ def test_append_step_equals_prefill_rows():
         assert np.allclose(got[3], O_sel[:, sl], rtol=1e-12, atol=1e-12)
         assert np.allclose(got[4], o_bar[:, sl], rtol=1e-12, atol=1e-12)
         assert np.allclose(got[5], s[:, sl], rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# backward pass: every analytic gradient against central finite differences
+# --------------------------------------------------------------------------
+
+def _fd(f, x, eps=1e-6):
+    """Central differences of the scalar f at x (float64 array), all entries."""
+    g = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = x[i]
+        x[i] = old + eps
+        hi = f()
+        x[i] = old - eps
+        lo = f()
+        x[i] = old
+        g[i] = (hi - lo) / (2 * eps)
+    return g
+
+
+def test_attention_backward_matches_finite_differences():
+    rng = np.random.default_rng(11)
+    S, d = 6, 3
+    q, K, V = rng.standard_normal((S, d)), rng.standard_normal((S, d)), rng.standard_normal((S, d))
+    dO = rng.standard_normal((S, d))
+    pos = np.arange(S)
+    loss = lambda: float((oracle.causal_attention(q, pos, K, V) * dO).sum())  # noqa: E731
+    dq, dK, dV = oracle.causal_attention_backward(q, pos, K, V, dO)
+    for got, x in ((dq, q), (dK, K), (dV, V)):
+        assert np.allclose(got, _fd(loss, x), atol=1e-8, rtol=1e-6)
+    # the last key is seen by the last row only; row 0 sees key 0 only
+    assert np.allclose(dq[0], 0.0)           # one visible key: softmax weight 1, no q dependence
+
+
+def _bwd_case(seed, B=1, S=5, N=4, G=2, k=2, d=3):
+    rng = np.random.default_rng(seed)
+    M = N // G
+    idx = np.stack([rng.permutation(M)[:k] for _ in range(B * S * G)]).reshape(B, S, G, k)
+    w = rng.uniform(0.1, 1.0, (B, S, G, k))
+    w /= w.sum(axis=-1, keepdims=True)
+    t = dict(Q=rng.standard_normal((B, S, N, d)), Qs=rng.standard_normal((B, S, d)),
+             K=rng.standard_normal((B, S, G, d)), V=rng.standard_normal((B, S, G, d)), w=w)
+    up = dict(dO_sel=rng.standard_normal((B, S, G, k, d)), do_bar=rng.standard_normal((B, S, G, d)),
+              ds=rng.standard_normal((B, S, d)))
+    return idx, t, up
+
+
+def check_prefill_backward():
+    idx, t, up = _bwd_case(12)
+
+    def loss():
+        O, ob, s = oracle.gqe_prefill_values(t["Q"], t["Qs"], t["K"], t["V"], idx, t["w"])
+        return float((O * up["dO_sel"]).sum() + (ob * up["do_bar"]).sum() + (s * up["ds"]).sum())
+    g = oracle.gqe_prefill_backward(t["Q"], t["Qs"], t["K"], t["V"], idx, t["w"], up["dO_sel"],
+                                    up["do_bar"], up["ds"])
+    for name, key in (("dQ", "Q"), ("dQs", "Qs"), ("dK", "K"), ("dV", "V"), ("dw", "w")):
+        assert np.allclose(g[name], _fd(loss, t[key]), atol=1e-8, rtol=1e-6), name
+    # a head a token did not select gets no query gradient
+    N, G = t["Q"].shape[2], t["K"].shape[2]
+    M = N // G
+    for i in range(t["Q"].shape[1]):
+        for g_ in range(G):
+            for m in range(M):
+                if m not in idx[0, i, g_]:
+                    assert not g["dQ"][0, i, g_ * M + m].any()
+
+
+def test_prefill_backward_matches_finite_differences():
+    check_prefill_backward()
+
+
+def test_shared_kv_gradient_is_the_sum_over_its_heads():
+    """[GQA article] 训练与部署: the shared K/V gradient equals the reduction
+    (a sum, not a mean) of the backward run with K/V logically repeated per
+    query head.  Here: k = M (every head of a group active), the routed
+    backward against per-head backwards on repeated K/V."""
+    idx, t, up = _bwd_case(13, k=2)
+    B, S, N, d = t["Q"].shape
+    G = t["K"].shape[2]
+    M = N // G
+    g = oracle.gqe_prefill_backward(t["Q"], t["Qs"], t["K"], t["V"], idx, t["w"], up["dO_sel"],
+                                    up["do_bar"], up["ds"])
+    pos = np.arange(S)
+    dK = np.zeros_like(t["K"])
+    for g_ in range(G):
+        for m in range(M):
+            # rows whose slot j selected expert m, with their upstream gradient
+            dO = np.zeros((S, d))
+            sel = np.zeros(S, bool)
+            for j in range(2):
+                hit = idx[0, :, g_, j] == m
+                dO[hit] = up["dO_sel"][0, hit, g_, j] + t["w"][0, hit, g_, j, None] * up["do_bar"][0, hit, g_]
+                sel |= hit
+            assert sel.all()                  # k = M: every token uses every head
+            Krep = t["K"][0, :, g_].copy()    # this head's own copy of the shared K
+            _, dk, _ = oracle.causal_attention_backward(t["Q"][0, :, g_ * M + m], pos, Krep,
+                                                        t["V"][0, :, g_], dO)
+            dK[0, :, g_] += dk
+    _, dk, _ = oracle.causal_attention_backward(t["Qs"][0], pos, t["K"][0, :, 0], t["V"][0, :, 0],
+                                                up["ds"][0])
+    dK[0, :, 0] += dk
+    assert np.allclose(g["dK"], dK, atol=1e-12)
+    assert not np.allclose(g["dK"][0, :, 1], dK[0, :, 1] / M)   # a mean would differ
+
+
+def test_router_backward_matches_finite_differences():
+    rng = np.random.default_rng(14)
+    B, S, G, M, dm, k = 1, 4, 2, 4, 5, 2
+    x = rng.standard_normal((B, S, dm))
+    Wr = rng.standard_normal((G, dm, M)) * 0.5
+    bias = rng.standard_normal((G, M)) * 0.1
+    p, _ = oracle.router_values(x, Wr, bias, np.zeros((B, S, G, k), np.int64))
+    idx = np.argsort(-p, axis=-1, kind="stable")[..., :k]
+    dw = rng.standard_normal((B, S, G, k))
+    dpx = rng.standard_normal((B, S, G, M))
+
+    def loss():
+        p_, w_ = oracle.router_values(x, Wr, bias, idx)
+        return float((w_ * dw).sum() + (p_ * dpx).sum())
+    g = oracle.router_backward(x, Wr, bias, idx, dw, dp_extra=dpx)
+    assert np.allclose(g["dx"], _fd(loss, x), atol=1e-8, rtol=1e-6)
+    assert np.allclose(g["dWr"], _fd(loss, Wr), atol=1e-8, rtol=1e-6)
+    assert np.allclose(g["dbias"], _fd(loss, bias), atol=1e-8, rtol=1e-6)
+    # k = 1: w is 1 for any p, so the weighted-sum slot gives the router nothing
+    g1 = oracle.router_backward(x, Wr, bias, idx[..., :1], dw[..., :1])
+    assert np.allclose(g1["dlogits"], 0.0, atol=1e-15)
+
+
+def test_load_balance_loss_values_and_gradient():
+    """Balanced routing and uniform p give alpha; everything on one expert
+    with p concentrated there gives alpha * M; the gradient in p is exact."""
+    B, S, G, M, k = 2, 8, 3, 4, 1
+    p = np.full((B, S, G, M), 1.0 / M)
+    idx = (np.arange(B * S * G) % M).reshape(B, S, G, 1)
+    L, _ = oracle.load_balance_loss(p, idx, alpha=0.5)
+    assert np.isclose(L, 0.5)
+    p1 = np.zeros((B, S, G, M))
+    p1[..., 0] = 1.0
+    L1, _ = oracle.load_balance_loss(p1, np.zeros((B, S, G, 1), np.int64), alpha=0.5)
+    assert np.isclose(L1, 0.5 * M)
+    rng = np.random.default_rng(15)
+    pr = rng.uniform(size=(B, S, G, M))
+    pr /= pr.sum(-1, keepdims=True)
+    idr = rng.integers(0, M, (B, S, G, 2))
+    _, dp = oracle.load_balance_loss(pr, idr)
+    assert np.allclose(dp, _fd(lambda: oracle.load_balance_loss(pr, idr)[0], pr), atol=1e-9)
+
+
+ALL_CHECKS.append(check_prefill_backward)
