@@ -1,4 +1,6 @@
-"""Plain, slow CPU oracle for causal GQE prefill (float64).
+"""Plain, slow CPU oracle for GQE (float64): causal prefill, decode and
+append steps over a KV cache, the layer around them (projections, W_O) and
+the backward pass.
 
 TEST INFRASTRUCTURE ONLY.  Imported by ``tests/``, ``__graft_entry__.smoke()``
 and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py``; never by
@@ -34,7 +36,8 @@ Readings where the pages are silent:
 * Scale 1/sqrt(d), causal: key position <= query position (diagonal kept).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-(closed forms, the pages' worked values, brute force, invariants).
+(closed forms, the pages' worked values, brute force, invariants, central
+finite differences for the gradients).
 """
 from __future__ import annotations
 
