@@ -210,9 +210,12 @@ size_t gqe_decode_workspace_size(const gqe_dims* dims);
  * Output element type: float32 if dims->out_fp32 else bf16.  A position or
  * first slot out of range latches GQE_ERR_BAD_POSITION and that sequence's
  * outputs are NaN; an expert index out of range latches GQE_ERR_BAD_INDEX
- * and its slot and o_bar are NaN.  The cache is read once per step: each CTA serves every
- * selected head of its KV head (and the shared head for KV head 0) over one
- * chunk of keys, and a second kernel merges the chunks.
+ * and its slot and o_bar are NaN.  The cache is read once per step: each
+ * CTA serves every selected head of its KV head (and the shared head for KV
+ * head 0) over one chunk of keys, and a second kernel merges the chunks.
+ * Errors: GQE_ERR_INVALID_ARG / GQE_ERR_UNSUPPORTED for bad dims, null or
+ * misaligned pointers or a stride below d or not a multiple of 8;
+ * GQE_ERR_WORKSPACE when ws_bytes < gqe_decode_workspace_size(dims).
  */
 gqe_status gqe_attention_decode(const gqe_dims* dims, const void* Q, const void* Qs,
                                 const void* Kc, const void* Vc, const int32_t* pos,
