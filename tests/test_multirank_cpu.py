@@ -96,3 +96,42 @@ def test_decode_summary_counts_cache_bytes():
     assert s["roofline"]["frac"] == pytest.approx(kv / 0.4e-3 / 1e9 / 6650.0)
     assert s["roofline"]["bound"] == "hbm" and s["gpu_launches"] == 80
     assert s["config"]["mode"] == "decode" and s["config"]["position"] == w.S - 1
+
+
+def test_decode_measurement_code_path_on_host(monkeypatch):
+    """bench.measure_decode end to end on the host with the device parts
+    stubbed (CUDA events, synchronisation and the two library calls), so its
+    Python plumbing - input shapes, step loop, event bookkeeping, summary -
+    is exercised without a GPU."""
+    from synth import WORKLOADS
+    from moe_routed_grouped_b200.layer import GqeDecode
+
+    class FakeEvent:
+        def __init__(self, enable_timing=False):
+            pass
+
+        def record(self, stream=None):
+            pass
+
+        def elapsed_time(self, other):
+            return 0.25
+
+    calls = []
+    monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(GqeDecode, "route", lambda self, x, W, bias=None, stream=None:
+                        calls.append(("route", tuple(x.shape), tuple(W.shape))))
+    monkeypatch.setattr(GqeDecode, "attention", lambda self, Q, Qs, Kc, Vc, pos, kv_start=None,
+                        stream=None: calls.append(("attn", tuple(Q.shape), tuple(Kc.shape),
+                                                   int(pos[0]))))
+    monkeypatch.setattr(GqeDecode, "device_status", lambda self, clear=True, stream=None: 0)
+    w = WORKLOADS["tiny"]
+    r = bench.measure_decode(torch, w, torch.device("cpu"), 0, 4, 3, lambda: None)
+    assert len(r["step_ms"]) == 4 and r["attn_ms"] == 0.25
+    assert r["kv_bytes"] == 2 * w.B * w.S * w.G * w.d * 2
+    assert calls[0] == ("route", (w.B, w.d_model), (w.G, w.d_model, w.M))
+    assert calls[1] == ("attn", (w.B, w.N, w.d), (w.B, w.S, w.G, w.d), w.S - 1)
+    assert len(calls) == 2 * (4 + 3)
+    s = bench.decode_summary(w, 1, 4, sum(r["step_ms"]), r["attn_ms"], r["kv_bytes"],
+                             {"hbm_gbs": 6650.0}, "measured")
+    assert s["value"] == pytest.approx(w.B * 4 / (sum(r["step_ms"]) / 1e3))
