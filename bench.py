@@ -353,6 +353,33 @@ def decode_summary(w, world, steps, tot_ms, attn_ms, kv_bytes, peaks, peak_src):
     }
 
 
+def decode_entries(torch, device, rank, local, flush, peaks, peak_src,
+                   names=("layer250m", "million"), steps=20, warmup=3):
+    """The decode step at the bench's own shape and over a 1M-token cache, for
+    the prefill line (one GPU).  A failure becomes an entry with its error,
+    so the prefill numbers of the line stand."""
+    dec = []
+    for name in names:
+        wd = WORKLOADS[name]
+        cs = ClockSampler(local)
+        cs.start()
+        try:
+            r = measure_decode(torch, wd, device, rank, steps, warmup, flush)
+            cs.stop()
+            e = decode_summary(wd, 1, steps, sum(r["step_ms"]), r["attn_ms"], r["kv_bytes"],
+                               peaks, peak_src)
+            e.update(workload=name, steps=steps, warmup=warmup,
+                     clocks=cs.summary(r["t0"], r["t1"]))
+            dec.append(e)
+            del r
+        except Exception as ex:  # noqa: BLE001
+            dec.append({"workload": name, "error": f"{type(ex).__name__}: {ex}"[:300]})
+        finally:
+            cs.stop()
+        torch.cuda.empty_cache()
+    return dec
+
+
 def run_decode(args, torch, w, device, rank, world, dist, peaks, peak_src, flush):
     """`--decode`: the decode step alone, as its own contract line."""
     clocks = ClockSampler(device.index)
@@ -598,31 +625,10 @@ def main():
         line["sweep"] = sweep
 
     if world == 1 and not args.no_decode:
-        # the decode step (one new token per sequence over a full cache) at the
-        # bench's own shape and over a 1M-token cache; a failure here is
-        # reported in the line and leaves the prefill numbers above standing
         if "res" in locals():
             del res
         torch.cuda.empty_cache()
-        dec = []
-        for name in ("layer250m", "million"):
-            wd = WORKLOADS[name]
-            cs = ClockSampler(local)
-            cs.start()
-            try:
-                r = measure_decode(torch, wd, device, rank, 20, 3, flush)
-                cs.stop()
-                e = decode_summary(wd, world, 20, sum(r["step_ms"]), r["attn_ms"], r["kv_bytes"],
-                                   peaks, peak_src)
-                e.update(workload=name, steps=20, warmup=3, clocks=cs.summary(r["t0"], r["t1"]))
-                dec.append(e)
-                del r
-            except Exception as ex:  # noqa: BLE001
-                dec.append({"workload": name, "error": f"{type(ex).__name__}: {ex}"[:300]})
-            finally:
-                cs.stop()
-            torch.cuda.empty_cache()
-        line["decode"] = dec
+        line["decode"] = decode_entries(torch, device, rank, local, flush, peaks, peak_src)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = make_inputs(w)

@@ -135,3 +135,21 @@ def test_decode_measurement_code_path_on_host(monkeypatch):
     s = bench.decode_summary(w, 1, 4, sum(r["step_ms"]), r["attn_ms"], r["kv_bytes"],
                              {"hbm_gbs": 6650.0}, "measured")
     assert s["value"] == pytest.approx(w.B * 4 / (sum(r["step_ms"]) / 1e3))
+
+
+def test_decode_entries_report_failures_in_place(monkeypatch):
+    """The prefill line's decode list: one entry per workload, and a failing
+    measurement becomes an entry with its error instead of ending the run."""
+    def fake(torch_, w, device, rank, steps, warmup, flush):
+        if w.name == "layer250m":
+            raise RuntimeError("device status 8 in the decode loop")
+        return dict(step_ms=[0.5] * steps, attn_ms=0.4, t0=0.0, t1=1.0,
+                    kv_bytes=2 * w.B * w.S * w.G * w.d * 2)
+    monkeypatch.setattr(bench, "measure_decode", fake)
+    dec = bench.decode_entries(torch, torch.device("cpu"), 0, 0, lambda: None,
+                               {"hbm_gbs": 6650.0}, "measured", names=("tiny", "layer250m"),
+                               steps=5, warmup=3)
+    assert [e["workload"] for e in dec] == ["tiny", "layer250m"]
+    assert dec[0]["unit"] == "tokens/s" and dec[0]["steps"] == 5 and "clocks" in dec[0]
+    assert dec[1] == {"workload": "layer250m",
+                      "error": "RuntimeError: device status 8 in the decode loop"}
