@@ -10,6 +10,28 @@ import torch
 from . import _lib
 
 
+def _device(device) -> torch.device:
+    dev = torch.device(device)
+    if dev.type == "cuda" and dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    return dev
+
+
+def _expect(t, name, shape, dtype, device):
+    """The C ABI takes raw pointers and cannot see shapes, so each tensor is
+    checked here: a wrong shape would otherwise be read out of bounds."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+
+
 class GqePrefill:
     """Buffers and calls for one (B, S, N, G, k, d, d_model) shape.
 
@@ -27,7 +49,7 @@ class GqePrefill:
         nbytes = _lib.gqe_workspace_size(self.dims)
         if nbytes == 0:
             raise _lib.GqeError(2, "gqe_workspace_size")
-        dev = torch.device(device)
+        dev = _device(device)
         self.device = dev
         self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
         self.out_dtype = torch.float32 if out_fp32 else torch.bfloat16
@@ -50,10 +72,24 @@ class GqePrefill:
         return self.concat[:, (self.G * self.k + self.G) * self.d:].view(self.B, self.S, self.d)
 
     def route(self, x, W_r, bias=None, stream=None):
+        bf, dv = torch.bfloat16, self.device
+        _expect(x, "x", (self.B, self.S, self.d_model), bf, dv)
+        _expect(W_r, "W_r", (self.G, self.d_model, self.M), bf, dv)
+        if bias is not None:
+            _expect(bias, "bias", (self.G, self.M), torch.float32, dv)
         _lib.gqe_route(self.dims, x, W_r, bias, self.topk_idx, self.p, self.w, self.ws, stream)
         return self.topk_idx, self.p, self.w
 
+    def _check_qkv(self, Q, K, V, Qs=None):
+        bf, dv = torch.bfloat16, self.device
+        _expect(Q, "Q", (self.B, self.S, self.N, self.d), bf, dv)
+        _expect(K, "K", (self.B, self.S, self.G, self.d), bf, dv)
+        _expect(V, "V", (self.B, self.S, self.G, self.d), bf, dv)
+        if Qs is not None:
+            _expect(Qs, "Qs", (self.B, self.S, self.d), bf, dv)
+
     def attention(self, Q, Qs, K, V, stream=None):
+        self._check_qkv(Q, K, V, Qs)
         a = self.G * self.k * self.d
         base = self.concat
         esz = base.element_size()
@@ -68,6 +104,9 @@ class GqePrefill:
         return self.attention(Q, Qs, K, V, stream)
 
     def dense(self, Q, K, V, out=None, stream=None):
+        self._check_qkv(Q, K, V)
+        if out is not None:
+            _expect(out, "out", (self.B, self.S, self.N, self.d), self.out_dtype, self.device)
         if out is None:
             if self._dense_out is None:
                 self._dense_out = torch.empty(self.B, self.S, self.N, self.d, dtype=self.out_dtype,
@@ -105,7 +144,7 @@ class GqeDecode:
         b = _lib.gqe_append_workspace_size(self.dims, n_new)
         if a == 0 or b == 0:
             raise _lib.GqeError(2, "gqe_append_workspace_size")
-        dev = torch.device(device)
+        dev = _device(device)
         self.device = dev
         self.ws = torch.zeros(max(a, b), dtype=torch.uint8, device=dev)
         self.out_dtype = torch.float32 if out_fp32 else torch.bfloat16
@@ -129,6 +168,11 @@ class GqeDecode:
 
     def route(self, x, W_r, bias=None, stream=None):
         """x: bf16 [B, d_model] (the new tokens; [B, n_new, d_model] if n_new > 1)."""
+        bf, dv = torch.bfloat16, self.device
+        _expect(x, "x", (*self._lead, self.d_model), bf, dv)
+        _expect(W_r, "W_r", (self.G, self.d_model, self.M), bf, dv)
+        if bias is not None:
+            _expect(bias, "bias", (self.G, self.M), torch.float32, dv)
         _lib.gqe_route(self.route_dims, x, W_r, bias, self.topk_idx, self.p, self.w, self.ws,
                        stream)
         return self.topk_idx, self.p, self.w
@@ -137,6 +181,14 @@ class GqeDecode:
         """Q [B, N, d], Qs [B, d] (n_new axis after B if n_new > 1), caches
         [B, T, G, d] (bf16), pos int32 [B] (slot of the first new token);
         kv_start int32 [B] (first valid slot, left padding) or None."""
+        bf, dv = torch.bfloat16, self.device
+        _expect(Q, "Q", (*self._lead, self.N, self.d), bf, dv)
+        _expect(Qs, "Qs", (*self._lead, self.d), bf, dv)
+        _expect(Kc, "Kc", (self.B, self.T, self.G, self.d), bf, dv)
+        _expect(Vc, "Vc", (self.B, self.T, self.G, self.d), bf, dv)
+        _expect(pos, "pos", (self.B,), torch.int32, dv)
+        if kv_start is not None:
+            _expect(kv_start, "kv_start", (self.B,), torch.int32, dv)
         a = self.G * self.k * self.d
         flat = self.concat.view(-1)
         if self.n_new == 1:

@@ -206,3 +206,43 @@ def test_prefill_wrapper_buffer_views_on_host():
     assert row[(2 * k + 1) * d:(2 * k + 2) * d].eq(2).all()
     assert row[width - d:].eq(3).all() and row.sum() == 5 * d
     assert L.ws.numel() == gqe.gqe_workspace_size(L.dims)
+
+
+def test_wrappers_refuse_wrong_tensors_before_any_call():
+    """Raw pointers carry no shape, so the torch wrappers check each tensor's
+    shape, dtype, layout and device first (host tensors here; nothing is
+    launched)."""
+    import torch
+    from moe_routed_grouped_b200.layer import GqeDecode, GqePrefill
+    B, S, N, G, k, d, dm = 1, 64, 16, 8, 1, 64, 64
+    L = GqePrefill(B, S, N, G, k, d, dm, device="cpu")
+    bf = torch.bfloat16
+    x = torch.zeros(B, S, dm, dtype=bf)
+    W = torch.zeros(G, dm, N // G, dtype=bf)
+    with pytest.raises(ValueError, match="x: shape"):
+        L.route(torch.zeros(B, S + 1, dm, dtype=bf), W)
+    with pytest.raises(ValueError, match="W_r: dtype"):
+        L.route(x, W.float())
+    with pytest.raises(ValueError, match="bias: dtype"):
+        L.route(x, W, torch.zeros(G, N // G, dtype=torch.float64))
+    Q = torch.zeros(B, S, N, d, dtype=bf)
+    K = torch.zeros(B, S, G, d, dtype=bf)
+    with pytest.raises(ValueError, match="Q: must be contiguous"):
+        L.attention(Q.transpose(1, 2).contiguous().transpose(1, 2), torch.zeros(B, S, d, dtype=bf),
+                    K, K)
+    with pytest.raises(ValueError, match="V: shape"):
+        L.dense(Q, K, torch.zeros(B, S, G, d + 1, dtype=bf))
+    with pytest.raises(TypeError):
+        L.dense(Q, K, object())
+    D = GqeDecode(2, 100, N, G, k, d, dm, device="cpu")
+    with pytest.raises(ValueError, match="pos: dtype"):
+        D.attention(torch.zeros(2, N, d, dtype=bf), torch.zeros(2, d, dtype=bf),
+                    torch.zeros(2, 100, G, d, dtype=bf), torch.zeros(2, 100, G, d, dtype=bf),
+                    torch.zeros(2, dtype=torch.int64))
+    with pytest.raises(ValueError, match="Kc: shape"):
+        D.attention(torch.zeros(2, N, d, dtype=bf), torch.zeros(2, d, dtype=bf),
+                    torch.zeros(2, 99, G, d, dtype=bf), torch.zeros(2, 100, G, d, dtype=bf),
+                    torch.zeros(2, dtype=torch.int32))
+    A = GqeDecode(2, 100, N, G, k, d, dm, device="cpu", n_new=3)
+    with pytest.raises(ValueError, match="x: shape"):
+        A.route(torch.zeros(2, dm, dtype=bf), W)      # needs the n_new axis
