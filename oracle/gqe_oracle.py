@@ -99,6 +99,15 @@ def _visible(key_pos: np.ndarray, query_pos: np.ndarray, key_start=None) -> np.n
 # router
 # ---------------------------------------------------------------------------
 
+def _group_softmax(L: np.ndarray) -> np.ndarray:
+    """[GQE review] 路由器: p_{i,g} = softmax(r_g(x_i)), over the group's M
+    experts only (the last axis), in float64; the maximum is subtracted
+    before exponentiating, which leaves the quotient unchanged."""
+    mx = L.max(axis=-1, keepdims=True)
+    e = np.exp(L - mx)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
 def router_logits(x: np.ndarray, Wr: np.ndarray, bias: Optional[np.ndarray]
                   ) -> Tuple[np.ndarray, np.ndarray]:
     """Router logits l[t, g, m] = sum_j x[t, j] W_r[g, j, m] (+ bias[g, m]).
@@ -203,10 +212,7 @@ def route(x_bits: np.ndarray, Wr_bits: np.ndarray, bias: Optional[np.ndarray], k
         # take the correctly rounded logits of this pair
         L[t, g] = exact_logits(xt, Wr[g], bg)
 
-    # p = softmax over the group's M experts (float64)
-    mx = L.max(axis=-1, keepdims=True)
-    e = np.exp(L - mx)
-    p = e / e.sum(axis=-1, keepdims=True)
+    p = _group_softmax(L)
     psel = np.take_along_axis(p, idx, axis=-1)
     den = np.zeros(psel.shape[:-1])
     for j in range(k):  # ascending slot order

@@ -370,6 +370,63 @@ def test_router_sums():
     check_router_sums()
 
 
+def _exact_logit(x_row, w_col, bias=0.0):
+    """The exact logit sum_j x_j w_j + bias as a Fraction (bf16 values and a
+    float32 bias are exact binary fractions)."""
+    return sum((Fraction(float(a)) * Fraction(float(b)) for a, b in zip(x_row, w_col)),
+               Fraction(float(bias)))
+
+
+def check_router_p_values():
+    """p = softmax of the group's logits ([GQE review] 路由器), pinned by facts
+    the test derives without a softmax of its own:
+    (a) two experts whose exact logit gap is D: p_0 = 1 / (1 + e^-D), the
+        logistic function;
+    (b) identical W_r columns: every expert gets exactly 1/M;
+    (c) x = 0 and bias b_m = ln(m + 1): p_m = (m + 1) / 10 (up to the float32
+        rounding of the logarithms), in every group;
+    (d) random logits with a bias: log p_a - log p_b is the exact logit
+        difference l_a - l_b."""
+    # (a) M = 2: the logistic closed form
+    xb = normal_bf16((1, 24, 16), 51)
+    Wb = normal_bf16((3, 16, 2), 52, std=0.3)
+    _, p, _, _ = oracle.route(xb, Wb, None, 1)
+    xf = bf16_bits_to_f32(xb).astype(np.float64)[0]
+    Wf = bf16_bits_to_f32(Wb).astype(np.float64)
+    for t in range(24):
+        for g in range(3):
+            D = float(_exact_logit(xf[t], Wf[g][:, 0]) - _exact_logit(xf[t], Wf[g][:, 1]))
+            want = 1.0 / (1.0 + math.exp(-D))
+            assert abs(p[0, t, g, 0] - want) <= 1e-14, (t, g, p[0, t, g, 0], want)
+            assert abs(p[0, t, g, 1] - (1.0 - want)) <= 1e-14, (t, g)
+    # (b) M = 4 identical columns: 1/M exactly, w = 1/k exactly
+    Wb4 = np.repeat(normal_bf16((2, 16, 1), 53, std=0.3), 4, axis=2)
+    for k in (1, 2, 4):
+        _, p4, w4, _ = oracle.route(xb, Wb4, None, k)
+        assert (p4 == 0.25).all(), p4.min()
+        assert (w4 == 1.0 / k).all()
+    # (c) logits = bias = ln(m + 1): p proportional to m + 1
+    zero = np.zeros((1, 8, 16), np.uint16)
+    bias = np.tile(np.log(np.arange(1, 5, dtype=np.float64)).astype(np.float32), (2, 1))
+    _, pc, _, _ = oracle.route(zero, Wb4, bias, 1)
+    assert np.abs(pc - np.array([0.1, 0.2, 0.3, 0.4])).max() <= 1e-6, pc[0, 0]
+    # (d) log-ratios are the exact logit differences (bias included)
+    Wr = normal_bf16((2, 16, 3), 54, std=0.5)
+    br = np.array([[0.75, -1.25, 0.0], [2.5, 0.5, -0.375]], np.float32)
+    _, pd, _, _ = oracle.route(xb[:, :8], Wr, br, 1)
+    Wrf = bf16_bits_to_f32(Wr).astype(np.float64)
+    for t in range(8):
+        for g in range(2):
+            ls = [_exact_logit(xf[t], Wrf[g][:, m], br[g, m]) for m in range(3)]
+            for a, b in ((0, 1), (0, 2), (1, 2)):
+                got = math.log(pd[0, t, g, a]) - math.log(pd[0, t, g, b])
+                assert abs(got - float(ls[a] - ls[b])) <= 1e-12, (t, g, a, b)
+
+
+def test_router_p_values():
+    check_router_p_values()
+
+
 # --------------------------------------------------------------------------
 # buckets
 # --------------------------------------------------------------------------
@@ -579,7 +636,8 @@ ALL_CHECKS = [check_kv_bytes, check_worked_examples, check_worked_example_routed
               check_geometric_scores, check_nonsquare_positions, check_head_to_kv_map,
               check_row0_and_hull, check_explicit_equals_repeat, check_router_sums,
               check_routed_kM_equals_dense, check_shared_head_is_dense_head_on_kv0,
-              check_k1_obar, check_obar_weighted_sum_k2, check_padding_key_validity]
+              check_k1_obar, check_obar_weighted_sum_k2, check_padding_key_validity,
+              check_router_p_values]
 
 
 def _caught(monkeypatch, name, fn):
@@ -603,10 +661,30 @@ def _caught(monkeypatch, name, fn):
     ("_scale", lambda d: 1.0 / d),                                  # wrong scale
     ("_kv_head_of", lambda h, N, G: h % G),                         # interleaved map
     ("_expert_head", lambda g, m, M: m * M + g),                    # transposed roles
+    ("_group_softmax", lambda L: _plain_softmax(2.0 * L)),          # temperature 1/2
+    ("_group_softmax", lambda L: _plain_softmax(0.5 * L)),          # temperature 2
+    ("_group_softmax", lambda L: _plain_softmax(-L)),               # sign of the logits
+    ("_group_softmax", lambda L: _plain_softmax(                     # over every head of
+        L.reshape(*L.shape[:-2], -1)).reshape(L.shape)),            # the token, not the group
 ])
 def test_planted_mistakes_are_caught(monkeypatch, name, fn):
     failed = _caught(monkeypatch, name, fn)
     assert failed, f"planted mistake in {name} went unnoticed"
+
+
+def _plain_softmax(L):
+    """Softmax over the last axis; used only to build planted mistakes."""
+    e = np.exp(L - L.max(axis=-1, keepdims=True))
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def test_planted_router_bias_sign_is_caught(monkeypatch):
+    """A bias entering the logits with the wrong sign must fail a pin."""
+    good = og.router_logits
+    monkeypatch.setattr(og, "router_logits",
+                        lambda x, Wr, bias: good(x, Wr, None if bias is None else -bias))
+    with pytest.raises(AssertionError):
+        check_router_p_values()
 
 
 def test_planted_kv_bytes_mistake(monkeypatch):
