@@ -148,21 +148,36 @@ gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void
  * the same outputs, and allocates nothing: its scratch is one 64 MiB device
  * array compiled into the library, present on every GPU that loads it until
  * the process exits.
- *  - The first call on a device looks up that array's device address (and
- *    zeroes its header) with the device current; make that first call before
- *    any stream capture.
+ *  - Every call looks up that array's device address with the device current
+ *    (host code cannot use the array's name as an address); the first call
+ *    on a device, and the first after its context was rebuilt, also zeroes
+ *    the array's header with a synchronous cudaMemset.  Make that first call
+ *    before any stream capture.
  *  - Shapes whose scratch (V in fp16, token lists, work list) exceeds
  *    64 MiB return GQE_ERR_WORKSPACE without launching anything.
  *  - All calls on a device share the one array and it keeps the previous
- *    call's contents (the call clears what must start at zero).  Calls that
- *    overlap on the GPU - different streams, or different host threads -
- *    race on it and give wrong results; order them.
- *  - Device-side errors are latched in the array and are not reported.
+ *    call's contents (each call clears the counters that must start at
+ *    zero).  Calls that overlap on the GPU - different streams, or different
+ *    host threads - race on it and give wrong results; order them.
+ *  - Device-side errors (an expert index outside [0, M), V outside the fp16
+ *    range, a bounded wait that ran out) are latched into a status word at
+ *    the start of the array, as the workspace calls latch them into theirs.
+ *    The word keeps the first error until gqe_static_device_status clears it.
  */
 gqe_status gqe_attention_prefill_static(const gqe_dims* dims, const void* Q, const void* Qs,
                                         const void* K, const void* V, const int32_t* topk_idx,
                                         const float* w, void* O_sel, void* o_bar, void* s_out,
                                         int64_t out_row_stride, void* stream);
+
+/*
+ * gqe_static_device_status - read (and with clear != 0 reset) the status
+ * word that gqe_attention_prefill_static latches device-side errors into, on
+ * the current device.  Like gqe_attention_prefill_static it has no
+ * counterpart in the sources.  Synchronises `stream` first, so the value
+ * covers every static call queued on it; returns GQE_OK or the latched
+ * gqe_status, and GQE_ERR_CUDA if the read itself failed.
+ */
+gqe_status gqe_static_device_status(int32_t clear, void* stream);
 
 /*
  * gqe_dense_gqa_prefill - the all-active GQA baseline ("16 heads all

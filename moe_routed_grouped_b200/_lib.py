@@ -19,6 +19,7 @@ EXPORTS = (
     "gqe_status_string", "gqe_selftest_bounded_wait", "gqe_set_profile_events",
     "gqe_attention_prefill_static", "gqe_set_pair_threshold", "gqe_decode_workspace_size",
     "gqe_attention_decode", "gqe_append_workspace_size", "gqe_attention_append",
+    "gqe_static_device_status",
 )
 
 STATUS = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED", 3: "GQE_ERR_CUDA",
@@ -60,6 +61,7 @@ def _load() -> ctypes.CDLL:
         "gqe_attention_decode": (I32, [S, P, P, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
         "gqe_append_workspace_size": (SZ, [S, I32]),
         "gqe_attention_append": (I32, [S, I32, P, P, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
+        "gqe_static_device_status": (I32, [I32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -164,6 +166,11 @@ def gqe_attention_prefill_static(dm, Q, Qs, K, V, topk_idx, w, O_sel, o_bar, s_o
                                          _ptr(topk_idx), _ptr(w), _ptr(O_sel), _ptr(o_bar),
                                          _ptr(s_out), int(out_row_stride), _stream(stream))
     return _check(r, "gqe_attention_prefill_static") if check else r
+
+
+def gqe_static_device_status(clear=1, stream=None) -> int:
+    """Status word of gqe_attention_prefill_static on the current device."""
+    return LIB.gqe_static_device_status(int(clear), _stream(stream))
 
 
 def gqe_decode_workspace_size(dm: GqeDims) -> int:

@@ -14,104 +14,7 @@ using namespace gqe;
 
 namespace {
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// Tiled map over a row-major tensor; dims innermost first, strides in bytes
-// for dims 1..rank-1; box of 64 elements (128 B, the swizzle span) x rows.
-bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
-                const uint64_t* dims, const uint64_t* strides, const uint32_t* box) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gd[5], gs[4];
-  cuuint32_t bx[5], es[5];
-  for (int i = 0; i < rank; ++i) {
-    gd[i] = dims[i];
-    bx[i] = box[i];
-    es[i] = 1;
-  }
-  for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
-  return fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gd, gs, bx, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// [B, S, H, d] (H heads) -> 4-D map with a {64, 1, 128, 1} box
-bool map_bshd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, int S, int H,
-              int d) {
-  const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(H),
-                            static_cast<uint64_t>(S), static_cast<uint64_t>(B)};
-  const uint64_t strides[3] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(H) * d * 2,
-                               static_cast<uint64_t>(S) * H * d * 2};
-  const uint32_t box[4] = {64, 1, static_cast<uint32_t>(kTileM), 1};
-  return encode_map(m, dt, 4, base, dims, strides, box);
-}
-
-// [B, S, d] -> 3-D map with a {64, 128, 1} box
-bool map_bsd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, int S, int d) {
-  const uint64_t dims[3] = {static_cast<uint64_t>(d), static_cast<uint64_t>(S),
-                            static_cast<uint64_t>(B)};
-  const uint64_t strides[2] = {static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(S) * d * 2};
-  const uint32_t box[3] = {64, static_cast<uint32_t>(kTileM), 1};
-  return encode_map(m, dt, 3, base, dims, strides, box);
-}
-
-bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// Shape checks shared by all entry points.  Unsupported combinations are
-// refused explicitly (never silently remapped).
-gqe_status check_dims(const gqe_dims* d, bool router) {
-  if (!d) return GQE_ERR_INVALID_ARG;
-  if (d->B < 1 || d->S < 1 || d->N < 1 || d->G < 1 || d->k < 1 || d->d < 1)
-    return GQE_ERR_INVALID_ARG;
-  if (d->N % d->G != 0) return GQE_ERR_INVALID_ARG;
-  const int64_t M = d->N / d->G;
-  if (d->k > M) return GQE_ERR_INVALID_ARG;
-  if (d->out_fp32 != 0 && d->out_fp32 != 1) return GQE_ERR_INVALID_ARG;
-  if (M > kMaxM) return GQE_ERR_UNSUPPORTED;
-  if (d->d != 64 && d->d != 128) return GQE_ERR_UNSUPPORTED;
-  const int64_t B = d->B, S = d->S, G = d->G, k = d->k;
-  const int64_t wide = k > M ? k : M;
-  if (B * S * G * wide >= (int64_t(1) << 31)) return GQE_ERR_UNSUPPORTED;
-  if (B * S * d->N >= (int64_t(1) << 31)) return GQE_ERR_UNSUPPORTED;
-  if (B * G * M >= (int64_t(1) << 24) || B >= (int64_t(1) << 24)) return GQE_ERR_UNSUPPORTED;
-  const int64_t nq = (S + kTileM - 1) / kTileM;
-  if ((nq + 2) * 4 > 200 * 1024) return GQE_ERR_UNSUPPORTED;  // scheduler histogram
-  if (router) {
-    if (d->d_model < 8 || d->d_model % 8 != 0) return GQE_ERR_UNSUPPORTED;
-    const int64_t gm = G * M;
-    if (gm != 4 && gm != 8 && gm != 16 && gm != 32) return GQE_ERR_UNSUPPORTED;
-  }
-  return GQE_OK;
-}
-
 gqe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
-
-cudaEvent_t g_prof_begin = nullptr, g_prof_end = nullptr;
-
-cudaError_t timed_attention(const AttnArgs& a, int64_t n_list, cudaStream_t s) {
-  const bool prof = g_prof_begin && g_prof_end;
-  if (prof && cudaEventRecord(g_prof_begin, s) != cudaSuccess) return cudaErrorUnknown;
-  cudaError_t e = launch_attention(a, n_list, s);
-  if (e == cudaSuccess && prof) e = cudaEventRecord(g_prof_end, s);
-  return e;
-}
 
 }  // namespace
 
@@ -405,8 +308,7 @@ const char* gqe_status_string(gqe_status s) {
 }
 
 void gqe_set_profile_events(void* begin, void* end) {
-  g_prof_begin = static_cast<cudaEvent_t>(begin);
-  g_prof_end = static_cast<cudaEvent_t>(end);
+  set_profile_events(static_cast<cudaEvent_t>(begin), static_cast<cudaEvent_t>(end));
 }
 
 gqe_status gqe_selftest_bounded_wait(void* ws, size_t ws_bytes, int32_t limit_us, void* stream) {

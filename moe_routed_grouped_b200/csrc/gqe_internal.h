@@ -167,4 +167,21 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 
 cudaError_t launch_selftest_wait(int* status, uint64_t limit_ns, cudaStream_t st);
 
+// ------------------------------------------------------------ host helpers
+// (gqe_host.cu; shared by every entry point)
+bool aligned16(const void* p);
+// Shape checks: unsupported combinations are refused, never remapped.
+gqe_status check_dims(const gqe_dims* d, bool router);
+// Tiled TMA map over a row-major tensor (dims innermost first, byte strides
+// for dims 1..rank-1), 128-byte swizzle.
+bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
+                const uint64_t* dims, const uint64_t* strides, const uint32_t* box);
+// [B, S, H, d] -> 4-D map with a {64, 1, 128, 1} box; [B, S, d] -> {64, 128, 1}.
+bool map_bshd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, int S, int H,
+              int d);
+bool map_bsd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, int S, int d);
+// The attention launch, bracketed by the profiling events when they are set.
+void set_profile_events(cudaEvent_t begin, cudaEvent_t end);
+cudaError_t timed_attention(const AttnArgs& a, int64_t n_list, cudaStream_t s);
+
 }  // namespace gqe

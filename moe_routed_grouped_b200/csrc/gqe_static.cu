@@ -24,10 +24,6 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-// Device address of g_static_scratch on each device, looked up once.
-void* g_scratch_ptr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
 // Regions of the static scratch: status word, counters, then the same
 // attention regions as a caller workspace (the router regions are unused).
 struct StaticLayout {
@@ -51,68 +47,31 @@ StaticLayout static_layout(const gqe_dims& d) {
   return L;
 }
 
-// Once per device, with that device current: the device address of the
-// static array (host code only sees a host-side stand-in for its name), and
-// a zeroed header.
+// The last device address of g_static_scratch seen on each device.  In host
+// code the array's name is only a host-side stand-in, so the address is
+// looked up with the device current on every call (a cheap host-side
+// lookup): if the context was torn down and rebuilt, the module is reloaded
+// and the array may move.  A new address means a freshly loaded module; its
+// header (status word and counters) is zeroed before first use.
+void* g_seen[kMaxDevices] = {};
+std::mutex g_seen_mu;
+
 cudaError_t scratch_for_current_device(uint8_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (e != cudaSuccess) return e;
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_seen_mu);
+  if (g_seen[dev] != p) {
     e = cudaMemset(p, 0, 512);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+    g_seen[dev] = p;
   }
-  *out = static_cast<uint8_t*>(g_scratch_ptr[dev]);
+  *out = static_cast<uint8_t*>(p);
   return cudaSuccess;
-}
-
-bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// Tiled TMA map, 128-byte swizzle, box of 64 elements x 128 rows; dims
-// innermost first, byte strides for dims 1..rank-1.
-bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
-            const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return false;
-    fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  return fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool map_bshd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, int S, int H,
-              int d) {
-  const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(S), cuuint64_t(B)};
-  const cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H) * d * 2,
-                                 cuuint64_t(S) * H * d * 2};
-  const cuuint32_t box[4] = {64, 1, gqe::kTileM, 1};
-  return encode(m, dt, 4, base, dims, strides, box);
-}
-
-bool map_bsd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, int S, int d) {
-  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(S), cuuint64_t(B)};
-  const cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(S) * d * 2};
-  const cuuint32_t box[3] = {64, gqe::kTileM, 1};
-  return encode(m, dt, 3, base, dims, strides, box);
 }
 
 }  // namespace
@@ -121,17 +80,11 @@ extern "C" gqe_status gqe_attention_prefill_static(
     const gqe_dims* dims, const void* Q, const void* Qs, const void* K, const void* V,
     const int32_t* topk_idx, const float* w, void* O_sel, void* o_bar, void* s_out,
     int64_t out_row_stride, void* stream) {
-  // the shape checks of gqe_attention_prefill
-  if (gqe_workspace_size(dims) == 0) {
-    if (!dims || dims->B < 1 || dims->S < 1 || dims->N < 1 || dims->G < 1 || dims->k < 1 ||
-        dims->d < 1 || dims->N % dims->G != 0 || dims->k > dims->N / dims->G ||
-        (dims->out_fp32 != 0 && dims->out_fp32 != 1))
-      return GQE_ERR_INVALID_ARG;
-    return GQE_ERR_UNSUPPORTED;
-  }
-  if (!aligned16(Q) || !aligned16(Qs) || !aligned16(K) || !aligned16(V) ||
-      !aligned16(topk_idx) || !aligned16(w) || !aligned16(O_sel) || !aligned16(o_bar) ||
-      !aligned16(s_out))
+  const gqe_status st = gqe::check_dims(dims, false);  // the checks of gqe_attention_prefill
+  if (st != GQE_OK) return st;
+  if (!gqe::aligned16(Q) || !gqe::aligned16(Qs) || !gqe::aligned16(K) || !gqe::aligned16(V) ||
+      !gqe::aligned16(topk_idx) || !gqe::aligned16(w) || !gqe::aligned16(O_sel) ||
+      !gqe::aligned16(o_bar) || !gqe::aligned16(s_out))
     return GQE_ERR_INVALID_ARG;
   if (out_row_stride < dims->d || out_row_stride % 8 != 0) return GQE_ERR_INVALID_ARG;
   const StaticLayout L = static_layout(*dims);
@@ -140,8 +93,9 @@ extern "C" gqe_status gqe_attention_prefill_static(
   uint8_t* sb = nullptr;
   if (scratch_for_current_device(&sb) != cudaSuccess) return GQE_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the array keeps the previous call's contents: status and counters start at 0
-  if (cudaMemsetAsync(sb, 0, 512, s) != cudaSuccess) return GQE_ERR_CUDA;
+  // the array keeps the previous call's contents: the counters start at 0;
+  // the status word keeps latching until gqe_static_device_status clears it
+  if (cudaMemsetAsync(sb + L.counters, 0, 256, s) != cudaSuccess) return GQE_ERR_CUDA;
 
   const int64_t B = dims->B, S = dims->S, G = dims->G, d = dims->d;
   int* status = reinterpret_cast<int*>(sb + L.status);
@@ -170,13 +124,13 @@ extern "C" gqe_status gqe_attention_prefill_static(
 
   gqe::AttnArgs a;
   std::memset(&a, 0, sizeof(a));
-  if (!map_bshd(&a.tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, dims->B, dims->S, dims->G,
+  if (!gqe::map_bshd(&a.tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, dims->B, dims->S, dims->G,
                      dims->d) ||
-      !map_bshd(&a.tmV, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, sb + L.v16, dims->B, dims->S,
+      !gqe::map_bshd(&a.tmV, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, sb + L.v16, dims->B, dims->S,
                      dims->G, dims->d) ||
-      !map_bshd(&a.tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, dims->B, dims->S, dims->N,
+      !gqe::map_bshd(&a.tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, dims->B, dims->S, dims->N,
                      dims->d) ||
-      !map_bsd(&a.tmQs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Qs, dims->B, dims->S, dims->d))
+      !gqe::map_bsd(&a.tmQs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Qs, dims->B, dims->S, dims->d))
     return GQE_ERR_CUDA;
   a.Q = static_cast<const uint16_t*>(Q);
   a.bucket_off = ba.bucket_off;
@@ -201,11 +155,24 @@ extern "C" gqe_status gqe_attention_prefill_static(
   a.pair = pair ? 1 : 0;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   a.wait_limit_ns = gqe::kWaitLimitNs;
-  if (gqe::launch_attention(a, L.n_raw_tiles, s) != cudaSuccess) return GQE_ERR_CUDA;
+  if (gqe::timed_attention(a, L.n_raw_tiles, s) != cudaSuccess) return GQE_ERR_CUDA;
   if (dims->k > 1) {
     gqe::CombineArgs c{O_sel, o_bar, w, out_row_stride, dims->B * dims->S, dims->G, dims->k,
                        dims->d, dims->out_fp32};
     if (gqe::launch_combine(c, s) != cudaSuccess) return GQE_ERR_CUDA;
   }
   return GQE_OK;
+}
+
+extern "C" gqe_status gqe_static_device_status(int32_t clear, void* stream) {
+  uint8_t* sb = nullptr;
+  if (scratch_for_current_device(&sb) != cudaSuccess) return GQE_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GQE_ERR_CUDA;
+  int32_t code = 0;
+  if (cudaMemcpy(&code, sb, sizeof(code), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GQE_ERR_CUDA;
+  if (clear && cudaMemset(sb, 0, sizeof(int32_t)) != cudaSuccess) return GQE_ERR_CUDA;
+  if (code < GQE_OK || code > GQE_ERR_BAD_POSITION) return GQE_ERR_CUDA;
+  return static_cast<gqe_status>(code);
 }

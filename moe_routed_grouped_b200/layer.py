@@ -103,6 +103,30 @@ class GqePrefill:
         self.route(x, W_r, bias, stream)
         return self.attention(Q, Qs, K, V, stream)
 
+    def attention_static(self, Q, Qs, K, V, out=None, stream=None):
+        """The attention call without a workspace (gqe_attention_prefill_static:
+        its scratch is a fixed array inside the library).  Uses this object's
+        topk_idx and w; writes into ``out`` (a concat buffer shaped like
+        ``concat``) or into ``concat``."""
+        self._check_qkv(Q, K, V, Qs)
+        dv = self.device
+        _expect(self.topk_idx, "topk_idx", (self.B, self.S, self.G, self.k), torch.int32, dv)
+        _expect(self.w, "w", (self.B, self.S, self.G, self.k), torch.float32, dv)
+        if out is None:
+            out = self.concat
+        _expect(out, "out", (self.B * self.S, self.row), self.out_dtype, dv)
+        a = self.G * self.k * self.d
+        flat = out.view(-1)
+        _lib.gqe_attention_prefill_static(self.dims, Q, Qs, K, V, self.topk_idx, self.w, out,
+                                          flat[a:], flat[a + self.G * self.d:], self.row,
+                                          stream)
+        return out
+
+    @staticmethod
+    def static_device_status(clear=True, stream=None) -> int:
+        """Errors latched by attention_static calls on the current device."""
+        return _lib.gqe_static_device_status(1 if clear else 0, stream)
+
     def dense(self, Q, K, V, out=None, stream=None):
         self._check_qkv(Q, K, V)
         if out is not None:
