@@ -13,7 +13,8 @@ collective on the data path); ranks only meet for barriers and the max-over-
 ranks of the device time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                  [--sweep] [--impl ours|reference] [--no-cpu-baseline] [--decode]
+                  [--no-configs] [--impl ours|reference] [--no-cpu-baseline]
+                  [--no-decode] [--decode]
 """
 from __future__ import annotations
 
@@ -65,7 +66,7 @@ def load_peaks():
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML every ~2 ms."""
+    """Samples SM clock and clock-event reasons through NVML every ~0.5 ms."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -108,7 +109,7 @@ class ClockSampler:
                                      int(self._reasons())))
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.0005)
 
     def start(self):
         if self.ok:
@@ -411,13 +412,68 @@ def measure_workload(torch, w, device, rank, steps, warmup, flush, host_gen, wit
         L.dense(dev["Q"], dev["K"], dev["V"])
 
     r_ms, r_attn, t0, t1 = timed_loop(torch, routed, steps, warmup, flush, with_attn_events)
-    d_ms, d_attn, _, _ = timed_loop(torch, dense, steps, max(1, warmup // 2), flush,
-                                    with_attn_events)
+    d_ms, d_attn, d0, d1 = timed_loop(torch, dense, steps, warmup, flush, with_attn_events)
     status = L.device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after {w.name}")
     return dict(L=L, dev=dev, host=host, routed_ms=r_ms, routed_attn_ms=r_attn, dense_ms=d_ms,
-                dense_attn_ms=d_attn, t0=t0, t1=t1)
+                dense_attn_ms=d_attn, t0=t0, t1=t1, dense_t0=d0, dense_t1=d1)
+
+
+# the long-context workloads every default line also measures: (name, timed steps)
+CONFIG_ENTRIES = (("imbalanced32k", 10), ("wide131k", 5), ("million", 3))
+
+
+def config_entry(torch, name, steps, warmup, device, rank, local, flush, peaks, peak_src):
+    """Routed GQE and dense GQA on one long-context workload, each timed over
+    its own steps with its own clock record (NVML samples every ~0.5 ms, so the
+    1M-token steps of about 2 s are sampled inside every step).  Inputs come
+    from torch's generator on the device with the synth recipe's
+    distributions (parity runs on the synth bits in the tests)."""
+    ws = WORKLOADS[name]
+    cs = ClockSampler(local)
+    cs.start()
+    try:
+        r = measure_workload(torch, ws, device, rank, steps, warmup, flush, False, True)
+    finally:
+        cs.stop()
+    rm, dm = statistics.mean(r["routed_ms"]), statistics.mean(r["dense_ms"])
+    ra, da = statistics.mean(r["routed_attn_ms"]), statistics.mean(r["dense_attn_ms"])
+    fr, fd = ws.useful_flop_routed(), ws.useful_flop_dense()
+    attn_tf, dense_attn_tf = fr / (ra / 1e3) / 1e12, fd / (da / 1e3) / 1e12
+    e = {
+        "workload": name, "B": ws.B, "S": ws.S, "N": ws.N, "G": ws.G, "k": ws.k, "d": ws.d,
+        "d_model": ws.d_model, "router_bias_expert0": ws.bias0, "steps": steps,
+        "warmup": warmup,
+        "routed_ms": rm, "routed_ms_median": statistics.median(r["routed_ms"]),
+        "routed_ms_best": min(r["routed_ms"]),
+        "dense_ms": dm, "dense_ms_median": statistics.median(r["dense_ms"]),
+        "dense_ms_best": min(r["dense_ms"]),
+        "routed_tokens_per_s": ws.B * ws.S / (rm / 1e3),
+        "dense_tokens_per_s": ws.B * ws.S / (dm / 1e3),
+        "routed_useful_tflops": fr / (rm / 1e3) / 1e12,
+        "dense_useful_tflops": fd / (dm / 1e3) / 1e12,
+        "routed_over_dense": dm / rm,
+        "roofline": {"kernel": ("attn_pair_kernel" if ws.d == 64 and
+                                2 * ws.B * ws.S * ws.G * ws.d * 2 >= 96 << 20
+                                else "attn_kernel<%d>" % ws.d) + " (routed + shared head)",
+                     "bound": "tensor", "achieved": attn_tf, "unit": "TFLOP/s",
+                     "peak": peaks["bf16_tflops"], "frac": attn_tf / peaks["bf16_tflops"],
+                     "peak_sustained": peaks.get("bf16_tflops_sustained"),
+                     "frac_sustained": (attn_tf / peaks["bf16_tflops_sustained"]
+                                        if peaks.get("bf16_tflops_sustained") else None),
+                     "peak_source": f"{peak_src} bf16 dense (burst; sustained beside it)",
+                     "attention_kernel_ms": ra, "per_launch_flop": fr},
+        "dense_attention_kernel_ms": da, "dense_attention_kernel_tflops": dense_attn_tf,
+        "dense_attention_frac": dense_attn_tf / peaks["bf16_tflops"],
+        "clocks_routed": cs.summary(r["t0"], r["t1"]),
+        "clocks_dense": cs.summary(r["dense_t0"], r["dense_t1"]),
+        "inputs": "torch generator on the device, the synth recipe's distributions",
+        "gpu_launches": steps * (4 + (1 if ws.k > 1 else 0)) + steps * 2,
+    }
+    del r
+    torch.cuda.empty_cache()
+    return e
 
 
 def e2e_measure(torch, w, L, dev, steps):
@@ -490,8 +546,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="layer250m", choices=sorted(WORKLOADS))
-    ap.add_argument("--sweep", action="store_true",
-                    help="also time the S=32k, 131k and 1M workloads (routed and dense)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="leave the S=32k, 131k and 1M entries out of the line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="leave the decode-step measurements out of the prefill line")
@@ -597,32 +653,20 @@ def main():
         "clocks": clocks.summary(res["t0"], res["t1"]),
     }
 
-    if args.sweep:
+    if world == 1 and not args.no_configs:
+        # the S >= 32k workloads, each with its own timing and clock record
         del res
         torch.cuda.empty_cache()
-        sweep = []
-        for name in ("imbalanced32k", "wide131k", "million"):
-            ws = WORKLOADS[name]
-            k_steps = 3 if ws.S >= 1 << 20 else 5
-            r = measure_workload(torch, ws, device, rank, k_steps, 3, flush, False, True)
-            rm = sum(r["routed_ms"]) / k_steps
-            dm = sum(r["dense_ms"]) / k_steps
-            sweep.append({
-                "workload": name, "S": ws.S, "routed_ms": rm, "dense_ms": dm,
-                "routed_ms_median": statistics.median(r["routed_ms"]),
-                "routed_ms_best": min(r["routed_ms"]),
-                "dense_ms_median": statistics.median(r["dense_ms"]),
-                "dense_ms_best": min(r["dense_ms"]),
-                "routed_tokens_per_s": ws.B * ws.S / (rm / 1e3),
-                "routed_useful_tflops": ws.useful_flop_routed() / (rm / 1e3) / 1e12,
-                "dense_useful_tflops": ws.useful_flop_dense() / (dm / 1e3) / 1e12,
-                "routed_attention_kernel_tflops":
-                    ws.useful_flop_routed() / (statistics.mean(r["routed_attn_ms"]) / 1e3) / 1e12,
-                "routed_over_dense": dm / rm,
-                "inputs": "torch generator, same distributions as the synth recipe"})
-            del r
-            torch.cuda.empty_cache()
-        line["sweep"] = sweep
+        entries = []
+        for name, k_steps in CONFIG_ENTRIES:
+            try:
+                entries.append(config_entry(torch, name, k_steps, 3, device, rank, local, flush,
+                                            peaks, peak_src))
+            except Exception as ex:  # noqa: BLE001  (reported in the entry, not hidden)
+                entries.append({"workload": name, "error": f"{type(ex).__name__}: {ex}"[:300]})
+                torch.cuda.empty_cache()
+        line["configs"] = entries
+        line["gpu_launches"] += sum(e.get("gpu_launches", 0) for e in entries)
 
     if world == 1 and not args.no_decode:
         if "res" in locals():

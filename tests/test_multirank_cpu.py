@@ -153,3 +153,27 @@ def test_decode_entries_report_failures_in_place(monkeypatch):
     assert dec[0]["unit"] == "tokens/s" and dec[0]["steps"] == 5 and "clocks" in dec[0]
     assert dec[1] == {"workload": "layer250m",
                       "error": "RuntimeError: device status 8 in the decode loop"}
+
+
+def test_config_entry_numbers_from_fake_timings(monkeypatch):
+    """A long-context entry of the default line: tokens/s, useful TFLOP/s,
+    the routed/dense ratio and the attention roofline against both peaks come
+    from the measured times by the stated formulas; each arm carries its own
+    clock record."""
+    def fake(torch_, w, device, rank, steps, warmup, flush, host_gen, ev):
+        assert not host_gen and ev and warmup == 3
+        return dict(routed_ms=[2.0] * steps, dense_ms=[3.0] * steps,
+                    routed_attn_ms=[1.5] * steps, dense_attn_ms=[2.5] * steps,
+                    t0=0.0, t1=1.0, dense_t0=1.0, dense_t1=2.0)
+    monkeypatch.setattr(bench, "measure_workload", fake)
+    peaks = {"bf16_tflops": 1652.2, "bf16_tflops_sustained": 1379.2, "hbm_gbs": 6548.2}
+    e = bench.config_entry(torch, "imbalanced32k", 4, 3, torch.device("cpu"), 0, 0,
+                           lambda: None, peaks, "measured")
+    w = bench.WORKLOADS["imbalanced32k"]
+    assert e["routed_tokens_per_s"] == pytest.approx(w.S / 2e-3)
+    assert e["routed_over_dense"] == pytest.approx(1.5)
+    tf = w.useful_flop_routed() / 1.5e-3 / 1e12
+    assert e["roofline"]["achieved"] == pytest.approx(tf)
+    assert e["roofline"]["frac"] == pytest.approx(tf / 1652.2)
+    assert e["roofline"]["frac_sustained"] == pytest.approx(tf / 1379.2)
+    assert "clocks_routed" in e and "clocks_dense" in e
