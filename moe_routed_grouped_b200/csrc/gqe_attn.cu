@@ -54,6 +54,12 @@ constexpr int kThreads = 192;
 // FMA pipe; the rest use the MUFU ex2 unit (16 lanes/clock/SM), which would
 // otherwise bound d = 64 attention at about half the tensor-core rate.
 constexpr int kPolyPairs = 2;
+// The pair kernel runs the longest calls (K/V beyond L2, S around 1M), where
+// the GPU sits at its power limit and clocks down: there the polynomial's
+// extra instructions cost more than the MUFU time they save, and one pair in
+// 8 is the measured optimum (A/B at S = 1M: 0 / 1 / 2 / 3 pairs took
+// 1.92 / 1.87 / 2.01 / 2.16 s for the routed call).
+constexpr int kPairPolyPairs = 1;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 
@@ -80,6 +86,145 @@ struct Waiter {
     return mbar_wait(bar, parity, abort, status, limit);
   }
 };
+
+// ---------------------------------------------------------------------------
+// The online softmax of one KV tile for the thread's query row (TMEM lane).
+//
+// S_j (128 fp32 columns) is read from TMEM into registers and released at
+// once, so the MMA warp can start S_{j+1} = Q K_{j+1}^T while this tile is
+// exponentiated.  P_j = 2^(S_j * scale * log2(e) - m) replaces S_j in the
+// registers and is packed to fp16; it goes back to TMEM for the P.V product
+// only after all of its exponentials, so the wait for the previous tile's
+// P.V (which reads P from the same TMEM columns) comes that late.  m is the
+// running maximum in log2 units, moved only when a tile's maximum exceeds it
+// by more than 8 (so P <= 2^8 always fits fp16), which makes O rescales rare;
+// the final division by the row sum l makes the result exact whatever m was
+// used.
+constexpr float kRescaleThreshold = 8.f;
+
+__device__ __forceinline__ void tile_load_s(uint32_t taddr, uint32_t (&sv)[4][32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, sv[c]);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
+}
+
+// Key t is visible to a row at absolute position pos iff kvs <= t <= pos.
+__device__ __forceinline__ void tile_mask(uint32_t (&sv)[4][32], int kbase, int pos, int kvs) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int t = kbase + 32 * c + e;
+      if (t > pos || t < kvs) sv[c][e] = __float_as_uint(-INFINITY);
+    }
+}
+
+// Row maximum of the raw scores: 8 independent chains of 3-input max.
+__device__ __forceinline__ float tile_max(const uint32_t (&sv)[4][32]) {
+  float mxp[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) mxp[q] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int e = 0; e < 32; e += 2)
+      mxp[(e >> 1) & 7] = fmax3f(mxp[(e >> 1) & 7], __uint_as_float(sv[c][e]),
+                                 __uint_as_float(sv[c][e + 1]));
+  return fmax3f(fmax3f(mxp[0], mxp[1], mxp[2]), fmax3f(mxp[3], mxp[4], mxp[5]),
+                fmaxf(mxp[6], mxp[7]));
+}
+
+// p = 2^(s * sl2 - m), packed to fp16 pairs into pk; returns the sum of the p.
+// kPoly of every 8 column pairs go to the FMA-pipe polynomial.
+template <int kPoly>
+__device__ __forceinline__ float tile_exp(const uint32_t (&sv)[4][32], float sl2, float m,
+                                          uint32_t (&pk)[4][16]) {
+  const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m, -m);
+  uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const uint64_t y2 =
+          f2_fma(f2_pack(__uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1])), sl2x2, negm2);
+      float p0, p1;
+      if (((e >> 1) & 7) < kPoly) {  // this pair on the FMA pipe
+        exp2_poly_pair(y2, p0, p1);
+      } else {                             // this pair on the MUFU unit
+        float y0, y1;
+        f2_unpack(y2, y0, y1);
+        p0 = ex2_approx(y0);
+        p1 = ex2_approx(y1);
+      }
+      rs2[(e >> 1) & 3] = f2_add(rs2[(e >> 1) & 3], f2_pack(p0, p1));
+      pk[c][e / 2] = pack_half2(p0, p1);
+    }
+  }
+  float r0, r1, r2, r3, r4, r5, r6, r7;
+  f2_unpack(rs2[0], r0, r1);
+  f2_unpack(rs2[1], r2, r3);
+  f2_unpack(rs2[2], r4, r5);
+  f2_unpack(rs2[3], r6, r7);
+  return ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
+}
+
+// TMEM addresses and barriers of one 128-row tile's softmax.
+struct SoftmaxCtx {
+  uint32_t tS, tP, tO;  // this warp's lane quarter of S, P and O
+  uint64_t *s_full, *s_free, *o_done, *p_full;
+};
+
+// One KV tile j of a softmax warp; returns false when a wait gave up (the
+// lanes agree, as the tcgen05 instructions that follow are warp-collective).
+// A row that has seen no visible key yet (all padding) keeps m = -inf and
+// l = 0: its exponentials are taken against 0, which gives P = 0.
+template <int D, int kPoly>
+__device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& x, const Waiter& wait, int j,
+                                             bool diag, int kbase, int pos, int kvs, float sl2,
+                                             float& m_used, float& l) {
+  const int lane = threadIdx.x & 31;
+  if (!__all_sync(0xFFFFFFFFu, wait(x.s_full, j & 1))) return false;
+  tc_fence_after();
+  uint32_t sv[4][32];
+  tile_load_s(x.tS, sv);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(x.s_free);  // S_j is in registers: S_{j+1} may start
+  if (diag) tile_mask(sv, kbase, pos, kvs);
+  float factor = 1.f;
+  const float mnew = fmaxf(m_used, tile_max(sv) * sl2);  // j = 0: m_used = -inf, factor 0
+  if (mnew - m_used > kRescaleThreshold) {
+    factor = ex2_approx(m_used - mnew);
+    m_used = mnew;
+  }
+  // P in fp16: 64 registers, 64 TMEM columns for the 128 keys
+  uint32_t pk[4][16];
+  l = l * factor + tile_exp<kPoly>(sv, sl2, m_used == -INFINITY ? 0.f : m_used, pk);
+  // P.V of the previous tile must be done before P and O are touched
+  if (j > 0) {
+    if (!__all_sync(0xFFFFFFFFu, wait(x.o_done, (j - 1) & 1))) return false;
+    tc_fence_after();
+    if (__any_sync(0xFFFFFFFFu, factor != 1.f)) {  // rare: rescale O
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(x.tO + 32 * c, ov);
+        tmem_ld_wait(ov);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+        tmem_st32(x.tO + 32 * c, ov);
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_st16(x.tP + 16 * c, pk[c]);
+  tmem_st_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(x.p_full);
+  return true;
+}
 
 // One query row of a routed tile: row r of the token's Q head, copied with
 // cp.async into the 128-byte swizzle the UMMA descriptor expects (16-byte
@@ -210,6 +355,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
     nrows = td.nrows;
     nkv = td.nkv;
   }
+  // chunked prefill: absolute position of query row 0 and the first valid
+  // KV slot of this sequence (0, 0 without offsets); KV tiles are visited
+  // from the one that holds kv_start on
+  int qoff = 0, kvs = 0;
+  if (!a.dense) seq_offsets(a.q_off, a.kv_start, b, S, a.T, a.status, &qoff, &kvs);
+  const int j0 = kvs / kTileN;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + kNumBars);
@@ -270,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
 #pragma unroll
         for (int atom = 0; atom < D / 64; ++atom)
           tma_load_4d(smem + C::kSmemK + s * C::kKVBytes + atom * C::kAtom, &a.tmK,
-                      &bars[kBarKFull + s], atom * 64, g, j * kTileN, b);
+                      &bars[kBarKFull + s], atom * 64, g, (j0 + j) * kTileN, b);
         if (round > 0 && !wait(&bars[kBarVEmpty + s], (round - 1) & 1)) {
           issued = 2 * j + 1;
           break;
@@ -279,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
 #pragma unroll
         for (int atom = 0; atom < D / 64; ++atom)
           tma_load_4d(smem + C::kSmemV + s * C::kKVBytes + atom * C::kAtom, &a.tmV,
-                      &bars[kBarVFull + s], atom * 64, g, j * kTileN, b);
+                      &bars[kBarVFull + s], atom * 64, g, (j0 + j) * kTileN, b);
         issued = 2 * j + 2;
       }
       if (*abort_flag) {
@@ -354,102 +505,20 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
       pos = row0 + rv;
       pos_first = row0;
     }
+    const int apos = qoff + pos, apos_first = qoff + pos_first;  // absolute positions
     const float sl2 = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    const SoftmaxCtx sx{tbase + lane_off + C::kTmemS, tbase + lane_off + C::kTmemP,
+                        tbase + lane_off + C::kTmemO, &bars[kBarSFull], &bars[kBarSFree],
+                        &bars[kBarODone], &bars[kBarPFull]};
     for (int j = 0; j < nkv; ++j) {
-      // the lanes must agree: they go on to warp-collective tcgen05 instructions
-      if (!__all_sync(0xFFFFFFFFu, wait(&bars[kBarSFull], j & 1))) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sv[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tbase + lane_off + C::kTmemS + 32 * c, sv[c]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarSFree]);
-
-      const int kbase = j * kTileN;
-      if (kbase + kTileN - 1 > pos_first) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (kbase + 32 * c + e > pos) sv[c][e] = __float_as_uint(-INFINITY);
+      const int kbase = (j0 + j) * kTileN;
+      const bool diag = kbase + kTileN - 1 > apos_first || kbase < kvs;
+      if (!softmax_tile<D, kPolyPairs>(sx, wait, j, diag, kbase, apos, kvs, sl2, m_used, l)) {
+        ok = false;
+        break;
       }
-      // row max: 8 independent chains of 3-input max
-      float mxp[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) mxp[q] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          mxp[(e >> 1) & 7] = fmax3f(mxp[(e >> 1) & 7], __uint_as_float(sv[c][e]),
-                                     __uint_as_float(sv[c][e + 1]));
-      const float mx = fmax3f(fmax3f(mxp[0], mxp[1], mxp[2]), fmax3f(mxp[3], mxp[4], mxp[5]),
-                              fmaxf(mxp[6], mxp[7]));
-      const float mnew = fmaxf(m_used, mx * sl2);
-      float factor = 1.f;
-      if (mnew - m_used > 8.f) {
-        factor = ex2_approx(m_used - mnew);
-        m_used = mnew;
-      }
-      l *= factor;
-      // P.V of the previous tile must be done before P and O are touched
-      if (j > 0) {
-        if (!__all_sync(0xFFFFFFFFu, wait(&bars[kBarODone], (j - 1) & 1))) { ok = false; break; }
-        tc_fence_after();
-      }
-      // p = 2^(s * scale * log2e - m), packed to fp16 and written to TMEM
-      // 32 columns at a time
-      const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_used, -m_used);
-      uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const uint64_t y2 =
-              f2_fma(f2_pack(__uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1])), sl2x2,
-                     negm2);
-          float p0, p1;
-          if (((e >> 1) & 7) < kPolyPairs) {  // this pair on the FMA pipe
-            exp2_poly_pair(y2, p0, p1);
-          } else {                             // this pair on the MUFU unit
-            float y0, y1;
-            f2_unpack(y2, y0, y1);
-            p0 = ex2_approx(y0);
-            p1 = ex2_approx(y1);
-          }
-          rs2[(e >> 1) & 3] = f2_add(rs2[(e >> 1) & 3], f2_pack(p0, p1));
-          pk[e / 2] = pack_half2(p0, p1);
-        }
-        tmem_st16(tbase + lane_off + C::kTmemP + 16 * c, pk);
-      }
-      float r0, r1, r2, r3, r4, r5, r6, r7;
-      f2_unpack(rs2[0], r0, r1);
-      f2_unpack(rs2[1], r2, r3);
-      f2_unpack(rs2[2], r4, r5);
-      f2_unpack(rs2[3], r6, r7);
-      l += ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
-      // rescale O (rare: only when the running max grew by more than 2^8)
-      if (j > 0 && __any_sync(0xFFFFFFFFu, factor != 1.f)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(tbase + lane_off + C::kTmemO + 32 * c, ov);
-          tmem_ld_wait(ov);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
-          tmem_st32(tbase + lane_off + C::kTmemO + 32 * c, ov);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarPFull]);
     }
     if (ok) ok = wait(&bars[kBarODone], (nkv - 1) & 1);
     ok = __all_sync(0xFFFFFFFFu, ok);
@@ -479,7 +548,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
       tc_fence_after();
       // every product is done, so the K/V stages are free for the staging rows
       float* stage = reinterpret_cast<float*>(smem + C::kSmemK) + warp * 32 * (D + 4);
-      store_rows_coalesced<D>(stage, tbase + lane_off + C::kTmemO, 1.f / l, dst, dst2, fp32);
+      // a padding row (no visible key) has l = 0 and is written as zeros
+      store_rows_coalesced<D>(stage, tbase + lane_off + C::kTmemO, l > 0.f ? 1.f / l : 0.f, dst,
+                              dst2, fp32);
     }
   }
 
@@ -683,7 +754,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     // stage is released when both tiles are done with it; the shorter tile
     // releases the longer one's remaining stages as they arrive.
     const int s = warp - kPairMmaWarp;
-    const int nk = sl[s].nkv;
+    const int nk = s ? sl[1].nkv : sl[0].nkv;
     if (lane == 0) {
       const uint32_t tS = tbase + s * C::kTmemSlot + C::kTmemS;
       const uint32_t tP = tbase + s * C::kTmemSlot + C::kTmemP;
@@ -758,103 +829,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const float sl2 = a.scale_log2;
       float m_used = -INFINITY, l = 0.f;
       bool ok = true;
+      const SoftmaxCtx sx{tsl + C::kTmemS, tsl + C::kTmemP, tsl + C::kTmemO, &bars[kPbSFull + s],
+                          &bars[kPbSFree + s], &bars[kPbODone + s], &bars[kPbPFull + s]};
       for (int j = 0; j < t.nkv; ++j) {
-        // the lanes must agree: they go on to warp-collective tcgen05 instructions
-        if (!__all_sync(0xFFFFFFFFu, wait(&bars[kPbSFull + s], j & 1))) { ok = false; break; }
-        tc_fence_after();
-        uint32_t sv[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tsl + C::kTmemS + 32 * c, sv[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kPbSFree + s]);
-
         const int kbase = j * kTileN;
-        if (kbase + kTileN - 1 > pos_first) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (kbase + 32 * c + e > pos) sv[c][e] = __float_as_uint(-INFINITY);
-        }
-        float mxp[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mxp[q] = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; e += 2)
-            mxp[(e >> 1) & 7] = fmax3f(mxp[(e >> 1) & 7], __uint_as_float(sv[c][e]),
-                                       __uint_as_float(sv[c][e + 1]));
-        const float mx = fmax3f(fmax3f(mxp[0], mxp[1], mxp[2]), fmax3f(mxp[3], mxp[4], mxp[5]),
-                                fmaxf(mxp[6], mxp[7]));
-        const float mnew = fmaxf(m_used, mx * sl2);
-        float factor = 1.f;
-        if (mnew - m_used > 8.f) {
-          factor = ex2_approx(m_used - mnew);
-          m_used = mnew;
-        }
-        l *= factor;
-        // P.V of the previous tile must be done before P and O are touched
-        if (j > 0) {
-          if (!__all_sync(0xFFFFFFFFu, wait(&bars[kPbODone + s], (j - 1) & 1))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-        }
-        // the turn: tile 1 exponentiates its j-th KV tile after tile 0 has,
-        // and tile 0 its j-th after tile 1 its (j-1)-th (while tile 1 has one)
-
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_used, -m_used);
-        uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const uint64_t y2 =
-                f2_fma(f2_pack(__uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1])), sl2x2,
-                       negm2);
-            float p0, p1;
-            if (((e >> 1) & 7) < kPolyPairs) {
-              exp2_poly_pair(y2, p0, p1);
-            } else {
-              float y0, y1;
-              f2_unpack(y2, y0, y1);
-              p0 = ex2_approx(y0);
-              p1 = ex2_approx(y1);
-            }
-            rs2[(e >> 1) & 3] = f2_add(rs2[(e >> 1) & 3], f2_pack(p0, p1));
-            pk[e / 2] = pack_half2(p0, p1);
-          }
-          tmem_st16(tsl + C::kTmemP + 16 * c, pk);
-        }
-        float r0, r1, r2, r3, r4, r5, r6, r7;
-        f2_unpack(rs2[0], r0, r1);
-        f2_unpack(rs2[1], r2, r3);
-        f2_unpack(rs2[2], r4, r5);
-        f2_unpack(rs2[3], r6, r7);
-        l += ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
-        if (j > 0 && __any_sync(0xFFFFFFFFu, factor != 1.f)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(tsl + C::kTmemO + 32 * c, ov);
-            tmem_ld_wait(ov);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
-            tmem_st32(tsl + C::kTmemO + 32 * c, ov);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bars[kPbPFull + s]);
-
+        if (!softmax_tile<D, kPairPolyPairs>(sx, wait, j, kbase + kTileN - 1 > pos_first, kbase,
+                                             pos, 0, sl2, m_used, l)) {
+          ok = false;
+          break;
         }
       }
       ok = __all_sync(0xFFFFFFFFu, ok && wait(&bars[kPbODone + s], (t.nkv - 1) & 1));
@@ -882,7 +864,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tc_fence_after();
         // K/V stages may still feed the other tile: stage in this warp's own region
         float* stage = reinterpret_cast<float*>(smem + C::kSmemStage) + warp * 32 * (D + 4);
-        store_rows_coalesced<D>(stage, tsl + C::kTmemO, 1.f / l, dst, dst2, fp32);
+        store_rows_coalesced<D>(stage, tsl + C::kTmemO, l > 0.f ? 1.f / l : 0.f, dst, dst2,
+                                fp32);
       }
     }
   }

@@ -125,8 +125,10 @@ def test_static_entry_with_pair_kernel(pair_kernel):
 
 @pytest.mark.parametrize("name", ["layer250m", "imbalanced32k"])
 def test_pair_kernel_equals_one_tile_kernel(name):
-    """Same bits from both kernels on a full-size workload; dense calls keep
-    the one-tile kernel whatever the threshold."""
+    """Both kernels agree on a full-size workload (the pair kernel sends 1 of
+    8 exponential pairs to the FMA polynomial, the one-tile kernel 2, so the
+    bits differ within the polynomial's 7.5e-5 relative error); dense calls
+    keep the one-tile kernel whatever the threshold (same bits)."""
     w = WORKLOADS[name]
     inp = make_inputs(w)
     dev = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).view(torch.bfloat16).cuda()
@@ -144,7 +146,8 @@ def test_pair_kernel_equals_one_tile_kernel(name):
             outs.append((L.concat.clone(), O.clone()))
         finally:
             gqe.gqe_set_pair_threshold(prev)
-    assert torch.equal(outs[0][0], outs[1][0]), "routed concat buffer differs"
+    check_close(outs[1][0].cpu().numpy(), outs[0][0].cpu().numpy(), "pair vs one-tile",
+                atol=1e-3, rtol_l2=1e-4)
     assert torch.equal(outs[0][1], outs[1][1]), "dense output differs"
 
 
