@@ -179,6 +179,37 @@ gqe_status gqe_attention_prefill_static(const gqe_dims* dims, const void* Q, con
  */
 gqe_status gqe_static_device_status(int32_t clear, void* stream);
 
+/* Bytes of workspace gqe_attention_prefill_chunk needs for `dims` (S = the
+ * chunk's query count) over caches of T >= S slots (0 if invalid). */
+size_t gqe_prefill_chunk_workspace_size(const gqe_dims* dims, int32_t T);
+
+/*
+ * gqe_attention_prefill_chunk - gqe_attention_prefill for a chunk of S new
+ * tokens per sequence over KV caches of T slots (chunked prefill), with
+ * optional left padding.  "AI 大模型之 GQA", 工程实操 非方形因果遮罩: Sq
+ * queries at the end of Sk keys, the mask taken on absolute positions; step
+ * 4: the causal condition intersected with key validity.  Query row i of
+ * sequence b sits at absolute position q_off[b] + i and sees cache slots
+ * kv_start[b]..q_off[b] + i (the chunk's own K/V must already be in the
+ * caches).  Rows whose position lies before kv_start[b] are padding: they
+ * see no key and their outputs are written as zeros.
+ *  Q, Qs    device bf16 [B, S, N, d], [B, S, d]   (the chunk's queries)
+ *  Kc, Vc   device bf16 [B, T, G, d]
+ *  q_off    device int32 [B] or NULL (= 0): 0 <= q_off[b] <= T - S
+ *  kv_start device int32 [B] or NULL (= 0): 0 <= kv_start[b] < T
+ *  topk_idx, w, outputs, out_row_stride as for gqe_attention_prefill (one
+ *  output row per chunk token); ws of gqe_prefill_chunk_workspace_size bytes.
+ * Positions are read on the device (so a chunk loop can be captured in a CUDA
+ * graph); a value outside its range latches GQE_ERR_BAD_POSITION and is
+ * taken as 0.  Always runs the one-tile attention kernel.
+ */
+gqe_status gqe_attention_prefill_chunk(const gqe_dims* dims, int32_t T, const void* Q,
+                                       const void* Qs, const void* Kc, const void* Vc,
+                                       const int32_t* q_off, const int32_t* kv_start,
+                                       const int32_t* topk_idx, const float* w, void* O_sel,
+                                       void* o_bar, void* s_out, int64_t out_row_stride,
+                                       void* ws, size_t ws_bytes, void* stream);
+
 /*
  * gqe_dense_gqa_prefill - the all-active GQA baseline ("16 heads all
  * active", review §四): every query head h attends KV head floor(h/M).
@@ -299,6 +330,76 @@ void gqe_set_profile_events(void* begin, void* end);
  * Results agree within rounding either way.  Process-wide setting, read at
  * each call; returns the previous value. */
 int64_t gqe_set_pair_threshold(int64_t kv_bytes);
+
+/* ------------------------------------------------------------------------
+ * The attention layer around the path: projections and W_O.
+ * Review §二 路由器: only the query heads the router selected are computed at
+ * all, so their query projection runs for the selected (token, head) pairs
+ * only; 三个关键部件: y_i = Concat(O_i, o_bar_i, s(x_i)) W_O.  The other
+ * projections are plain linear maps (K_{i,g} = x_i W_K[g], V likewise, the
+ * shared head's query x_i W_s).  All run on the tensor cores with bf16
+ * operands and float32 accumulation.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * gqe_linear - C[r, n] = sum_k A[r, k] * W[n / nc][k, n % nc] for r < rows,
+ * n < nb*nc: A times a stack of nb matrices [K, nc] read as one [K, nb*nc]
+ * operand, so x . W_K for all G KV heads is one call whose output is K in its
+ * [B, S, G, d] layout (rows = B*S, nb = G, nc = d, ldc = G*d).
+ *  A   device bf16, rows x K at row stride lda elements (lda >= K, lda % 8 == 0)
+ *  W   device bf16 [nb, K, nc] (row-major)
+ *  C   device, rows x nb*nc at row stride ldc elements; float32 if c_fp32
+ *      else bf16 (round to nearest even); ldc*element size a multiple of 16 B
+ * K and nc must be multiples of 64 (GQE_ERR_UNSUPPORTED otherwise).
+ */
+gqe_status gqe_linear(int32_t rows, int32_t K, int32_t nb, int32_t nc, const void* A, int64_t lda,
+                      const void* W, void* C, int64_t ldc, int32_t c_fp32, void* stream);
+
+/*
+ * gqe_routed_q_project - the query projection of the selected heads only:
+ * Q[b, i, h, :] = x[b, i, :] . W_Q[h] for every (b, i, g, j) with
+ * h = g*M + topk_idx[b, i, g, j].  Rows of heads a token did not select are
+ * not written.  Each CTA takes one tile of a (batch, group, expert) bucket
+ * (the lists gqe_attention_prefill builds), gathers its x rows and multiplies
+ * them by that expert's W_Q[h].
+ *  x        device bf16 [B, S, d_model] (d_model % 64 == 0)
+ *  W_Q      device bf16 [N, d_model, d]
+ *  topk_idx device int32 [B, S, G, k]
+ *  Q        device bf16 [B, S, N, d]
+ *  ws       workspace of gqe_workspace_size(dims) bytes
+ */
+gqe_status gqe_routed_q_project(const gqe_dims* dims, const void* x, const void* W_Q,
+                                const int32_t* topk_idx, void* Q, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/*
+ * gqe_layer_prefill - the whole GQE attention layer, causal prefill, x -> y:
+ * gqe_route, then K, V and Qs by gqe_linear, Q of the selected heads by
+ * gqe_routed_q_project, gqe_attention_prefill into a bf16 concat buffer
+ * (whatever dims->out_fp32 says: the buffer feeds W_O in bf16), then
+ * y = concat . W_O by gqe_linear.  The caller owns every buffer:
+ *  W_K, W_V  device bf16 [G, d_model, d];  W_s bf16 [d_model, d]
+ *  W_r, bias as for gqe_route;  W_O bf16 [(G*k + G + 1)*d, d_model], rows
+ *            in concat order
+ *  topk_idx, p, w as for gqe_route;  Q bf16 [B, S, N, d] (selected rows);
+ *  Qs bf16 [B, S, d];  K, V bf16 [B, S, G, d];
+ *  concat    bf16 [B*S, (G*k + G + 1)*d];  y float32 [B, S, d_model]
+ */
+gqe_status gqe_layer_prefill(const gqe_dims* dims, const void* x, const void* W_Q,
+                             const void* W_K, const void* W_V, const void* W_s, const void* W_r,
+                             const float* bias, const void* W_O, int32_t* topk_idx, float* p,
+                             float* w, void* Q, void* Qs, void* K, void* V, void* concat,
+                             float* y, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * gqe_dense_layer_prefill - the all-active GQA layer baseline (review §四):
+ * Q of all N heads, K, V, dense GQA attention into O bf16 [B, S, N, d], then
+ * y = O . W_O with W_O bf16 [N*d, d_model].
+ */
+gqe_status gqe_dense_layer_prefill(const gqe_dims* dims, const void* x, const void* W_Q,
+                                   const void* W_K, const void* W_V, const void* W_O, void* Q,
+                                   void* K, void* V, void* O, float* y, void* ws,
+                                   size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

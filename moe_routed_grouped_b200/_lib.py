@@ -19,7 +19,8 @@ EXPORTS = (
     "gqe_status_string", "gqe_selftest_bounded_wait", "gqe_set_profile_events",
     "gqe_attention_prefill_static", "gqe_set_pair_threshold", "gqe_decode_workspace_size",
     "gqe_attention_decode", "gqe_append_workspace_size", "gqe_attention_append",
-    "gqe_static_device_status",
+    "gqe_static_device_status", "gqe_linear", "gqe_routed_q_project", "gqe_layer_prefill",
+    "gqe_dense_layer_prefill", "gqe_prefill_chunk_workspace_size", "gqe_attention_prefill_chunk",
 )
 
 STATUS = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED", 3: "GQE_ERR_CUDA",
@@ -62,6 +63,12 @@ def _load() -> ctypes.CDLL:
         "gqe_append_workspace_size": (SZ, [S, I32]),
         "gqe_attention_append": (I32, [S, I32, P, P, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
         "gqe_static_device_status": (I32, [I32, P]),
+        "gqe_linear": (I32, [I32, I32, I32, I32, P, I64, P, P, I64, I32, P]),
+        "gqe_routed_q_project": (I32, [S, P, P, P, P, P, SZ, P]),
+        "gqe_layer_prefill": (I32, [S] + [P] * 18 + [SZ, P]),
+        "gqe_dense_layer_prefill": (I32, [S] + [P] * 11 + [SZ, P]),
+        "gqe_prefill_chunk_workspace_size": (SZ, [S, I32]),
+        "gqe_attention_prefill_chunk": (I32, [S, I32] + [P] * 11 + [I64, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -171,6 +178,50 @@ def gqe_attention_prefill_static(dm, Q, Qs, K, V, topk_idx, w, O_sel, o_bar, s_o
 def gqe_static_device_status(clear=1, stream=None) -> int:
     """Status word of gqe_attention_prefill_static on the current device."""
     return LIB.gqe_static_device_status(int(clear), _stream(stream))
+
+
+def gqe_prefill_chunk_workspace_size(dm: GqeDims, T: int) -> int:
+    return LIB.gqe_prefill_chunk_workspace_size(ctypes.byref(dm), int(T))
+
+
+def gqe_attention_prefill_chunk(dm, T, Q, Qs, Kc, Vc, q_off, kv_start, topk_idx, w, O_sel, o_bar,
+                                s_out, out_row_stride, ws, stream=None, check=True):
+    """A chunk of dm.S queries per sequence at q_off[b] + i over caches of T
+    slots; q_off / kv_start: device int32 [B] or None."""
+    r = LIB.gqe_attention_prefill_chunk(
+        ctypes.byref(dm), int(T), _ptr(Q), _ptr(Qs), _ptr(Kc), _ptr(Vc), _ptr(q_off),
+        _ptr(kv_start), _ptr(topk_idx), _ptr(w), _ptr(O_sel), _ptr(o_bar), _ptr(s_out),
+        int(out_row_stride), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_attention_prefill_chunk") if check else r
+
+
+def gqe_linear(rows, K, nb, nc, A, lda, W, C, ldc, c_fp32, stream=None, check=True):
+    """C[rows, nb*nc] = A[rows, :K] . W[nb, K, nc] (stacked along the columns)."""
+    r = LIB.gqe_linear(int(rows), int(K), int(nb), int(nc), _ptr(A), int(lda), _ptr(W), _ptr(C),
+                       int(ldc), int(c_fp32), _stream(stream))
+    return _check(r, "gqe_linear") if check else r
+
+
+def gqe_routed_q_project(dm, x, W_Q, topk_idx, Q, ws, stream=None, check=True):
+    r = LIB.gqe_routed_q_project(ctypes.byref(dm), _ptr(x), _ptr(W_Q), _ptr(topk_idx), _ptr(Q),
+                                 _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_routed_q_project") if check else r
+
+
+def gqe_layer_prefill(dm, x, W_Q, W_K, W_V, W_s, W_r, bias, W_O, topk_idx, p, w, Q, Qs, K, V,
+                      concat, y, ws, stream=None, check=True):
+    r = LIB.gqe_layer_prefill(ctypes.byref(dm), *[_ptr(t) for t in (
+        x, W_Q, W_K, W_V, W_s, W_r, bias, W_O, topk_idx, p, w, Q, Qs, K, V, concat, y, ws)],
+        ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_layer_prefill") if check else r
+
+
+def gqe_dense_layer_prefill(dm, x, W_Q, W_K, W_V, W_O, Q, K, V, O, y, ws, stream=None,
+                            check=True):
+    r = LIB.gqe_dense_layer_prefill(ctypes.byref(dm), *[_ptr(t) for t in (
+        x, W_Q, W_K, W_V, W_O, Q, K, V, O, y, ws)], ws.numel() * ws.element_size(),
+        _stream(stream))
+    return _check(r, "gqe_dense_layer_prefill") if check else r
 
 
 def gqe_decode_workspace_size(dm: GqeDims) -> int:

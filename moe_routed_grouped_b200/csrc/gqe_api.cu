@@ -75,6 +75,7 @@ static BucketArgs bucket_args(const gqe_dims* dims, const int32_t* topk_idx, int
   a.k = dims->k;
   a.cap_bg = L.cap_bg;
   a.n_raw_tiles = L.n_raw_tiles;
+  a.T = dims->S;
   return a;
 }
 
@@ -103,42 +104,60 @@ static AttnArgs attn_common(const gqe_dims* dims, uint8_t* wb, const WsLayout& L
   a.k = dims->k;
   a.d = dims->d;
   a.out_fp32 = dims->out_fp32;
+  a.T = dims->S;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dims->d)));
   a.wait_limit_ns = kWaitLimitNs;
   return a;
 }
 
-gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void* Qs,
-                                 const void* K, const void* V, const int32_t* topk_idx,
-                                 const float* w, void* O_sel, void* o_bar, void* s_out,
-                                 int64_t out_row_stride, void* ws, size_t ws_bytes,
-                                 void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The routed prefill over a KV sequence of T slots (T = S and null offsets:
+// plain prefill; otherwise a chunk of S queries at absolute positions
+// q_off[b] + i over a cache, with the first valid slot kv_start[b]).
+gqe_status attention_prefill_impl(const gqe_dims* dims, int32_t T, const void* Q, const void* Qs,
+                                  const void* K, const void* V, const int32_t* q_off,
+                                  const int32_t* kv_start, const int32_t* topk_idx,
+                                  const float* w, void* O_sel, void* o_bar, void* s_out,
+                                  int64_t out_row_stride, void* ws, size_t ws_bytes,
+                                  void* stream) {
   gqe_status st = check_dims(dims, false);
   if (st != GQE_OK) return st;
+  if (T < dims->S) return GQE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(dims->B) * T * dims->G * dims->d >= (int64_t(1) << 40) ||
+      (static_cast<int64_t>(T) / kTileN + 3) * 4 > 200 * 1024)
+    return GQE_ERR_UNSUPPORTED;
   if (!aligned16(Q) || !aligned16(Qs) || !aligned16(K) || !aligned16(V) ||
       !aligned16(topk_idx) || !aligned16(w) || !aligned16(O_sel) || !aligned16(o_bar) ||
-      !aligned16(s_out))
+      !aligned16(s_out) || (q_off && !aligned16(q_off)) || (kv_start && !aligned16(kv_start)))
     return GQE_ERR_INVALID_ARG;
   if (out_row_stride < dims->d || out_row_stride % 8 != 0) return GQE_ERR_INVALID_ARG;
-  const WsLayout L = make_ws_layout(*dims);
+  const WsLayout L = make_ws_layout(*dims, T);
   if (!aligned16(ws) || ws_bytes < L.total) return GQE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* wb = static_cast<uint8_t*>(ws);
-  const int64_t B = dims->B, S = dims->S, G = dims->G, d = dims->d;
+  const int64_t B = dims->B, G = dims->G, d = dims->d;
+  const bool chunked = q_off || kv_start || T != dims->S;
 
   ConvertArgs cv{static_cast<const uint16_t*>(V), reinterpret_cast<uint16_t*>(wb + L.v16),
-                 B * S * G * d, reinterpret_cast<int*>(wb + L.status)};
+                 B * T * G * d, reinterpret_cast<int*>(wb + L.status)};
   // one decision for the call: the work-list format and the kernel follow it
-  const bool pair = pair_kernel_for(*dims);
+  // (chunked calls always take the one-tile kernel)
+  const bool pair = !chunked && pair_kernel_for(*dims);
   BucketArgs ba = bucket_args(dims, topk_idx, reinterpret_cast<int32_t*>(wb + L.bucket_off),
                               reinterpret_cast<int32_t*>(wb + L.bucket_tok), wb, L);
   ba.pairs = pair ? 1 : 0;
+  ba.q_off = q_off;
+  ba.kv_start = kv_start;
+  ba.T = T;
   cudaError_t e = launch_prep(ba, &cv, true, s);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
 
   AttnArgs a = attn_common(dims, wb, L);
-  if (!map_bshd(&a.tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, dims->B, dims->S, dims->G, dims->d) ||
-      !map_bshd(&a.tmV, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wb + L.v16, dims->B, dims->S, dims->G,
+  if (!map_bshd(&a.tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, dims->B, T, dims->G, dims->d) ||
+      !map_bshd(&a.tmV, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wb + L.v16, dims->B, T, dims->G,
                 dims->d) ||
       !map_bshd(&a.tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, dims->B, dims->S, dims->N, dims->d) ||
       !map_bsd(&a.tmQs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Qs, dims->B, dims->S, dims->d))
@@ -153,6 +172,9 @@ gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void
   a.o_bar = o_bar;
   a.s_out = s_out;
   a.out_row_stride = out_row_stride;
+  a.q_off = q_off;
+  a.kv_start = kv_start;
+  a.T = T;
   a.dense = 0;
   a.pair = pair ? 1 : 0;
   e = timed_attention(a, L.n_raw_tiles, s);
@@ -165,6 +187,36 @@ gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void
     if (e != cudaSuccess) return GQE_ERR_CUDA;
   }
   return GQE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void* Qs,
+                                 const void* K, const void* V, const int32_t* topk_idx,
+                                 const float* w, void* O_sel, void* o_bar, void* s_out,
+                                 int64_t out_row_stride, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (!dims) return GQE_ERR_INVALID_ARG;
+  return attention_prefill_impl(dims, dims->S, Q, Qs, K, V, nullptr, nullptr, topk_idx, w, O_sel,
+                                o_bar, s_out, out_row_stride, ws, ws_bytes, stream);
+}
+
+size_t gqe_prefill_chunk_workspace_size(const gqe_dims* dims, int32_t T) {
+  if (check_dims(dims, false) != GQE_OK || T < dims->S) return 0;
+  return make_ws_layout(*dims, T).total;
+}
+
+gqe_status gqe_attention_prefill_chunk(const gqe_dims* dims, int32_t T, const void* Q,
+                                       const void* Qs, const void* Kc, const void* Vc,
+                                       const int32_t* q_off, const int32_t* kv_start,
+                                       const int32_t* topk_idx, const float* w, void* O_sel,
+                                       void* o_bar, void* s_out, int64_t out_row_stride,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  if (!dims) return GQE_ERR_INVALID_ARG;
+  return attention_prefill_impl(dims, T, Q, Qs, Kc, Vc, q_off, kv_start, topk_idx, w, O_sel,
+                                o_bar, s_out, out_row_stride, ws, ws_bytes, stream);
 }
 
 gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void* K,
@@ -196,6 +248,145 @@ gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void
 }
 
 int64_t gqe_set_pair_threshold(int64_t kv_bytes) { return set_pair_threshold(kv_bytes); }
+
+// ------------------------------------------------------------ projections
+
+gqe_status gqe_linear(int32_t rows, int32_t K, int32_t nb, int32_t nc, const void* A, int64_t lda,
+                      const void* W, void* C, int64_t ldc, int32_t c_fp32, void* stream) {
+  if (rows < 1 || K < 64 || K % 64 != 0 || nb < 1 || nc < 64 || nc % 64 != 0)
+    return GQE_ERR_UNSUPPORTED;
+  if (c_fp32 != 0 && c_fp32 != 1) return GQE_ERR_INVALID_ARG;
+  const int64_t n_total = static_cast<int64_t>(nb) * nc;
+  if (lda < K || lda % 8 != 0 || ldc < n_total || ldc % (c_fp32 ? 4 : 8) != 0)
+    return GQE_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(W) || !aligned16(C)) return GQE_ERR_INVALID_ARG;
+  if (n_total > (int64_t(1) << 30) || static_cast<int64_t>(rows) * ldc >= (int64_t(1) << 40))
+    return GQE_ERR_UNSUPPORTED;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  const uint64_t adims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows)};
+  const uint64_t astr[1] = {static_cast<uint64_t>(lda) * 2};
+  const uint32_t abox[2] = {64, static_cast<uint32_t>(kTileM)};
+  const uint64_t bdims[3] = {static_cast<uint64_t>(nc), static_cast<uint64_t>(K),
+                             static_cast<uint64_t>(nb)};
+  const uint64_t bstr[2] = {static_cast<uint64_t>(nc) * 2, static_cast<uint64_t>(K) * nc * 2};
+  const uint32_t bbox[3] = {64, 64, 1};
+  if (!encode_map(&g.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, adims, astr, abox) ||
+      !encode_map(&g.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, W, bdims, bstr, bbox))
+    return GQE_ERR_CUDA;
+  g.C = C;
+  g.ldc = ldc;
+  g.c_fp32 = c_fp32;
+  g.K = K;
+  g.nc = nc;
+  g.n_total = static_cast<int>(n_total);
+  g.rows = rows;
+  g.wait_limit_ns = kWaitLimitNs;
+  g.status = nullptr;
+  // column tile: 256 when that still gives two tiles per SM, else 128 or 64
+  const int64_t mt = (rows + kTileM - 1) / kTileM;
+  int bn = 64;
+  if (n_total % 256 == 0 && mt * (n_total / 256) >= 296) bn = 256;
+  else if (n_total % 128 == 0) bn = 128;
+  return from_cuda(launch_gemm_dense(g, bn, static_cast<cudaStream_t>(stream)));
+}
+
+gqe_status gqe_routed_q_project(const gqe_dims* dims, const void* x, const void* W_Q,
+                                const int32_t* topk_idx, void* Q, void* ws, size_t ws_bytes,
+                                void* stream) {
+  gqe_status st = check_dims(dims, false);
+  if (st != GQE_OK) return st;
+  if (dims->d_model < 64 || dims->d_model % 64 != 0) return GQE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(W_Q) || !aligned16(topk_idx) || !aligned16(Q))
+    return GQE_ERR_INVALID_ARG;
+  const WsLayout L = make_ws_layout(*dims);
+  if (!aligned16(ws) || ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  // the bucket lists and the work list the attention call builds too
+  BucketArgs ba = bucket_args(dims, topk_idx, reinterpret_cast<int32_t*>(wb + L.bucket_off),
+                              reinterpret_cast<int32_t*>(wb + L.bucket_tok), wb, L);
+  ba.pairs = 0;
+  if (launch_prep(ba, nullptr, true, s) != cudaSuccess) return GQE_ERR_CUDA;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  const uint64_t bdims[3] = {static_cast<uint64_t>(dims->d), static_cast<uint64_t>(dims->d_model),
+                             static_cast<uint64_t>(dims->N)};
+  const uint64_t bstr[2] = {static_cast<uint64_t>(dims->d) * 2,
+                            static_cast<uint64_t>(dims->d_model) * dims->d * 2};
+  const uint32_t bbox[3] = {64, 64, 1};
+  if (!encode_map(&g.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, W_Q, bdims, bstr, bbox))
+    return GQE_ERR_CUDA;
+  g.A = static_cast<const uint16_t*>(x);
+  g.lda = dims->d_model;
+  g.C = Q;
+  g.K = dims->d_model;
+  g.nc = dims->d;
+  g.bucket_off = reinterpret_cast<const int32_t*>(wb + L.bucket_off);
+  g.bucket_tok = reinterpret_cast<const int32_t*>(wb + L.bucket_tok);
+  g.tiles = reinterpret_cast<const TileDesc*>(wb + L.tiles);
+  g.tile_count = reinterpret_cast<const int32_t*>(wb + L.counters) + 1;
+  g.B = dims->B;
+  g.S = dims->S;
+  g.N = dims->N;
+  g.G = dims->G;
+  g.M = dims->N / dims->G;
+  g.d = dims->d;
+  g.status = reinterpret_cast<int*>(wb + L.status);
+  g.wait_limit_ns = kWaitLimitNs;
+  return from_cuda(launch_gemm_routed(g, L.n_raw_tiles, s));
+}
+
+gqe_status gqe_layer_prefill(const gqe_dims* dims, const void* x, const void* W_Q,
+                             const void* W_K, const void* W_V, const void* W_s, const void* W_r,
+                             const float* bias, const void* W_O, int32_t* topk_idx, float* p,
+                             float* w, void* Q, void* Qs, void* K, void* V, void* concat,
+                             float* y, void* ws, size_t ws_bytes, void* stream) {
+  gqe_status st = check_dims(dims, true);
+  if (st != GQE_OK) return st;
+  if (dims->d_model % 64 != 0) return GQE_ERR_UNSUPPORTED;
+  gqe_dims db = *dims;
+  db.out_fp32 = 0;  // the concat buffer feeds W_O as bf16
+  const int32_t T = dims->B * dims->S, dm = dims->d_model, d = dims->d, G = dims->G;
+  const int64_t row = static_cast<int64_t>(G * dims->k + G + 1) * d;
+  if (!aligned16(concat) || !aligned16(y)) return GQE_ERR_INVALID_ARG;
+  if ((st = gqe_route(&db, x, W_r, bias, topk_idx, p, w, ws, ws_bytes, stream)) != GQE_OK)
+    return st;
+  if ((st = gqe_linear(T, dm, G, d, x, dm, W_K, K, int64_t(G) * d, 0, stream)) != GQE_OK)
+    return st;
+  if ((st = gqe_linear(T, dm, G, d, x, dm, W_V, V, int64_t(G) * d, 0, stream)) != GQE_OK)
+    return st;
+  if ((st = gqe_linear(T, dm, 1, d, x, dm, W_s, Qs, d, 0, stream)) != GQE_OK) return st;
+  if ((st = gqe_routed_q_project(&db, x, W_Q, topk_idx, Q, ws, ws_bytes, stream)) != GQE_OK)
+    return st;
+  uint16_t* cb = static_cast<uint16_t*>(concat);
+  const int64_t a = int64_t(G) * dims->k * d;
+  if ((st = gqe_attention_prefill(&db, Q, Qs, K, V, topk_idx, w, cb, cb + a, cb + a + G * d, row,
+                                  ws, ws_bytes, stream)) != GQE_OK)
+    return st;
+  return gqe_linear(T, static_cast<int32_t>(row), 1, dm, concat, row, W_O, y, dm, 1, stream);
+}
+
+gqe_status gqe_dense_layer_prefill(const gqe_dims* dims, const void* x, const void* W_Q,
+                                   const void* W_K, const void* W_V, const void* W_O, void* Q,
+                                   void* K, void* V, void* O, float* y, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  gqe_status st = check_dims(dims, false);
+  if (st != GQE_OK) return st;
+  if (dims->d_model < 64 || dims->d_model % 64 != 0) return GQE_ERR_UNSUPPORTED;
+  gqe_dims db = *dims;
+  db.out_fp32 = 0;  // O feeds W_O as bf16
+  const int32_t T = dims->B * dims->S, dm = dims->d_model, d = dims->d, G = dims->G,
+                N = dims->N;
+  if ((st = gqe_linear(T, dm, N, d, x, dm, W_Q, Q, int64_t(N) * d, 0, stream)) != GQE_OK)
+    return st;
+  if ((st = gqe_linear(T, dm, G, d, x, dm, W_K, K, int64_t(G) * d, 0, stream)) != GQE_OK)
+    return st;
+  if ((st = gqe_linear(T, dm, G, d, x, dm, W_V, V, int64_t(G) * d, 0, stream)) != GQE_OK)
+    return st;
+  if ((st = gqe_dense_gqa_prefill(&db, Q, K, V, O, ws, ws_bytes, stream)) != GQE_OK) return st;
+  return gqe_linear(T, N * d, 1, dm, O, int64_t(N) * d, W_O, y, dm, 1, stream);
+}
 
 size_t gqe_decode_workspace_size(const gqe_dims* dims) {
   if (check_dims(dims, false) != GQE_OK) return 0;

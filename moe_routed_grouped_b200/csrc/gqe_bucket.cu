@@ -102,6 +102,9 @@ __device__ void bucket_body(const BucketArgs& a, int bg) {
 
   // routed work items: ceil(cnt/128) tiles per expert; unused slots get nkv 0
   TileDesc* slots = a.tiles_raw + static_cast<int64_t>(bg) * a.cap_bg;
+  int qo, kvs;
+  seq_offsets(a.q_off, a.kv_start, b, S, a.T, a.status, &qo, &kvs);
+  const int j0 = kvs / kTileN;
   if (!a.pairs) {
     int first = 0;
     for (int m = 0; m < M; ++m) {
@@ -114,7 +117,9 @@ __device__ void bucket_body(const BucketArgs& a, int bg) {
         d.code = (kRouted << 24) | (bg * M + m);
         d.row0 = row0;
         d.nrows = nrows;
-        d.nkv = last / kTileN + 1;
+        // KV tiles from the one of kv_start to the last row's; at least one,
+        // so rows that are all padding are still written (as zeros)
+        d.nkv = max(1, (qo + last) / kTileN + 1 - j0);
         slots[first + t] = d;
       }
       first += nt;
@@ -139,7 +144,7 @@ __device__ void bucket_body(const BucketArgs& a, int bg) {
   const int ntiles = tfirst[M];
   const int32_t* tok = a.bucket_tok + base;
   auto tile_nkv = [&](int m, int t) {
-    return tok[start[m] + min(t * kTileM + kTileM - 1, cnt[m] - 1)] / kTileN + 1;
+    return max(1, (qo + tok[start[m] + min(t * kTileM + kTileM - 1, cnt[m] - 1)]) / kTileN + 1 - j0);
   };
   for (int i = tid; i < ntiles; i += kBucketThreads) {
     int m = 0;
@@ -176,26 +181,29 @@ __device__ void bucket_body(const BucketArgs& a, int bg) {
 // pairs: query tiles q and q-1 of one batch), then the work items (tiles, or
 // pairs by the KV-tile count of their first tile) are sorted longest first,
 // so the heaviest work starts first and the grid's tail is short.  Counting
-// sort on nkv in [1, ceil(S/128)].
+// sort on nkv in [1, ceil(T/128)].
 constexpr int kSchedThreads = 1024;
 
-__device__ void schedule_body(const BucketArgs& a, int* hist /* nq + 2 bins */) {
+__device__ void schedule_body(const BucketArgs& a, int* hist /* ceil(T/128) + 2 bins */) {
   const int tid = threadIdx.x;
   const int nq = (a.S + kTileM - 1) / kTileM;
   const int nq2 = nq + (nq & 1);
+  const int nkv_max = (a.T + kTileN - 1) / kTileN;
   const int64_t n_routed = static_cast<int64_t>(a.B) * a.G * a.cap_bg;
   TileDesc* shared_tiles = a.tiles_raw + n_routed;
-  for (int v = tid; v < nq + 2; v += kSchedThreads) hist[v] = 0;
+  for (int v = tid; v < nkv_max + 2; v += kSchedThreads) hist[v] = 0;
   // the shared head's tiles: every token, KV head 0; slot i of a batch holds
   // query tile nq-1-i (so pair i/2 is tiles nq-1-2(i/2) and nq-2-2(i/2))
   for (int64_t t = tid; t < static_cast<int64_t>(a.B) * nq2; t += kSchedThreads) {
     const int b = static_cast<int>(t / nq2), q = nq - 1 - static_cast<int>(t % nq2);
     TileDesc d{0, 0, 0, 0};
     if (q >= 0) {
+      int qo, kvs;
+      seq_offsets(a.q_off, a.kv_start, b, a.S, a.T, a.status, &qo, &kvs);
       d.code = (kShared << 24) | b;
       d.row0 = q * kTileM;
       d.nrows = min(kTileM, a.S - q * kTileM);
-      d.nkv = q + 1;
+      d.nkv = max(1, (qo + d.row0 + d.nrows - 1) / kTileN + 1 - kvs / kTileN);
     }
     shared_tiles[t] = d;
   }
@@ -209,7 +217,7 @@ __device__ void schedule_body(const BucketArgs& a, int* hist /* nq + 2 bins */) 
   __syncthreads();
   if (tid == 0) {  // exclusive scan from the largest nkv down
     int s = 0;
-    for (int v = nq; v >= 1; --v) {
+    for (int v = nkv_max; v >= 1; --v) {
       const int c = hist[v];
       hist[v] = s;
       s += c;
@@ -321,8 +329,8 @@ __global__ void combine_kernel(const CombineArgs a) {
 
 cudaError_t launch_prep(const BucketArgs& a, const ConvertArgs* cv, bool with_schedule,
                         cudaStream_t st) {
-  const int nq = (a.S + kTileM - 1) / kTileM;
-  const size_t smem = with_schedule ? sizeof(int) * (nq + 2) : 0;
+  const int nkv_max = (a.T + kTileN - 1) / kTileN;
+  const size_t smem = with_schedule ? sizeof(int) * (nkv_max + 2) : 0;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

@@ -60,9 +60,11 @@ struct WsLayout {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-inline WsLayout make_ws_layout(const gqe_dims& d) {
+// T: KV slots per sequence (the V conversion's size); S when not chunked.
+inline WsLayout make_ws_layout(const gqe_dims& d, int64_t T = -1) {
   WsLayout L{};
   const int64_t B = d.B, S = d.S, G = d.G, M = d.N / d.G, k = d.k, hd = d.d;
+  if (T < S) T = S;
   tile_list_dims(B, S, G, M, k, &L.cap_bg, &L.n_raw_tiles);
   size_t off = 0;
   L.status = off;     off += 256;
@@ -70,7 +72,7 @@ inline WsLayout make_ws_layout(const gqe_dims& d) {
   L.fix_list = off;   off = align_up(off + sizeof(int32_t) * B * S * G, 256);
   L.wt = off;         off = align_up(off + sizeof(float) * d.d_model * G * M, 256);
   L.wsq = off;        off = align_up(off + sizeof(float) * G * M, 256);
-  L.v16 = off;        off = align_up(off + sizeof(uint16_t) * B * S * G * hd, 256);
+  L.v16 = off;        off = align_up(off + sizeof(uint16_t) * B * T * G * hd, 256);
   L.bucket_off = off; off = align_up(off + sizeof(int32_t) * (B * G * M + 1), 256);
   L.bucket_tok = off; off = align_up(off + sizeof(int32_t) * B * G * S * k, 256);
   L.tiles_raw = off;  off = align_up(off + sizeof(TileDesc) * L.n_raw_tiles, 256);
@@ -97,6 +99,27 @@ struct RouteArgs {
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 
+// Chunked prefill over a cache: query row i of sequence b sits at absolute
+// position q_off[b] + i of a KV sequence of T slots, and sees slots
+// kv_start[b]..q_off[b] + i ("AI 大模型之 GQA", 工程实操: the causal mask on
+// absolute positions, intersected with key validity).  Null arrays mean 0.
+// A value outside its range (q_off not in [0, T - S], kv_start not in
+// [0, T)) latches GQE_ERR_BAD_POSITION and is taken as 0.
+__device__ __forceinline__ void seq_offsets(const int32_t* q_off, const int32_t* kv_start, int b,
+                                            int S, int T, int* status, int* qo, int* kvs) {
+  int o = q_off ? q_off[b] : 0, v = kv_start ? kv_start[b] : 0;
+  if (o < 0 || o > T - S) {
+    atomicCAS(status, 0, GQE_ERR_BAD_POSITION);
+    o = 0;
+  }
+  if (v < 0 || v >= T) {
+    atomicCAS(status, 0, GQE_ERR_BAD_POSITION);
+    v = 0;
+  }
+  *qo = o;
+  *kvs = v;
+}
+
 struct BucketArgs {
   const int32_t* topk_idx;  // [B,S,G,k]
   int32_t* bucket_off;      // [B*G*M+1]
@@ -110,6 +133,12 @@ struct BucketArgs {
   int pairs;                // 1: build the paired list of the pair kernel
   int64_t cap_bg;
   int64_t n_raw_tiles;
+  // chunked prefill (see seq_offsets); T = S and null arrays otherwise.  A
+  // tile's nkv is then the number of KV tiles it visits, from the tile of
+  // kv_start[b] on.
+  const int32_t* q_off;
+  const int32_t* kv_start;
+  int T;
 };
 
 struct ConvertArgs {
@@ -142,6 +171,9 @@ struct AttnArgs {
   int* status;
   int B, S, N, G, M, k, d;
   int out_fp32;
+  const int32_t* q_off;     // chunked prefill (see seq_offsets); null: 0
+  const int32_t* kv_start;  // null: 0
+  int T;                    // KV slots per sequence (K/V maps are [B, T, G, d])
   int dense;          // 1: dense GQA tiles from blockIdx; 0: routed/shared list
   int pair;           // 1: the pair kernel on a paired list (d = 64 only)
   float scale_log2;   // log2(e) / sqrt(d)
@@ -166,6 +198,34 @@ struct CombineArgs {
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 
 cudaError_t launch_selftest_wait(int* status, uint64_t limit_ns, cudaStream_t st);
+
+// Projections (gqe_gemm.cu): bf16 operands, fp32 accumulation in TMEM.
+struct GemmArgs {
+  CUtensorMap tmA;      // dense form: bf16 A [rows, K] (row stride lda), box {64, 128}
+  CUtensorMap tmB;      // bf16 B stack [nb, K, nc], box {64, 64, 1}
+  const uint16_t* A;    // routed form: bf16 x [B, S, lda] (rows gathered)
+  int64_t lda;
+  void* C;              // dense form: [rows, ldc] (fp32 or bf16); routed form: bf16 Q [B,S,N,d]
+  int64_t ldc;
+  int c_fp32;
+  int K;                // reduction length, a multiple of 64
+  int nc;               // columns of one B matrix (a multiple of 64)
+  int n_total;          // columns of C in the dense form (nb * nc or a part of it)
+  int rows;             // rows of A and C in the dense form
+  // routed form: the attention work list and the bucket lists
+  const int32_t* bucket_off;
+  const int32_t* bucket_tok;
+  const TileDesc* tiles;
+  const int32_t* tile_count;
+  int B, S, N, G, M, d;
+  int* status;
+  uint64_t wait_limit_ns;
+};
+// C = A . B over 128-row tiles and bn-column tiles (bn in {64, 128, 256},
+// n_total % bn == 0).
+cudaError_t launch_gemm_dense(const GemmArgs& a, int bn, cudaStream_t st);
+// Q of the selected heads, one CTA per routed tile of the work list.
+cudaError_t launch_gemm_routed(const GemmArgs& a, int64_t n_list, cudaStream_t st);
 
 // ------------------------------------------------------------ host helpers
 // (gqe_host.cu; shared by every entry point)

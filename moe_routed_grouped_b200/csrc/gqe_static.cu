@@ -118,6 +118,7 @@ extern "C" gqe_status gqe_attention_prefill_static(
   ba.k = dims->k;
   ba.cap_bg = L.cap_bg;
   ba.n_raw_tiles = L.n_raw_tiles;
+  ba.T = dims->S;
   const bool pair = gqe::pair_kernel_for(*dims);  // one decision: list format and kernel
   ba.pairs = pair ? 1 : 0;
   if (gqe::launch_prep(ba, &cv, true, s) != cudaSuccess) return GQE_ERR_CUDA;
@@ -151,6 +152,7 @@ extern "C" gqe_status gqe_attention_prefill_static(
   a.k = dims->k;
   a.d = dims->d;
   a.out_fp32 = dims->out_fp32;
+  a.T = dims->S;
   a.dense = 0;
   a.pair = pair ? 1 : 0;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));

@@ -143,6 +143,65 @@ class GqePrefill:
         return _lib.gqe_get_device_status(self.ws, 1 if clear else 0, stream)
 
 
+class GqeChunk:
+    """Buffers and calls for chunked prefill: S new tokens per sequence over
+    KV caches of T slots (gqe_route on the chunk, then
+    gqe_attention_prefill_chunk).  ``concat`` has one W_O input row per chunk
+    token (row b*S + i), laid out as in :class:`GqePrefill`."""
+
+    def __init__(self, B, S, T, N, G, k, d, d_model, out_fp32=True, device="cuda"):
+        if N % G:
+            raise ValueError("N must be a multiple of G")
+        self.B, self.S, self.T, self.N, self.G, self.k, self.d = B, S, T, N, G, k, d
+        self.d_model, self.M = d_model, N // G
+        self.dims = _lib.dims(B, S, N, G, k, d, d_model, 1 if out_fp32 else 0)
+        a = _lib.gqe_workspace_size(self.dims)
+        b = _lib.gqe_prefill_chunk_workspace_size(self.dims, T)
+        if a == 0 or b == 0:
+            raise _lib.GqeError(2, "gqe_prefill_chunk_workspace_size")
+        dev = _device(device)
+        self.device = dev
+        self.ws = torch.zeros(max(a, b), dtype=torch.uint8, device=dev)
+        self.out_dtype = torch.float32 if out_fp32 else torch.bfloat16
+        self.row = (G * k + G + 1) * d
+        self.concat = torch.empty(B * S, self.row, dtype=self.out_dtype, device=dev)
+        self.topk_idx = torch.empty(B, S, G, k, dtype=torch.int32, device=dev)
+        self.p = torch.empty(B, S, G, self.M, dtype=torch.float32, device=dev)
+        self.w = torch.empty(B, S, G, k, dtype=torch.float32, device=dev)
+
+    O_sel = GqePrefill.O_sel
+    o_bar = GqePrefill.o_bar
+    s_out = GqePrefill.s_out
+
+    def route(self, x, W_r, bias=None, stream=None):
+        return GqePrefill.route(self, x, W_r, bias, stream)
+
+    def attention(self, Q, Qs, Kc, Vc, q_off=None, kv_start=None, stream=None):
+        """Q [B, S, N, d], Qs [B, S, d] (the chunk), caches Kc, Vc [B, T, G, d];
+        q_off, kv_start: int32 [B] on the device, or None (0)."""
+        bf, dv = torch.bfloat16, self.device
+        _expect(Q, "Q", (self.B, self.S, self.N, self.d), bf, dv)
+        _expect(Qs, "Qs", (self.B, self.S, self.d), bf, dv)
+        _expect(Kc, "Kc", (self.B, self.T, self.G, self.d), bf, dv)
+        _expect(Vc, "Vc", (self.B, self.T, self.G, self.d), bf, dv)
+        for t, name in ((q_off, "q_off"), (kv_start, "kv_start")):
+            if t is not None:
+                _expect(t, name, (self.B,), torch.int32, dv)
+        a = self.G * self.k * self.d
+        flat = self.concat.view(-1)
+        _lib.gqe_attention_prefill_chunk(self.dims, self.T, Q, Qs, Kc, Vc, q_off, kv_start,
+                                         self.topk_idx, self.w, self.concat, flat[a:],
+                                         flat[a + self.G * self.d:], self.row, self.ws, stream)
+        return self.concat
+
+    def forward(self, x, W_r, bias, Q, Qs, Kc, Vc, q_off=None, kv_start=None, stream=None):
+        self.route(x, W_r, bias, stream)
+        return self.attention(Q, Qs, Kc, Vc, q_off, kv_start, stream)
+
+    def device_status(self, clear=True, stream=None) -> int:
+        return _lib.gqe_get_device_status(self.ws, 1 if clear else 0, stream)
+
+
 class GqeDecode:
     """Buffers and calls for one decode step of B sequences over KV caches of
     capacity T (shape [B, T, G, d]); with ``n_new`` > 1, n_new new tokens per
@@ -246,6 +305,85 @@ class GqeDecode:
         with torch.cuda.graph(g):
             self.forward(x, W_r, bias, Q, Qs, Kc, Vc, pos, kv_start)
         return g
+
+    def device_status(self, clear=True, stream=None) -> int:
+        return _lib.gqe_get_device_status(self.ws, 1 if clear else 0, stream)
+
+
+class GqeLayer:
+    """Buffers and calls for the whole GQE attention layer of one shape,
+    x -> y (gqe_layer_prefill), and the all-active GQA layer baseline
+    (gqe_dense_layer_prefill).
+
+    Weights (bf16): W_Q [N, d_model, d], W_K and W_V [G, d_model, d], W_s
+    [d_model, d], W_r [G, d_model, M], W_O [(G*k + G + 1)*d, d_model] (rows in
+    concat order); the baseline's W_O is [N*d, d_model].  Intermediates are
+    kept in this object: ``Q`` (only the selected heads' rows are written),
+    ``Qs``, ``K``, ``V``, ``concat`` (bf16), ``topk_idx``, ``p``, ``w``; the
+    output ``y`` is float32 [B, S, d_model].
+    """
+
+    def __init__(self, B, S, N, G, k, d, d_model, device="cuda"):
+        if N % G:
+            raise ValueError("N must be a multiple of G")
+        self.B, self.S, self.N, self.G, self.k, self.d, self.d_model = B, S, N, G, k, d, d_model
+        self.M = N // G
+        self.dims = _lib.dims(B, S, N, G, k, d, d_model, 0)
+        nbytes = _lib.gqe_workspace_size(self.dims)
+        if nbytes == 0:
+            raise _lib.GqeError(2, "gqe_workspace_size")
+        dev = _device(device)
+        self.device = dev
+        bf = torch.bfloat16
+        self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        self.row = (G * k + G + 1) * d
+        self.Q = torch.zeros(B, S, N, d, dtype=bf, device=dev)
+        self.Qs = torch.empty(B, S, d, dtype=bf, device=dev)
+        self.K = torch.empty(B, S, G, d, dtype=bf, device=dev)
+        self.V = torch.empty(B, S, G, d, dtype=bf, device=dev)
+        self.concat = torch.empty(B * S, self.row, dtype=bf, device=dev)
+        self.y = torch.empty(B, S, d_model, dtype=torch.float32, device=dev)
+        self.topk_idx = torch.empty(B, S, G, k, dtype=torch.int32, device=dev)
+        self.p = torch.empty(B, S, G, self.M, dtype=torch.float32, device=dev)
+        self.w = torch.empty(B, S, G, k, dtype=torch.float32, device=dev)
+        self._dense = None
+
+    def _check_weights(self, W_Q, W_K, W_V):
+        bf, dv = torch.bfloat16, self.device
+        _expect(W_Q, "W_Q", (self.N, self.d_model, self.d), bf, dv)
+        _expect(W_K, "W_K", (self.G, self.d_model, self.d), bf, dv)
+        _expect(W_V, "W_V", (self.G, self.d_model, self.d), bf, dv)
+
+    def forward(self, x, W_Q, W_K, W_V, W_s, W_r, bias, W_O, stream=None):
+        bf, dv = torch.bfloat16, self.device
+        _expect(x, "x", (self.B, self.S, self.d_model), bf, dv)
+        self._check_weights(W_Q, W_K, W_V)
+        _expect(W_s, "W_s", (self.d_model, self.d), bf, dv)
+        _expect(W_r, "W_r", (self.G, self.d_model, self.M), bf, dv)
+        if bias is not None:
+            _expect(bias, "bias", (self.G, self.M), torch.float32, dv)
+        _expect(W_O, "W_O", (self.row, self.d_model), bf, dv)
+        _lib.gqe_layer_prefill(self.dims, x, W_Q, W_K, W_V, W_s, W_r, bias, W_O, self.topk_idx,
+                               self.p, self.w, self.Q, self.Qs, self.K, self.V, self.concat,
+                               self.y, self.ws, stream)
+        return self.y
+
+    def dense(self, x, W_Q, W_K, W_V, W_O, stream=None):
+        """The all-active GQA layer; returns its own y (float32)."""
+        bf, dv = torch.bfloat16, self.device
+        _expect(x, "x", (self.B, self.S, self.d_model), bf, dv)
+        self._check_weights(W_Q, W_K, W_V)
+        _expect(W_O, "W_O", (self.N * self.d, self.d_model), bf, dv)
+        if self._dense is None:
+            B, S, N, d = self.B, self.S, self.N, self.d
+            self._dense = dict(Q=torch.empty(B, S, N, d, dtype=bf, device=dv),
+                               K=torch.empty_like(self.K), V=torch.empty_like(self.V),
+                               O=torch.empty(B, S, N, d, dtype=bf, device=dv),
+                               y=torch.empty_like(self.y))
+        t = self._dense
+        _lib.gqe_dense_layer_prefill(self.dims, x, W_Q, W_K, W_V, W_O, t["Q"], t["K"], t["V"],
+                                     t["O"], t["y"], self.ws, stream)
+        return t["y"]
 
     def device_status(self, clear=True, stream=None) -> int:
         return _lib.gqe_get_device_status(self.ws, 1 if clear else 0, stream)
