@@ -420,6 +420,69 @@ def measure_workload(torch, w, device, rank, steps, warmup, flush, host_gen, wit
                 dense_attn_ms=d_attn, t0=t0, t1=t1, dense_t0=d0, dense_t1=d1)
 
 
+def layer_entry(torch, device, local, flush, peaks, peak_src, steps=20, warmup=3):
+    """The whole attention layer at the bench shape (gqe_layer_prefill: router,
+    K/V/Qs projections, the selected heads' Q projection, attention, W_O)
+    against the all-active GQA layer (gqe_dense_layer_prefill), plus the W_O
+    projection alone against the tensor-core peak.  Random bf16 weights with
+    std d_model^-1/2; inputs from torch's generator."""
+    from moe_routed_grouped_b200.layer import GqeLayer
+    import moe_routed_grouped_b200 as gqe
+    w = WORKLOADS["layer250m"]
+    B, S, N, G, k, d, dm, M = w.B, w.S, w.N, w.G, w.k, w.d, w.d_model, w.M
+    g = torch.Generator(device=device)
+    g.manual_seed(9100)
+
+    def rn(*shape, std=1.0):
+        t = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        t.normal_(0.0, std, generator=g)
+        return t
+    row = (G * k + G + 1) * d
+    sd = dm ** -0.5
+    W = dict(Q=rn(N, dm, d, std=sd), K=rn(G, dm, d, std=sd), V=rn(G, dm, d, std=sd),
+             s=rn(dm, d, std=sd), r=rn(G, dm, M, std=sd), O=rn(row, dm, std=row ** -0.5),
+             Od=rn(N * d, dm, std=(N * d) ** -0.5))
+    x = rn(B, S, dm)
+    L = GqeLayer(B, S, N, G, k, d, dm, device=device)
+    cs = ClockSampler(local)
+    cs.start()
+    try:
+        r_ms, _, t0, t1 = timed_loop(
+            torch, lambda: L.forward(x, W["Q"], W["K"], W["V"], W["s"], W["r"], None, W["O"]),
+            steps, warmup, flush)
+        d_ms, _, d0, d1 = timed_loop(
+            torch, lambda: L.dense(x, W["Q"], W["K"], W["V"], W["Od"]), steps, warmup, flush)
+        T = B * S
+        Y = torch.empty(T, dm, dtype=torch.float32, device=device)
+        o_ms, _, _, _ = timed_loop(
+            torch, lambda: gqe.gqe_linear(T, row, 1, dm, L.concat, row, W["O"], Y, dm, 1),
+            steps, warmup, flush)
+    finally:
+        cs.stop()
+    if L.device_status() != 0:
+        raise RuntimeError("device status after the layer loop")
+    T = B * S
+    attn_r, attn_d = w.useful_flop_routed(), w.useful_flop_dense()
+    proj_r = 2.0 * T * dm * (2 * G * d + d + G * k * d) + 2.0 * T * row * dm + 2.0 * T * dm * G * M
+    proj_d = 2.0 * T * dm * (2 * G * d + N * d) + 2.0 * T * N * d * dm
+    rm, dmm, om = statistics.mean(r_ms), statistics.mean(d_ms), statistics.mean(o_ms)
+    o_tf = 2.0 * T * row * dm / (om / 1e3) / 1e12
+    return {"workload": "layer250m", "steps": steps, "warmup": warmup,
+            "routed_ms": rm, "dense_ms": dmm, "routed_over_dense": dmm / rm,
+            "routed_tokens_per_s": T / (rm / 1e3), "dense_tokens_per_s": T / (dmm / 1e3),
+            "routed_flop": attn_r + proj_r, "dense_flop": attn_d + proj_d,
+            "routed_tflops": (attn_r + proj_r) / (rm / 1e3) / 1e12,
+            "dense_tflops": (attn_d + proj_d) / (dmm / 1e3) / 1e12,
+            "w_o_gemm": {"kernel": "gemm_dense_kernel (T x %d x %d, bf16 in, fp32 out)" % (row, dm),
+                         "ms": om, "tflops": o_tf, "peak": peaks["bf16_tflops"],
+                         "frac": o_tf / peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16 dense (burst)"},
+            "clocks": cs.summary(t0, d1),
+            # routed layer 10 kernels (2 router, 3 projections, 2 routed Q, 2 attention,
+            # W_O), dense layer 6, W_O alone 1
+            "gpu_launches": steps * (10 + 6 + 1)}
+
+
 # the long-context workloads every default line also measures: (name, timed steps)
 CONFIG_ENTRIES = (("imbalanced32k", 10), ("wide131k", 5), ("million", 3))
 
@@ -654,6 +717,12 @@ def main():
     }
 
     if world == 1 and not args.no_configs:
+        try:
+            line["layer"] = layer_entry(torch, device, local, flush, peaks, peak_src)
+            line["gpu_launches"] += line["layer"]["gpu_launches"]
+        except Exception as ex:  # noqa: BLE001  (reported in the entry, not hidden)
+            line["layer"] = {"workload": "layer250m", "error": f"{type(ex).__name__}: {ex}"[:300]}
+        torch.cuda.empty_cache()
         # the S >= 32k workloads, each with its own timing and clock record
         del res
         torch.cuda.empty_cache()
