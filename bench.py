@@ -602,6 +602,74 @@ def e2e_measure(torch, w, L, dev, steps):
     return ms, h2d, d2h
 
 
+# Small cases that run a kernel a few times without timing, for a profiler to
+# capture one launch (inputs from torch's generator; a few hundred MB on the
+# device at most, more than the 126 MB L2).
+NCU_CASES = ("attn_d64_32k", "attn_d128_32k", "pair_d64_32k", "layer250m", "bwd_d64_8k",
+             "decode_32k")
+
+
+def run_ncu_case(torch, name, device, reps=2):
+    import moe_routed_grouped_b200 as gqe
+    from moe_routed_grouped_b200.layer import GqeDecode, GqeLayer, GqePrefill
+    g = torch.Generator(device=device)
+    g.manual_seed(5)
+
+    def rn(*shape, std=1.0):
+        t = torch.empty(shape, dtype=torch.bfloat16, device=device)
+        t.normal_(0.0, std, generator=g)
+        return t
+    if name == "layer250m":
+        w = WORKLOADS["layer250m"]
+        B, S, N, G, k, d, dm, M = w.B, w.S, w.N, w.G, w.k, w.d, w.d_model, w.M
+        row, sd = (G * k + G + 1) * d, dm ** -0.5
+        W = [rn(N, dm, d, std=sd), rn(G, dm, d, std=sd), rn(G, dm, d, std=sd), rn(dm, d, std=sd),
+             rn(G, dm, M, std=sd)]
+        Wo, x = rn(row, dm, std=row ** -0.5), rn(B, S, dm)
+        L = GqeLayer(B, S, N, G, k, d, dm, device=device)
+        for _ in range(reps):
+            L.forward(x, *W, None, Wo)
+    elif name == "decode_32k":
+        B, T, N, G, k, d, dm = 1, 32768, 16, 8, 1, 64, 1024
+        L = GqeDecode(B, T, N, G, k, d, dm, device=device)
+        args = (rn(B, dm), rn(G, dm, N // G, std=dm ** -0.5), None, rn(B, N, d), rn(B, d),
+                rn(B, T, G, d), rn(B, T, G, d),
+                torch.full((B,), T - 1, dtype=torch.int32, device=device))
+        for _ in range(reps):
+            L.forward(*args)
+    else:
+        shapes = {"attn_d64_32k": (1, 32768, 16, 8, 1, 64, 1024, 1.5),
+                  "attn_d128_32k": (1, 32768, 32, 8, 2, 128, 1024, 0.0),
+                  "pair_d64_32k": (1, 32768, 16, 8, 1, 64, 1024, 1.5),
+                  "bwd_d64_8k": (1, 8192, 16, 8, 1, 64, 1024, 0.0)}
+        B, S, N, G, k, d, dm, b0 = shapes[name]
+        M = N // G
+        bias = None
+        if b0:
+            bias = torch.zeros(G, M, dtype=torch.float32, device=device)
+            bias[:, 0] = b0
+        x, Wr = rn(B, S, dm), rn(G, dm, M, std=dm ** -0.5)
+        Q, Qs, K, V = rn(B, S, N, d), rn(B, S, d), rn(B, S, G, d), rn(B, S, G, d)
+        L = GqePrefill(B, S, N, G, k, d, dm, device=device)
+        prev = gqe.gqe_set_pair_threshold(0 if name.startswith("pair") else -1)
+        try:
+            if name.startswith("bwd"):
+                L.forward_train(x, Wr, bias, Q, Qs, K, V)
+                dcat = torch.randn(B * S, L.row, generator=g, device=device)
+                for _ in range(reps):
+                    L.backward(dcat)
+            else:
+                L.route(x, Wr, bias)
+                for _ in range(reps):
+                    L.attention(Q, Qs, K, V)
+        finally:
+            gqe.gqe_set_pair_threshold(prev)
+    torch.cuda.synchronize()
+    st = L.device_status()
+    print(json.dumps({"ncu_case": name, "device_status": st}), flush=True)
+    return 0 if st == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -614,6 +682,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="leave the decode-step measurements out of the prefill line")
+    ap.add_argument("--ncu-case", choices=NCU_CASES, default=None,
+                    help="run one small case's kernels a few times, untimed, for a profiler")
     ap.add_argument("--decode", action="store_true",
                     help="time one decode step per sequence over a full cache of S tokens "
                          "instead of the prefill (prints its own line)")
@@ -646,6 +716,9 @@ def main():
     peaks, peak_src = load_peaks()
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     flush = lambda: flush_buf.zero_()  # noqa: E731
+
+    if args.ncu_case:
+        return run_ncu_case(torch, args.ncu_case, device)
 
     w = WORKLOADS[args.workload]
     if args.decode:

@@ -332,6 +332,59 @@ void gqe_set_profile_events(void* begin, void* end);
 int64_t gqe_set_pair_threshold(int64_t kv_bytes);
 
 /* ------------------------------------------------------------------------
+ * Training: the forward call that also keeps each row's log-sum-exp, and the
+ * backward pass of the path.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * gqe_attention_prefill_train - gqe_attention_prefill (float32 outputs:
+ * dims->out_fp32 must be 1) that also writes, per routed slot and per
+ * shared-head row, the base-2 log-sum-exp of that row's scaled scores
+ * (log2 sum_t 2^(q.k_t log2(e)/sqrt(d))): what the backward pass needs to
+ * rebuild the softmax without a second forward.
+ *  lse_sel  device float32 [B, S, G, k] (slot order);  lse_s float32 [B, S]
+ */
+gqe_status gqe_attention_prefill_train(const gqe_dims* dims, const void* Q, const void* Qs,
+                                       const void* K, const void* V, const int32_t* topk_idx,
+                                       const float* w, void* O_sel, void* o_bar, void* s_out,
+                                       int64_t out_row_stride, float* lse_sel, float* lse_s,
+                                       void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace gqe_prefill_backward needs for `dims` (0 if invalid). */
+size_t gqe_prefill_backward_workspace_size(const gqe_dims* dims);
+
+/*
+ * gqe_prefill_backward - gradients of the path's outputs (O_sel, o_bar, s)
+ * with respect to Q, Qs, K, V and the weights w, for upstream gradients in
+ * the concat layout.  "AI 大模型之 GQA", 训练与部署 共享键值的梯度归约: each
+ * query head's attention backward is computed on its own and the gradients
+ * of a KV head are the SUM over every head that reads it (the routed experts
+ * of the group that a token selected, and the shared head for KV head 0);
+ * review §二 三个关键部件: o_bar = sum_j w_j o_j, so slot j receives
+ * dO_sel_j + w_j d(o_bar), and dw_j = <d(o_bar), o_j> (the gradient the
+ * weighted-sum slot gives the router; at k = 1, w = 1 and the caller may
+ * drop it).  The selection itself is held fixed.
+ *  Q, Qs, K, V, topk_idx, w  the forward's inputs (bf16 / int32 / float32)
+ *  O_sel, s_out  the forward's float32 outputs, rows at out_row_stride
+ *                (the concat buffer of gqe_attention_prefill_train)
+ *  lse_sel, lse_s  from gqe_attention_prefill_train
+ *  dO_sel, do_bar, ds  float32 upstream gradients, rows at dout_row_stride
+ *                (the concat layout: slot j of group g at (g*k + j)*d)
+ *  dQ   float32 [B, S, N, d]: rows of heads a token did not select are 0
+ *  dQs  float32 [B, S, d];  dK, dV float32 [B, S, G, d];  dw float32 [B, S, G, k]
+ *  ws   gqe_prefill_backward_workspace_size(dims) bytes
+ * The tensor-core products take bf16 operands: the effective dO, P and dS
+ * are rounded to bf16 (float32 accumulation).
+ */
+gqe_status gqe_prefill_backward(const gqe_dims* dims, const void* Q, const void* Qs,
+                                const void* K, const void* V, const int32_t* topk_idx,
+                                const float* w, const float* O_sel, const float* s_out,
+                                int64_t out_row_stride, const float* lse_sel, const float* lse_s,
+                                const float* dO_sel, const float* do_bar, const float* ds,
+                                int64_t dout_row_stride, float* dQ, float* dQs, float* dK,
+                                float* dV, float* dw, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * The attention layer around the path: projections and W_O.
  * Review §二 路由器: only the query heads the router selected are computed at
  * all, so their query projection runs for the selected (token, head) pairs

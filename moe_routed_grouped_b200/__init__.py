@@ -13,5 +13,6 @@ from ._lib import (  # noqa: F401
     gqe_selftest_bounded_wait, gqe_set_pair_threshold, gqe_set_profile_events, gqe_status_string,
     gqe_workspace_size, gqe_static_device_status, gqe_linear, gqe_routed_q_project,
     gqe_layer_prefill, gqe_dense_layer_prefill, gqe_prefill_chunk_workspace_size,
-    gqe_attention_prefill_chunk,
+    gqe_attention_prefill_chunk, gqe_attention_prefill_train, gqe_prefill_backward_workspace_size,
+    gqe_prefill_backward,
 )

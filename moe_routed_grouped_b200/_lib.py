@@ -21,6 +21,7 @@ EXPORTS = (
     "gqe_attention_decode", "gqe_append_workspace_size", "gqe_attention_append",
     "gqe_static_device_status", "gqe_linear", "gqe_routed_q_project", "gqe_layer_prefill",
     "gqe_dense_layer_prefill", "gqe_prefill_chunk_workspace_size", "gqe_attention_prefill_chunk",
+    "gqe_attention_prefill_train", "gqe_prefill_backward_workspace_size", "gqe_prefill_backward",
 )
 
 STATUS = {0: "GQE_OK", 1: "GQE_ERR_INVALID_ARG", 2: "GQE_ERR_UNSUPPORTED", 3: "GQE_ERR_CUDA",
@@ -69,6 +70,10 @@ def _load() -> ctypes.CDLL:
         "gqe_dense_layer_prefill": (I32, [S] + [P] * 11 + [SZ, P]),
         "gqe_prefill_chunk_workspace_size": (SZ, [S, I32]),
         "gqe_attention_prefill_chunk": (I32, [S, I32] + [P] * 11 + [I64, P, SZ, P]),
+        "gqe_attention_prefill_train": (I32, [S] + [P] * 9 + [I64, P, P, P, SZ, P]),
+        "gqe_prefill_backward_workspace_size": (SZ, [S]),
+        "gqe_prefill_backward": (I32, [S] + [P] * 8 + [I64, P, P, P, P, P, I64] + [P] * 5
+                                 + [P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -193,6 +198,30 @@ def gqe_attention_prefill_chunk(dm, T, Q, Qs, Kc, Vc, q_off, kv_start, topk_idx,
         _ptr(kv_start), _ptr(topk_idx), _ptr(w), _ptr(O_sel), _ptr(o_bar), _ptr(s_out),
         int(out_row_stride), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     return _check(r, "gqe_attention_prefill_chunk") if check else r
+
+
+def gqe_attention_prefill_train(dm, Q, Qs, K, V, topk_idx, w, O_sel, o_bar, s_out,
+                                out_row_stride, lse_sel, lse_s, ws, stream=None, check=True):
+    r = LIB.gqe_attention_prefill_train(
+        ctypes.byref(dm), _ptr(Q), _ptr(Qs), _ptr(K), _ptr(V), _ptr(topk_idx), _ptr(w),
+        _ptr(O_sel), _ptr(o_bar), _ptr(s_out), int(out_row_stride), _ptr(lse_sel), _ptr(lse_s),
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_attention_prefill_train") if check else r
+
+
+def gqe_prefill_backward_workspace_size(dm: GqeDims) -> int:
+    return LIB.gqe_prefill_backward_workspace_size(ctypes.byref(dm))
+
+
+def gqe_prefill_backward(dm, Q, Qs, K, V, topk_idx, w, O_sel, s_out, out_row_stride, lse_sel,
+                         lse_s, dO_sel, do_bar, ds, dout_row_stride, dQ, dQs, dK, dV, dw, ws,
+                         stream=None, check=True):
+    r = LIB.gqe_prefill_backward(
+        ctypes.byref(dm), _ptr(Q), _ptr(Qs), _ptr(K), _ptr(V), _ptr(topk_idx), _ptr(w),
+        _ptr(O_sel), _ptr(s_out), int(out_row_stride), _ptr(lse_sel), _ptr(lse_s), _ptr(dO_sel),
+        _ptr(do_bar), _ptr(ds), int(dout_row_stride), _ptr(dQ), _ptr(dQs), _ptr(dK), _ptr(dV),
+        _ptr(dw), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    return _check(r, "gqe_prefill_backward") if check else r
 
 
 def gqe_linear(rows, K, nb, nc, A, lda, W, C, ldc, c_fp32, stream=None, check=True):

@@ -122,7 +122,8 @@ gqe_status attention_prefill_impl(const gqe_dims* dims, int32_t T, const void* Q
                                   const int32_t* kv_start, const int32_t* topk_idx,
                                   const float* w, void* O_sel, void* o_bar, void* s_out,
                                   int64_t out_row_stride, void* ws, size_t ws_bytes,
-                                  void* stream) {
+                                  void* stream, float* lse_sel = nullptr,
+                                  float* lse_s = nullptr) {
   gqe_status st = check_dims(dims, false);
   if (st != GQE_OK) return st;
   if (T < dims->S) return GQE_ERR_INVALID_ARG;
@@ -175,6 +176,8 @@ gqe_status attention_prefill_impl(const gqe_dims* dims, int32_t T, const void* Q
   a.q_off = q_off;
   a.kv_start = kv_start;
   a.T = T;
+  a.lse_sel = lse_sel;
+  a.lse_s = lse_s;
   a.dense = 0;
   a.pair = pair ? 1 : 0;
   e = timed_attention(a, L.n_raw_tiles, s);
@@ -206,6 +209,19 @@ gqe_status gqe_attention_prefill(const gqe_dims* dims, const void* Q, const void
 size_t gqe_prefill_chunk_workspace_size(const gqe_dims* dims, int32_t T) {
   if (check_dims(dims, false) != GQE_OK || T < dims->S) return 0;
   return make_ws_layout(*dims, T).total;
+}
+
+gqe_status gqe_attention_prefill_train(const gqe_dims* dims, const void* Q, const void* Qs,
+                                       const void* K, const void* V, const int32_t* topk_idx,
+                                       const float* w, void* O_sel, void* o_bar, void* s_out,
+                                       int64_t out_row_stride, float* lse_sel, float* lse_s,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  if (!dims) return GQE_ERR_INVALID_ARG;
+  if (dims->out_fp32 != 1 || !aligned16(lse_sel) || !aligned16(lse_s))
+    return GQE_ERR_INVALID_ARG;
+  return attention_prefill_impl(dims, dims->S, Q, Qs, K, V, nullptr, nullptr, topk_idx, w, O_sel,
+                                o_bar, s_out, out_row_stride, ws, ws_bytes, stream, lse_sel,
+                                lse_s);
 }
 
 gqe_status gqe_attention_prefill_chunk(const gqe_dims* dims, int32_t T, const void* Q,
@@ -248,6 +264,106 @@ gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void
 }
 
 int64_t gqe_set_pair_threshold(int64_t kv_bytes) { return set_pair_threshold(kv_bytes); }
+
+// ------------------------------------------------------------ backward
+
+namespace {
+struct BwdLayout {
+  size_t dO_r, D_r, dO_s, D_s, total;
+};
+BwdLayout bwd_layout(const gqe_dims& d) {
+  BwdLayout L{};
+  const WsLayout W = make_ws_layout(d);
+  const int64_t T = static_cast<int64_t>(d.B) * d.S, R = T * d.G * d.k;
+  size_t off = W.total;
+  L.dO_r = off; off = align_up(off + sizeof(uint16_t) * R * d.d, 256);
+  L.D_r = off;  off = align_up(off + sizeof(float) * R, 256);
+  L.dO_s = off; off = align_up(off + sizeof(uint16_t) * T * d.d, 256);
+  L.D_s = off;  off = align_up(off + sizeof(float) * T, 256);
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+size_t gqe_prefill_backward_workspace_size(const gqe_dims* dims) {
+  if (check_dims(dims, false) != GQE_OK) return 0;
+  return bwd_layout(*dims).total;
+}
+
+gqe_status gqe_prefill_backward(const gqe_dims* dims, const void* Q, const void* Qs,
+                                const void* K, const void* V, const int32_t* topk_idx,
+                                const float* w, const float* O_sel, const float* s_out,
+                                int64_t out_row_stride, const float* lse_sel, const float* lse_s,
+                                const float* dO_sel, const float* do_bar, const float* ds,
+                                int64_t dout_row_stride, float* dQ, float* dQs, float* dK,
+                                float* dV, float* dw, void* ws, size_t ws_bytes, void* stream) {
+  gqe_status st = check_dims(dims, false);
+  if (st != GQE_OK) return st;
+  const void* ptrs[] = {Q, Qs, K, V, topk_idx, w, O_sel, s_out, lse_sel, lse_s, dO_sel, do_bar,
+                        ds, dQ, dQs, dK, dV, dw};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return GQE_ERR_INVALID_ARG;
+  if (out_row_stride < dims->d || out_row_stride % 4 != 0 || dout_row_stride < dims->d ||
+      dout_row_stride % 4 != 0)
+    return GQE_ERR_INVALID_ARG;
+  const WsLayout L = make_ws_layout(*dims);
+  const BwdLayout BL = bwd_layout(*dims);
+  if (!aligned16(ws) || ws_bytes < BL.total) return GQE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  BucketArgs ba = bucket_args(dims, topk_idx, reinterpret_cast<int32_t*>(wb + L.bucket_off),
+                              reinterpret_cast<int32_t*>(wb + L.bucket_tok), wb, L);
+  if (launch_prep(ba, nullptr, false, s) != cudaSuccess) return GQE_ERR_CUDA;
+  const int64_t T = static_cast<int64_t>(dims->B) * dims->S;
+  if (cudaMemsetAsync(dQ, 0, sizeof(float) * T * dims->N * dims->d, s) != cudaSuccess ||
+      cudaMemsetAsync(dQs, 0, sizeof(float) * T * dims->d, s) != cudaSuccess)
+    return GQE_ERR_CUDA;
+  BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if (!map_bshd(&a.tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, dims->B, dims->S, dims->G, dims->d) ||
+      !map_bshd(&a.tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, dims->B, dims->S, dims->G, dims->d))
+    return GQE_ERR_CUDA;
+  a.Q = static_cast<const uint16_t*>(Q);
+  a.Qs = static_cast<const uint16_t*>(Qs);
+  a.topk_idx = topk_idx;
+  a.w = w;
+  a.bucket_off = reinterpret_cast<const int32_t*>(wb + L.bucket_off);
+  a.bucket_tok = reinterpret_cast<const int32_t*>(wb + L.bucket_tok);
+  a.O_sel = O_sel;
+  a.s_out = s_out;
+  a.out_row_stride = out_row_stride;
+  a.lse_sel = lse_sel;
+  a.lse_s = lse_s;
+  a.dO_sel = dO_sel;
+  a.do_bar = do_bar;
+  a.ds = ds;
+  a.dout_row_stride = dout_row_stride;
+  a.dO_r_out = reinterpret_cast<uint16_t*>(wb + BL.dO_r);
+  a.dO_r = a.dO_r_out;
+  a.D_r_out = reinterpret_cast<float*>(wb + BL.D_r);
+  a.D_r = a.D_r_out;
+  a.dO_s_out = reinterpret_cast<uint16_t*>(wb + BL.dO_s);
+  a.dO_s = a.dO_s_out;
+  a.D_s_out = reinterpret_cast<float*>(wb + BL.D_s);
+  a.D_s = a.D_s_out;
+  a.dQ = dQ;
+  a.dQs = dQs;
+  a.dK = dK;
+  a.dV = dV;
+  a.dw = dw;
+  a.status = reinterpret_cast<int*>(wb + L.status);
+  a.B = dims->B;
+  a.S = dims->S;
+  a.N = dims->N;
+  a.G = dims->G;
+  a.M = dims->N / dims->G;
+  a.k = dims->k;
+  a.d = dims->d;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(dims->d)));
+  a.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(dims->d)));
+  a.wait_limit_ns = kWaitLimitNs;
+  return from_cuda(launch_bwd(a, s));
+}
 
 // ------------------------------------------------------------ projections
 

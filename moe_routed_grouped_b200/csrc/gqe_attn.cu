@@ -110,14 +110,23 @@ __device__ __forceinline__ void tile_load_s(uint32_t taddr, uint32_t (&sv)[4][32
 }
 
 // Key t is visible to a row at absolute position pos iff kvs <= t <= pos.
-__device__ __forceinline__ void tile_mask(uint32_t (&sv)[4][32], int kbase, int pos, int kvs) {
+// The causal part: columns past lim = pos - kbase are masked (one compare
+// with a constant column index per element).
+__device__ __forceinline__ void tile_mask_causal(uint32_t (&sv)[4][32], int lim) {
 #pragma unroll
   for (int c = 0; c < 4; ++c)
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int t = kbase + 32 * c + e;
-      if (t > pos || t < kvs) sv[c][e] = __float_as_uint(-INFINITY);
-    }
+    for (int e = 0; e < 32; ++e)
+      if (32 * c + e > lim) sv[c][e] = __float_as_uint(-INFINITY);
+}
+// The first-valid-slot part (left padding): columns before first are masked;
+// only the tile that holds kv_start needs it.
+__device__ __forceinline__ void tile_mask_below(uint32_t (&sv)[4][32], int first) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (32 * c + e < first) sv[c][e] = __float_as_uint(-INFINITY);
 }
 
 // Row maximum of the raw scores: 8 independent chains of 3-input max.
@@ -191,7 +200,8 @@ __device__ __forceinline__ bool softmax_tile(const SoftmaxCtx& x, const Waiter& 
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(x.s_free);  // S_j is in registers: S_{j+1} may start
-  if (diag) tile_mask(sv, kbase, pos, kvs);
+  if (diag) tile_mask_causal(sv, pos - kbase);
+  if (kbase < kvs) tile_mask_below(sv, kvs - kbase);
   float factor = 1.f;
   const float mnew = fmaxf(m_used, tile_max(sv) * sl2);  // j = 0: m_used = -inf, factor 0
   if (mnew - m_used > kRescaleThreshold) {
@@ -514,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
                         &bars[kBarODone], &bars[kBarPFull]};
     for (int j = 0; j < nkv; ++j) {
       const int kbase = (j0 + j) * kTileN;
-      const bool diag = kbase + kTileN - 1 > apos_first || kbase < kvs;
+      const bool diag = kbase + kTileN - 1 > apos_first;
       if (!softmax_tile<D, kPolyPairs>(sx, wait, j, diag, kbase, apos, kvs, sl2, m_used, l)) {
         ok = false;
         break;
@@ -542,7 +552,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
         if (a.k == 1)
           dst2 = static_cast<uint8_t*>(a.o_bar) +
                  (tokrow * a.out_row_stride + static_cast<int64_t>(g) * D) * esz;
+        if (a.lse_sel) a.lse_sel[(tokrow * G + g) * a.k + slot] = m_used + log2f(l);
       }
+      if (kind == kShared && a.lse_s) a.lse_s[tokrow] = m_used + log2f(l);
     }
     if (ok) {
       tc_fence_after();
@@ -858,7 +870,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (a.k == 1)
             dst2 = static_cast<uint8_t*>(a.o_bar) +
                    (tokrow * a.out_row_stride + static_cast<int64_t>(t.g) * D) * esz;
+          if (a.lse_sel) a.lse_sel[(tokrow * G + t.g) * a.k + slot] = m_used + log2f(l);
         }
+        if (t.kind == kShared && a.lse_s) a.lse_s[tokrow] = m_used + log2f(l);
       }
       if (ok) {
         tc_fence_after();

@@ -174,6 +174,8 @@ struct AttnArgs {
   const int32_t* q_off;     // chunked prefill (see seq_offsets); null: 0
   const int32_t* kv_start;  // null: 0
   int T;                    // KV slots per sequence (K/V maps are [B, T, G, d])
+  float* lse_sel;           // optional [B,S,G,k]: base-2 log-sum-exp of the scaled
+  float* lse_s;             //   scores per routed slot / shared row (for the backward)
   int dense;          // 1: dense GQA tiles from blockIdx; 0: routed/shared list
   int pair;           // 1: the pair kernel on a paired list (d = 64 only)
   float scale_log2;   // log2(e) / sqrt(d)
@@ -181,6 +183,50 @@ struct AttnArgs {
 };
 // n_list: length of the work list (routed/shared); unused for dense tiles.
 cudaError_t launch_attention(const AttnArgs& a, int64_t n_list, cudaStream_t st);
+
+// Backward of the routed prefill (gqe_bwd.cu).
+struct BwdArgs {
+  CUtensorMap tmK;          // bf16 K [B,S,G,d], box {64,1,128,1}
+  CUtensorMap tmV;          // bf16 V [B,S,G,d]
+  const uint16_t* Q;        // bf16 [B,S,N,d]
+  const uint16_t* Qs;       // bf16 [B,S,d]
+  const int32_t* topk_idx;  // [B,S,G,k]
+  const float* w;           // [B,S,G,k]
+  const int32_t* bucket_off;
+  const int32_t* bucket_tok;
+  // forward outputs (float32 concat rows at out_row_stride) and statistics
+  const float* O_sel;       // slot j of group g at (g*k + j)*d
+  const float* s_out;
+  int64_t out_row_stride;
+  const float* lse_sel;     // [B,S,G,k] base-2 log-sum-exp of the scaled scores
+  const float* lse_s;       // [B,S]
+  // upstream gradients (float32 rows at dout_row_stride, the concat layout)
+  const float* dO_sel;
+  const float* do_bar;
+  const float* ds;
+  int64_t dout_row_stride;
+  // workspace: effective dO of the slots and of the shared head, and D
+  uint16_t* dO_r_out;       // [B,S,G,k,d] bf16 (written by the prep kernel)
+  const uint16_t* dO_r;
+  float* D_r_out;           // [B,S,G,k]
+  const float* D_r;
+  uint16_t* dO_s_out;       // [B,S,d] bf16
+  const uint16_t* dO_s;
+  float* D_s_out;           // [B,S]
+  const float* D_s;
+  // gradients (float32): dQ and dQs accumulated atomically (zeroed first)
+  float* dQ;                // [B,S,N,d]
+  float* dQs;               // [B,S,d]
+  float* dK;                // [B,S,G,d]
+  float* dV;                // [B,S,G,d]
+  float* dw;                // [B,S,G,k]
+  int* status;
+  int B, S, N, G, M, k, d;
+  float scale_log2;         // log2(e) / sqrt(d)
+  float inv_sqrt_d;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t st);
 // K/V working-set size from which routed d = 64 calls use the pair kernel;
 // returns the previous value (negative: never).  pair_kernel_for() is the
 // decision for one call: taken once, then passed to the bucketing (list
