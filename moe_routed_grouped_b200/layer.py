@@ -143,6 +143,54 @@ class GqePrefill:
         return _lib.gqe_get_device_status(self.ws, 1 if clear else 0, stream)
 
 
+    # ---------------------------------------------------------- training
+    def forward_train(self, x, W_r, bias, Q, Qs, K, V, stream=None):
+        """forward() that also keeps each row's log-sum-exp (``lse_sel``
+        [B,S,G,k], ``lse_s`` [B,S]) for :meth:`backward`; float32 outputs."""
+        if self.out_dtype != torch.float32:
+            raise ValueError("training needs float32 outputs (out_fp32=True)")
+        self._check_qkv(Q, K, V, Qs)
+        self.route(x, W_r, bias, stream)
+        dv = self.device
+        if not hasattr(self, "lse_sel"):
+            self.lse_sel = torch.empty(self.B, self.S, self.G, self.k, dtype=torch.float32,
+                                       device=dv)
+            self.lse_s = torch.empty(self.B, self.S, dtype=torch.float32, device=dv)
+        a = self.G * self.k * self.d
+        flat = self.concat.view(-1)
+        _lib.gqe_attention_prefill_train(self.dims, Q, Qs, K, V, self.topk_idx, self.w,
+                                         self.concat, flat[a:], flat[a + self.G * self.d:],
+                                         self.row, self.lse_sel, self.lse_s, self.ws, stream)
+        self._saved = (Q, Qs, K, V)
+        return self.concat
+
+    def backward(self, dconcat, stream=None):
+        """Gradients for an upstream gradient of the concat buffer (float32
+        [B*S, row], the same layout): dict(dQ [B,S,N,d], dQs [B,S,d],
+        dK, dV [B,S,G,d], dw [B,S,G,k]), float32.  Uses the tensors of the
+        last forward_train()."""
+        Q, Qs, K, V = self._saved
+        dv = self.device
+        _expect(dconcat, "dconcat", (self.B * self.S, self.row), torch.float32, dv)
+        n = _lib.gqe_prefill_backward_workspace_size(self.dims)
+        if not hasattr(self, "_bws") or self._bws.numel() < n:
+            self._bws = torch.zeros(n, dtype=torch.uint8, device=dv)
+        B, S, N, G, k, d = self.B, self.S, self.N, self.G, self.k, self.d
+        f = torch.float32
+        out = dict(dQ=torch.empty(B, S, N, d, dtype=f, device=dv),
+                   dQs=torch.empty(B, S, d, dtype=f, device=dv),
+                   dK=torch.empty(B, S, G, d, dtype=f, device=dv),
+                   dV=torch.empty(B, S, G, d, dtype=f, device=dv),
+                   dw=torch.empty(B, S, G, k, dtype=f, device=dv))
+        a = G * k * d
+        cf, df = self.concat.view(-1), dconcat.view(-1)
+        _lib.gqe_prefill_backward(self.dims, Q, Qs, K, V, self.topk_idx, self.w, self.concat,
+                                  cf[a + G * d:], self.row, self.lse_sel, self.lse_s, dconcat,
+                                  df[a:], df[a + G * d:], self.row, out["dQ"], out["dQs"],
+                                  out["dK"], out["dV"], out["dw"], self._bws, stream)
+        return out
+
+
 class GqeChunk:
     """Buffers and calls for chunked prefill: S new tokens per sequence over
     KV caches of T slots (gqe_route on the chunk, then
@@ -308,54 +356,6 @@ class GqeDecode:
 
     def device_status(self, clear=True, stream=None) -> int:
         return _lib.gqe_get_device_status(self.ws, 1 if clear else 0, stream)
-
-    # ---------------------------------------------------------- training
-    def forward_train(self, x, W_r, bias, Q, Qs, K, V, stream=None):
-        """forward() that also keeps each row's log-sum-exp (``lse_sel``
-        [B,S,G,k], ``lse_s`` [B,S]) for :meth:`backward`; float32 outputs."""
-        if self.out_dtype != torch.float32:
-            raise ValueError("training needs float32 outputs (out_fp32=True)")
-        self._check_qkv(Q, K, V, Qs)
-        self.route(x, W_r, bias, stream)
-        dv = self.device
-        if not hasattr(self, "lse_sel"):
-            self.lse_sel = torch.empty(self.B, self.S, self.G, self.k, dtype=torch.float32,
-                                       device=dv)
-            self.lse_s = torch.empty(self.B, self.S, dtype=torch.float32, device=dv)
-        a = self.G * self.k * self.d
-        flat = self.concat.view(-1)
-        _lib.gqe_attention_prefill_train(self.dims, Q, Qs, K, V, self.topk_idx, self.w,
-                                         self.concat, flat[a:], flat[a + self.G * self.d:],
-                                         self.row, self.lse_sel, self.lse_s, self.ws, stream)
-        self._saved = (Q, Qs, K, V)
-        return self.concat
-
-    def backward(self, dconcat, stream=None):
-        """Gradients for an upstream gradient of the concat buffer (float32
-        [B*S, row], the same layout): dict(dQ [B,S,N,d], dQs [B,S,d],
-        dK, dV [B,S,G,d], dw [B,S,G,k]), float32.  Uses the tensors of the
-        last forward_train()."""
-        Q, Qs, K, V = self._saved
-        dv = self.device
-        _expect(dconcat, "dconcat", (self.B * self.S, self.row), torch.float32, dv)
-        n = _lib.gqe_prefill_backward_workspace_size(self.dims)
-        if not hasattr(self, "_bws") or self._bws.numel() < n:
-            self._bws = torch.zeros(n, dtype=torch.uint8, device=dv)
-        B, S, N, G, k, d = self.B, self.S, self.N, self.G, self.k, self.d
-        f = torch.float32
-        out = dict(dQ=torch.empty(B, S, N, d, dtype=f, device=dv),
-                   dQs=torch.empty(B, S, d, dtype=f, device=dv),
-                   dK=torch.empty(B, S, G, d, dtype=f, device=dv),
-                   dV=torch.empty(B, S, G, d, dtype=f, device=dv),
-                   dw=torch.empty(B, S, G, k, dtype=f, device=dv))
-        a = G * k * d
-        cf, df = self.concat.view(-1), dconcat.view(-1)
-        _lib.gqe_prefill_backward(self.dims, Q, Qs, K, V, self.topk_idx, self.w, self.concat,
-                                  cf[a + G * d:], self.row, self.lse_sel, self.lse_s, dconcat,
-                                  df[a:], df[a + G * d:], self.row, out["dQ"], out["dQs"],
-                                  out["dK"], out["dV"], out["dw"], self._bws, stream)
-        return out
-
 
 class GqeLayer:
     """Buffers and calls for the whole GQE attention layer of one shape,

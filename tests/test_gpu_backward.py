@@ -11,7 +11,7 @@ Tolerance, from the arithmetic: the tensor-core products take bf16 operands,
 so the effective dO, P and dS are each rounded to bf16 (relative error at
 most 2^-9 each, float32 accumulation); the gradients are held to 1e-2
 relative L2 and 2e-2 of their largest magnitude elementwise.  dw is a float32
-dot product of float32 values: 1e-4.
+dot product with the forward's output o_j, so it carries the forward's 1e-3.
 """
 import numpy as np
 import pytest
@@ -58,8 +58,10 @@ def test_backward_matches_oracle(shape):
         got = grads[name].cpu().numpy()
         r = ref[name]
         check_close(got, r, name, atol=2e-2 * float(np.abs(r).max()), rtol_l2=1e-2)
-    check_close(grads["dw"].cpu().numpy(), ref["dw"], "dw", atol=1e-4 * float(np.abs(ref["dw"]).max()) + 1e-6,
-                rtol_l2=1e-4)
+    # dw = <d(o_bar), o_j> reads the forward's o_j, so it carries the forward
+    # output's tolerance (relative L2 1e-3)
+    check_close(grads["dw"].cpu().numpy(), ref["dw"], "dw",
+                atol=1e-3 * float(np.abs(ref["dw"]).max()) + 1e-6, rtol_l2=1e-3)
 
 
 def test_backward_zero_upstream_gives_zero_gradients():
