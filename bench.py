@@ -483,6 +483,90 @@ def layer_entry(torch, device, local, flush, peaks, peak_src, steps=20, warmup=3
             "gpu_launches": steps * (10 + 6 + 1)}
 
 
+def backward_entry(torch, device, local, flush, peaks, peak_src, steps=10, warmup=3):
+    """The training step of the path at the bench shape: the forward that keeps
+    each row's log-sum-exp (gqe_attention_prefill_train) and the backward pass
+    (gqe_prefill_backward), timed separately.  Useful backward work: 5 products
+    of 2d flop per visible (query, key) pair and active head (S, dP, dV, dK,
+    dQ)."""
+    from moe_routed_grouped_b200.layer import GqePrefill
+    w = WORKLOADS["layer250m"]
+    dev, _ = gpu_inputs(torch, w, device, 0, False)
+    L = GqePrefill(w.B, w.S, w.N, w.G, w.k, w.d, w.d_model, out_fp32=True, device=device)
+    g = torch.Generator(device=device)
+    g.manual_seed(9300)
+    dcat = torch.randn(w.B * w.S, L.row, generator=g, device=device)
+    fwd = lambda: L.forward_train(dev["x"], dev["W_r"], dev["bias"], dev["Q"], dev["Qs"],  # noqa: E731
+                                  dev["K"], dev["V"])
+    cs = ClockSampler(local)
+    cs.start()
+    try:
+        f_ms, _, t0, _ = timed_loop(torch, fwd, steps, warmup, flush)
+        fwd()
+        b_ms, _, _, t1 = timed_loop(torch, lambda: L.backward(dcat), steps, warmup, flush)
+    finally:
+        cs.stop()
+    if L.device_status() != 0:
+        raise RuntimeError("device status after the backward loop")
+    pairs = (w.G * w.k + 1) * w.B * w.S * (w.S + 1) / 2.0
+    bwd_flop = pairs * 5 * 2 * w.d
+    fm, bm = statistics.mean(f_ms), statistics.mean(b_ms)
+    tf = bwd_flop / (bm / 1e3) / 1e12
+    return {"workload": "layer250m", "steps": steps, "warmup": warmup,
+            "forward_train_ms": fm, "backward_ms": bm,
+            "backward_tokens_per_s": w.B * w.S / (bm / 1e3),
+            "backward_useful_tflops": tf, "backward_frac_of_peak": tf / peaks["bf16_tflops"],
+            "backward_flop": bwd_flop,
+            "flop_definition": "5 products x 2d flop per visible (query, key) pair, G*k+1 heads",
+            "peak_source": f"{peak_src} bf16 dense (burst)",
+            "clocks": cs.summary(t0, t1),
+            # forward: route_prep, route, prep, attention; backward: bucket prep,
+            # 2 memsets (not kernels of this library), bwd prep, bwd
+            "gpu_launches": steps * 4 + steps * 3}
+
+
+def chunk_entry(torch, device, local, flush, peaks, peak_src, steps=5, warmup=3, chunk=4096):
+    """Chunked prefill (gqe_attention_prefill_chunk): the 32k biased workload
+    processed as S / chunk chunks over a full KV cache, each chunk's queries at
+    their absolute positions, against the one-shot prefill of the same
+    sequence.  Same useful work; the difference is the chunks' extra work
+    (each chunk re-reads the cache prefix) and launch overhead."""
+    from moe_routed_grouped_b200.layer import GqeChunk, GqePrefill
+    w = WORKLOADS["imbalanced32k"]
+    dev, _ = gpu_inputs(torch, w, device, 0, False)
+    n = w.S // chunk
+    C = GqeChunk(w.B, chunk, w.S, w.N, w.G, w.k, w.d, w.d_model, device=device)
+    P = GqePrefill(w.B, w.S, w.N, w.G, w.k, w.d, w.d_model, device=device)
+    P.route(dev["x"], dev["W_r"], dev["bias"])
+    offs = [torch.tensor([i * chunk], dtype=torch.int32, device=device) for i in range(n)]
+    parts = [{k: dev[k][:, i * chunk:(i + 1) * chunk].contiguous() for k in ("x", "Q", "Qs")}
+             for i in range(n)]
+
+    def chunked():
+        for i in range(n):
+            C.forward(parts[i]["x"], dev["W_r"], dev["bias"], parts[i]["Q"], parts[i]["Qs"],
+                      dev["K"], dev["V"], offs[i])
+    cs = ClockSampler(local)
+    cs.start()
+    try:
+        c_ms, _, t0, _ = timed_loop(torch, chunked, steps, warmup, flush)
+        o_ms, _, _, t1 = timed_loop(torch, lambda: P.attention(dev["Q"], dev["Qs"], dev["K"],
+                                                               dev["V"]), steps, warmup, flush)
+    finally:
+        cs.stop()
+    if C.device_status() != 0 or P.device_status() != 0:
+        raise RuntimeError("device status after the chunk loop")
+    cm, om = statistics.mean(c_ms), statistics.mean(o_ms)
+    fl = w.useful_flop_routed()
+    return {"workload": "imbalanced32k", "chunk": chunk, "chunks": n, "steps": steps,
+            "warmup": warmup, "chunked_ms": cm, "one_shot_attention_ms": om,
+            "chunked_tokens_per_s": w.B * w.S / (cm / 1e3),
+            "chunked_useful_tflops": fl / (cm / 1e3) / 1e12,
+            "chunked_over_one_shot": om / cm,
+            "note": "chunked includes the router per chunk; one-shot is the attention call alone",
+            "clocks": cs.summary(t0, t1), "gpu_launches": steps * n * 5 + steps * 2}
+
+
 # the long-context workloads every default line also measures: (name, timed steps)
 CONFIG_ENTRIES = (("imbalanced32k", 10), ("wide131k", 5), ("million", 3))
 
@@ -790,12 +874,15 @@ def main():
     }
 
     if world == 1 and not args.no_configs:
-        try:
-            line["layer"] = layer_entry(torch, device, local, flush, peaks, peak_src)
-            line["gpu_launches"] += line["layer"]["gpu_launches"]
-        except Exception as ex:  # noqa: BLE001  (reported in the entry, not hidden)
-            line["layer"] = {"workload": "layer250m", "error": f"{type(ex).__name__}: {ex}"[:300]}
-        torch.cuda.empty_cache()
+        for key, fn, wl in (("layer", layer_entry, "layer250m"),
+                            ("backward", backward_entry, "layer250m"),
+                            ("chunked", chunk_entry, "imbalanced32k")):
+            try:
+                line[key] = fn(torch, device, local, flush, peaks, peak_src)
+                line["gpu_launches"] += line[key]["gpu_launches"]
+            except Exception as ex:  # noqa: BLE001  (reported in the entry, not hidden)
+                line[key] = {"workload": wl, "error": f"{type(ex).__name__}: {ex}"[:300]}
+            torch.cuda.empty_cache()
         # the S >= 32k workloads, each with its own timing and clock record
         del res
         torch.cuda.empty_cache()
