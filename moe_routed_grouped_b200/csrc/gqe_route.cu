@@ -22,6 +22,7 @@ namespace {
 constexpr int kRouteWarps = 4;
 constexpr int kRouteThreads = 32 * kRouteWarps;
 constexpr int kRouteChunk = 32;     // d_model rows per chunk; warp w owns chunks w, w+4, ...
+constexpr int kRouteMaxWarps = 4;   // warps that take exact ranks (sizes their shared arrays)
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
   return __uint_as_float(b << 16);
@@ -102,6 +103,135 @@ __device__ __forceinline__ void load_wt_chunk(const float* wt, int c0, int rows,
   }
 }
 
+// Softmax, provisional top-k and certification of one (token, group) pair
+// with at most MM experts, every per-expert value in registers (loops over
+// MM with compile-time indices).  p = e^(l - max) / s is formed as
+// e^(l - max) * (1/s); w renormalises the selected p.  Returns whether every
+// rank beats every later candidate by more than the two error bounds.
+template <int MM>
+__device__ __noinline__ bool decide_pair_small(const float* l, const float* e, int M, int k,
+                                                  float* prow, int32_t* irow, float* wrow) {
+  float lv[MM], ev[MM], xv[MM];
+#pragma unroll
+  for (int m = 0; m < MM; ++m) {
+    lv[m] = m < M ? l[m] : -INFINITY;
+    ev[m] = m < M ? e[m] : 0.f;
+  }
+  float mx = lv[0];
+#pragma unroll
+  for (int m = 1; m < MM; ++m)
+    if (m < M) mx = fmaxf(mx, lv[m]);
+  float s = 0.f;
+#pragma unroll
+  for (int m = 0; m < MM; ++m)
+    if (m < M) {
+      xv[m] = expf(lv[m] - mx);
+      s += xv[m];
+    }
+  const float inv = 1.0f / s;
+#pragma unroll
+  for (int m = 0; m < MM; ++m)
+    if (m < M) {
+      xv[m] *= inv;
+      prow[m] = xv[m];
+    }
+  uint32_t taken = 0;
+  bool certain = true;
+  float den = 0.f, pr[MM];
+#pragma unroll
+  for (int r = 0; r < MM; ++r) {
+    if (r >= k) break;
+    int best = -1;
+    float bl = 0.f, be = 0.f, bp = 0.f;
+#pragma unroll
+    for (int m = 0; m < MM; ++m)
+      if (m < M && !(taken & (1u << m)) && (best < 0 || lv[m] > bl)) {
+        best = m;
+        bl = lv[m];
+        be = ev[m];
+        bp = xv[m];
+      }
+    taken |= 1u << best;
+    irow[r] = best;
+    pr[r] = bp;
+    den += bp;
+    // rank r must beat every later candidate by more than both bounds
+#pragma unroll
+    for (int m = 0; m < MM; ++m)
+      if (m < M && !(taken & (1u << m)) && !(bl - lv[m] > (be + ev[m]) * 1.001f)) certain = false;
+  }
+#pragma unroll
+  for (int r = 0; r < MM; ++r)
+    if (r < k) wrow[r] = (k == 1) ? 1.0f : pr[r] / den;
+  return certain;
+}
+
+// The same for any M <= kMaxM, reading the values from shared memory.
+__device__ __noinline__ bool decide_pair_any(const float* l, const float* e, int M, int k,
+                                                float* prow, int32_t* irow, float* wrow) {
+  float mx = l[0];
+  for (int m = 1; m < M; ++m) mx = fmaxf(mx, l[m]);
+  float s = 0.f;
+  for (int m = 0; m < M; ++m) s += expf(l[m] - mx);
+  const float inv = 1.0f / s;
+  for (int m = 0; m < M; ++m) prow[m] = expf(l[m] - mx) * inv;
+  uint32_t taken = 0;
+  bool certain = true;
+  float den = 0.f;
+  for (int r = 0; r < k; ++r) {
+    int best = -1;
+    for (int m = 0; m < M; ++m) {
+      if (taken & (1u << m)) continue;
+      if (best < 0 || l[m] > l[best]) best = m;
+    }
+    taken |= 1u << best;
+    irow[r] = best;
+    den += expf(l[best] - mx) * inv;
+    if (r < M - 1)
+      for (int m = 0; m < M; ++m)
+        if (!(taken & (1u << m)) && !(l[best] - l[m] > (e[best] + e[m]) * 1.001f))
+          certain = false;
+  }
+  for (int r = 0; r < k; ++r)
+    wrow[r] = (k == 1) ? 1.0f : (expf(l[irow[r]] - mx) * inv) / den;
+  return certain;
+}
+
+// The steps after the logits, for one tile of ntok tokens starting at t0:
+// per (token, group) the softmax, the provisional top-k and its certification
+// against the bounds err, then the exact ranks of the undecided pairs (one
+// warp per pair).  lgt and err have row stride GM + 1; every thread of the
+// CTA calls this.
+template <int GM>
+__device__ __forceinline__ void route_tile_epilogue(const RouteArgs& a, const float* lgt,
+                                                    const float* err, int t0, int ntok,
+                                                    int* nflag, int* flags, int (*sel)[kMaxM]) {
+  const int tid = threadIdx.x, warp = tid >> 5, nthreads = blockDim.x;
+  const int M = a.M, G = a.G, k = a.k;
+  for (int q = tid; q < ntok * G; q += nthreads) {
+    const int ql = q / G, g = q % G;
+    const float* l = lgt + ql * (GM + 1) + g * M;
+    const float* e = err + ql * (GM + 1) + g * M;
+    const int64_t row = static_cast<int64_t>(t0 + ql) * G + g;
+    float* prow = a.p + row * M;
+    int32_t* irow = a.topk_idx + row * k;
+    float* wrow = a.w + row * k;
+    const bool certain = M <= 8 ? decide_pair_small<(GM < 8 ? GM : 8)>(l, e, M, k, prow, irow, wrow)
+                                : decide_pair_any(l, e, M, k, prow, irow, wrow);
+    if (!certain) flags[atomicAdd(nflag, 1)] = q;
+  }
+  __syncthreads();
+  const int nf = *nflag;
+  if (nf > 0) {  // undecided pairs: exact ranks, one warp per pair (at most kRouteMaxWarps)
+    if (tid == 0) atomicAdd(a.fix_count, nf);
+    const int nw = min(nthreads / 32, kRouteMaxWarps);
+    for (int f = warp; warp < nw && f < nf; f += nw) {
+      const int q = flags[f];
+      exact_rank_pair(a, t0 + q / G, q % G, sel[warp]);
+    }
+  }
+}
+
 // Persistent CTAs of 4 warps; a tile is a.tok <= kTok tokens (sized so the
 // tiles fill the SMs evenly; lane l takes tokens l and l + 32).  Warp w sums the
 // products of the d_model chunks w, w+4, ... ; lane l keeps its tokens' x
@@ -113,14 +243,14 @@ __device__ __forceinline__ void load_wt_chunk(const float* wt, int c0, int rows,
 // rounding chain is 32 + ceil(n_chunks/4) + 4 (with the bias): that is the D
 // of the bound |l_hat - l| <= D u ||x|| ||w_c||, u = 2^-24.
 template <int GM>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
+__global__ void __launch_bounds__(kRouteThreads, 3) route_kernel(const RouteArgs a) {
   using Sh = RouteShape<GM>;
   constexpr int TPL = Sh::kTPL;
   const int TOK = a.tok;
   extern __shared__ __align__(16) uint8_t route_smem_raw[];
   RouteSmem<GM>& sm = *reinterpret_cast<RouteSmem<GM>*>(route_smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int dm = a.dm, M = a.M, G = a.G, k = a.k;
+  const int dm = a.dm;
   const int nchunks = (dm + kRouteChunk - 1) / kRouteChunk;
   const int ntiles = (a.T + TOK - 1) / TOK;
   const float cerr =
@@ -236,53 +366,279 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     if (nonfinite) latch_status(a.status, GQE_ERR_NONFINITE);
     __syncthreads();
 
-    // per (token, group): softmax, provisional top-k, certification
-    for (int q = tid; q < ntok * G; q += kRouteThreads) {
-      const int ql = q / G, g = q % G;
-      const float* l = &sm.lgt[ql][g * M];
-      const float* e = &sm.err[ql][g * M];
-      const int64_t row = static_cast<int64_t>(t0 + ql) * G + g;
-      float mx = l[0];
-      for (int m = 1; m < M; ++m) mx = fmaxf(mx, l[m]);
-      float s = 0.f;
-      for (int m = 0; m < M; ++m) s += expf(l[m] - mx);
-      float* prow = a.p + row * M;
-      for (int m = 0; m < M; ++m) prow[m] = expf(l[m] - mx) / s;
-      int32_t* irow = a.topk_idx + row * k;
-      uint32_t taken = 0;
-      bool certain = true;
-      float den = 0.f;
-      for (int r = 0; r < k; ++r) {
-        int best = -1;
-        for (int m = 0; m < M; ++m) {
-          if (taken & (1u << m)) continue;
-          if (best < 0 || l[m] > l[best]) best = m;
-        }
-        taken |= 1u << best;
-        irow[r] = best;
-        den += expf(l[best] - mx) / s;
-        // rank r must beat every later candidate by more than both bounds
-        if (r < M - 1)
-          for (int m = 0; m < M; ++m)
-            if (!(taken & (1u << m)) && !(l[best] - l[m] > (e[best] + e[m]) * 1.001f))
-              certain = false;
-      }
-      float* wrow = a.w + row * k;
-      for (int r = 0; r < k; ++r)
-        wrow[r] = (k == 1) ? 1.0f : (expf(l[irow[r]] - mx) / s) / den;
-      if (!certain) sm.flags[atomicAdd(&sm.nflag, 1)] = q;
-    }
-    __syncthreads();
-    const int nf = sm.nflag;
-    if (nf > 0) {  // undecided pairs: exact ranks, one warp per pair
-      if (tid == 0) atomicAdd(a.fix_count, nf);
-      for (int f = warp; f < nf; f += kRouteWarps) {
-        const int q = sm.flags[f];
-        exact_rank_pair(a, t0 + q / G, q % G, sm.sel[warp]);
-      }
-    }
+    route_tile_epilogue<GM>(a, &sm.lgt[0][0], &sm.err[0][0], t0, ntok, &sm.nflag, sm.flags,
+                            sm.sel);
     __syncthreads();
   }
+}
+
+// ------------------------------------------------------------------------
+// Router with W_r resident in shared memory (d_model * G * M float32 within
+// kWresMaxW): one persistent CTA of 16 warps per SM over tiles of 64
+// consecutive tokens.  Lane l of warp (cg, ks) takes tokens l and l + 32 of
+// the tile, the CPW columns of column group cg and rows [ks*dm/KS,
+// (ks+1)*dm/KS) of d_model (a K slice): every W_r load of a warp is one
+// broadcast address, and each loaded W_r value serves two tokens (a 16-byte
+// shared-memory load per 32 lanes returns 512 bytes, so the loads, not the
+// FMAs, would bound a one-token lane).
+//
+// x streams per warp: each warp copies its own slice of the coming tiles into
+// a ring of kWresRing groups of 8 values x 64 tokens with cp.async, waiting
+// only for its own copies, so the copies run ahead across tile boundaries.
+//
+// Each step takes a pair of rows (2p, 2p+1): one f32x2 FMA per column and
+// token adds x[2p] w[2p][c] to the even half and x[2p+1] w[2p+1][c] to the
+// odd half of the accumulator, with W_r stored as (w[2p][c], w[2p+1][c])
+// pairs (one 16-byte load gives two columns; laid out by route_pairs_kernel).
+// The halves are added, the K slices are added in slice order, then the
+// bias: the longest rounding chain is D = dm/(2 KS) + 1 + (KS - 1) + 1, the
+// D of the bound |l_hat - l| <= D u ||x|| ||w_c|| used to certify each
+// decision, as in route_kernel; the steps after the logits are
+// route_tile_epilogue's.
+constexpr int kWresWarps = 16;
+constexpr int kWresThreads = 32 * kWresWarps;
+constexpr int kWresTok = 64;                   // tokens per tile (two per lane)
+constexpr int kWresRing = 4;                   // x groups in flight per warp
+constexpr int kWresMaxW = 64 << 10;            // most bytes of float32 W_r
+constexpr int kWresMaxSmem = 215 << 10;        // most dynamic shared memory
+
+template <int GM>
+struct WresShape {
+  static constexpr int CPW = GM < 16 ? GM : 16;  // columns per warp
+  static constexpr int CGW = GM / CPW;           // column groups
+  static constexpr int KS = kWresWarps / CGW;    // K slices
+};
+
+template <int GM>
+struct WresFixed {
+  using Sh = WresShape<GM>;
+  uint16_t ring[kWresWarps][kWresRing][kWresTok * 8];  // x groups: [token][8 values]
+  float xsqp[Sh::KS][kWresTok];                        // per-slice sums of x^2
+  float lgt[kWresTok][GM + 1];
+  float err[kWresTok][GM + 1];
+  float wsqp[kWresWarps][GM];                          // per-warp column sums of squares
+  float wnorm[GM];
+  float bias[GM];
+  uint64_t wbar;                                       // the W_r copy
+  int nflag;
+  int flags[kWresTok * GM];
+  int sel[kRouteMaxWarps][kMaxM];
+};
+
+__host__ __device__ constexpr size_t align128(size_t x) { return (x + 127) / 128 * 128; }
+
+// Dynamic shared memory: W_r as [dm/2][GM] float pairs, the per-slice
+// partial logits part[KS][64][GM+1], then the fixed part.
+template <int GM>
+struct WresLayout {
+  size_t part, fixed, total;
+  __host__ __device__ explicit WresLayout(int dm) {
+    part = align128(static_cast<size_t>(dm) * GM * 4);
+    fixed = align128(part + sizeof(float) * WresShape<GM>::KS * kWresTok * (GM + 1));
+    total = fixed + sizeof(WresFixed<GM>);
+  }
+};
+
+// W_r [G][dm][M] bf16 -> float32 pairs: 16-byte unit d holds rows 2p, 2p+1
+// of columns c, c+1 (p = d / (GM/2), c = 2 (d % (GM/2))).
+template <int GM>
+__global__ void __launch_bounds__(256) route_pairs_kernel(const RouteArgs a) {
+  const int d = blockIdx.x * 256 + threadIdx.x;
+  if (d >= a.dm * GM / 4) return;
+  const int dm = a.dm, M = a.M;
+  const int p = d / (GM / 2), c = 2 * (d % (GM / 2));
+  const int g0 = c / M, m0 = c % M, g1 = (c + 1) / M, m1 = (c + 1) % M;
+  const uint16_t* w0 = a.Wr + (static_cast<int64_t>(g0) * dm + 2 * p) * M + m0;
+  const uint16_t* w1 = a.Wr + (static_cast<int64_t>(g1) * dm + 2 * p) * M + m1;
+  reinterpret_cast<float4*>(a.wt)[d] =
+      make_float4(bf16_bits_to_float(w0[0]), bf16_bits_to_float(w0[M]), bf16_bits_to_float(w1[0]),
+                  bf16_bits_to_float(w1[M]));
+}
+
+template <int GM>
+__global__ void __launch_bounds__(kWresThreads, 1) route_wres_kernel(const RouteArgs a) {
+  using Sh = WresShape<GM>;
+  constexpr int CPW = Sh::CPW, CGW = Sh::CGW, KS = Sh::KS;
+  extern __shared__ __align__(128) uint8_t wres_smem_raw[];
+  const int dm = a.dm;
+  const WresLayout<GM> lay(dm);
+  WresFixed<GM>& sm = *reinterpret_cast<WresFixed<GM>*>(wres_smem_raw + lay.fixed);
+  const float2* Ws = reinterpret_cast<const float2*>(wres_smem_raw);
+  float* part = reinterpret_cast<float*>(wres_smem_raw + lay.part);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cg = warp % CGW, ks = warp / CGW;
+  const int slice = dm / KS;                 // values of d_model per K slice
+  const int nq = slice / 8;                  // 8-value groups per slice
+  const float cerr = static_cast<float>(slice / 2 + KS + 1) * 5.9604645e-8f * 1.01f;
+  const int ntiles = (a.T + kWresTok - 1) / kWresTok;
+  const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+  // W_r pairs by one bulk copy
+  const uint32_t wbytes = static_cast<uint32_t>(dm) * GM * 4;
+  if (tid == 0) {
+    mbar_init(&sm.wbar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {  // in 4 KB pieces, each CTA starting at a different one
+    mbar_arrive_expect_tx(&sm.wbar, wbytes);
+    const uint32_t npc = (wbytes + 4095) / 4096;
+    for (uint32_t i = 0; i < npc; ++i) {
+      const uint32_t pc = (i + blockIdx.x) % npc, off = pc * 4096;
+      const uint32_t len = wbytes - off < 4096 ? wbytes - off : 4096;
+      bulk_load(wres_smem_raw + off, reinterpret_cast<const uint8_t*>(a.wt) + off, len, &sm.wbar);
+    }
+  }
+
+  // this warp's x groups, in the order it reduces them: groups 0..nq-1 of
+  // tile blockIdx.x, then of tile blockIdx.x + gridDim.x, ...; lane l copies
+  // tokens l and l + 32 of a group into ring slot (group number) % kWresRing
+  uint16_t (*ring)[kWresTok * 8] = sm.ring[warp];
+  int f_tile = blockIdx.x, f_q = 0, f_slot = 0;
+  auto fetch = [&]() {
+    if (f_tile < ntiles) {
+      const int e = ks * slice + 8 * f_q;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = f_tile * kWresTok + lane + 32 * h;
+        const bool in = t < a.T;
+        cp_async_16(&ring[f_slot][(lane + 32 * h) * 8],
+                    a.x + static_cast<int64_t>(in ? t : 0) * dm + e, in ? 16u : 0u);
+      }
+      if (++f_q == nq) {
+        f_q = 0;
+        f_tile += gridDim.x;
+      }
+    }
+    cp_async_commit();
+    f_slot = f_slot + 1 == kWresRing ? 0 : f_slot + 1;
+  };
+#pragma unroll
+  for (int i = 0; i < kWresRing - 1; ++i) fetch();
+
+  for (int c = tid; c < GM; c += kWresThreads) sm.bias[c] = a.bias ? a.bias[c] : 0.f;
+  const bool wok = mbar_wait(&sm.wbar, 0, nullptr, a.status, kWaitLimitNs);
+  if (__syncthreads_or(!wok)) {  // let this thread's copies land, then stop
+    cp_async_wait_all();
+    return;
+  }
+  // column norms: the lanes of a warp with the same column pair add their
+  // row pairs (rows 2p, 2p+1 with p = warp-and-lane order), then the warps in order
+  {
+    const float4* Wv = reinterpret_cast<const float4*>(Ws);
+    const int c = 2 * (tid % (GM / 2));
+    float s0 = 0.f, s1 = 0.f;
+    for (int d = tid; d < dm * GM / 4; d += kWresThreads) {
+      const float4 f = Wv[d];
+      s0 = fmaf(f.x, f.x, s0);
+      s0 = fmaf(f.y, f.y, s0);
+      s1 = fmaf(f.z, f.z, s1);
+      s1 = fmaf(f.w, f.w, s1);
+    }
+#pragma unroll
+    for (int off = GM / 2; off < 32; off <<= 1) {
+      s0 += __shfl_xor_sync(0xFFFFFFFFu, s0, off);
+      s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, off);
+    }
+    if (lane < GM / 2) {
+      sm.wsqp[warp][c] = s0;
+      sm.wsqp[warp][c + 1] = s1;
+    }
+  }
+  __syncthreads();
+  for (int c = tid; c < GM; c += kWresThreads) {
+    float s2 = 0.f;
+    for (int r = 0; r < kWresWarps; ++r) s2 += sm.wsqp[r][c];
+    sm.wnorm[c] = sqrtf(s2);
+  }
+
+  // this warp's W_r pairs start at row pair ks*slice/2, column cg*CPW
+  const float4* wbase =
+      reinterpret_cast<const float4*>(Ws + static_cast<int64_t>(ks) * (slice / 2) * GM + cg * CPW);
+  int slot = 0;  // ring slot of this warp's next group
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int t0 = tile * kWresTok;
+    const int ntok = min(kWresTok, a.T - t0);
+    if (tid == 0) sm.nflag = 0;
+    uint64_t acc[2][CPW];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int c = 0; c < CPW; ++c) acc[h][c] = 0;  // the bits of (+0, +0)
+    uint64_t xq[2] = {0, 0};
+    const float4* wr = wbase;
+#pragma unroll 1
+    for (int q = 0; q < nq; ++q) {
+      fetch();
+      cp_async_wait_group<kWresRing - 1>();  // this lane's copies of the group have landed
+      __syncwarp();
+      const uint32_t* g32 = reinterpret_cast<const uint32_t*>(ring[slot]);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        // (x[2p], x[2p+1]) of the two tokens: the halves of one 32-bit word
+        const uint32_t wa = g32[lane * 4 + r], wb = g32[(lane + 32) * 4 + r];
+        const uint64_t x0 = f2_pack(__uint_as_float(wa << 16), __uint_as_float(wa & 0xFFFF0000u));
+        const uint64_t x1 = f2_pack(__uint_as_float(wb << 16), __uint_as_float(wb & 0xFFFF0000u));
+#pragma unroll
+        for (int c2 = 0; c2 < CPW / 2; ++c2) {
+          const float4 w4 = wr[c2];
+          const uint64_t wlo = f2_pack(w4.x, w4.y), whi = f2_pack(w4.z, w4.w);
+          acc[0][2 * c2] = f2_fma(x0, wlo, acc[0][2 * c2]);
+          acc[0][2 * c2 + 1] = f2_fma(x0, whi, acc[0][2 * c2 + 1]);
+          acc[1][2 * c2] = f2_fma(x1, wlo, acc[1][2 * c2]);
+          acc[1][2 * c2 + 1] = f2_fma(x1, whi, acc[1][2 * c2 + 1]);
+          if (c2 % 4 == 3) asm volatile("" ::: "memory");  // at most 4 loads ahead
+        }
+        if (cg == 0) {
+          xq[0] = f2_fma(x0, x0, xq[0]);
+          xq[1] = f2_fma(x1, x1, xq[1]);
+        }
+        wr += GM / 2;
+        // keep the next row pair's loads below this one's FMAs (registers)
+        asm volatile("" ::: "memory");
+      }
+      __syncwarp();  // the ring slot is read before a later fetch overwrites it
+      slot = slot + 1 == kWresRing ? 0 : slot + 1;
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int c = 0; c < CPW; ++c) {
+        float lo, hi;
+        f2_unpack(acc[h][c], lo, hi);
+        part[(ks * kWresTok + lane + 32 * h) * (GM + 1) + cg * CPW + c] = lo + hi;
+      }
+      if (cg == 0) {
+        float lo, hi;
+        f2_unpack(xq[h], lo, hi);
+        sm.xsqp[ks][lane + 32 * h] = lo + hi;
+      }
+    }
+    __syncthreads();
+
+    // logits (slice sums in slice order, then the bias) and their bounds
+    bool nonfinite = false;
+    for (int qq = tid; qq < ntok * GM; qq += kWresThreads) {
+      const int ql = qq / GM, col = qq % GM;
+      const float bv = sm.bias[col];
+      float l = part[ql * (GM + 1) + col], x2 = sm.xsqp[0][ql];
+#pragma unroll
+      for (int w = 1; w < KS; ++w) {
+        l += part[(w * kWresTok + ql) * (GM + 1) + col];
+        x2 += sm.xsqp[w][ql];
+      }
+      l += bv;
+      sm.lgt[ql][col] = l;
+      sm.err[ql][col] = cerr * fmaf(sqrtf(x2), sm.wnorm[col], fabsf(bv)) + 1e-36f;
+      nonfinite |= !isfinite(l);
+    }
+    if (nonfinite) latch_status(a.status, GQE_ERR_NONFINITE);
+    __syncthreads();
+    route_tile_epilogue<GM>(a, &sm.lgt[0][0], &sm.err[0][0], t0, ntok, &sm.nflag, sm.flags,
+                            sm.sel);
+    __syncthreads();
+  }
+  cp_async_wait_all();  // the empty trailing groups
 }
 
 // ------------------------------------------------------------------------
@@ -497,8 +853,8 @@ __device__ void logit64(const RouteArgs& a, int t, int g, int m, double& l, doub
 // float64 pass decides every pair whose gaps exceed its bound; only pairs
 // still undecided (in practice exact ties) take the fixed-point path.
 __device__ void exact_rank_pair(const RouteArgs& a, int t, int g, int* sel) {
-  __shared__ Exact ex[kRouteWarps][kMaxM];
-  __shared__ double l64[kRouteWarps][kMaxM], e64[kRouteWarps][kMaxM];
+  __shared__ Exact ex[kRouteMaxWarps][kMaxM];
+  __shared__ double l64[kRouteMaxWarps][kMaxM], e64[kRouteMaxWarps][kMaxM];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = a.M, k = a.k;
   bool bad = false;
@@ -596,14 +952,48 @@ cudaError_t launch_route_gm(const RouteArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int GM>
+cudaError_t launch_route_wres(const RouteArgs& a, cudaStream_t st) {
+  static int configured = -1;
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int smem = static_cast<int>(WresLayout<GM>(a.dm).total);
+  if (configured != dev) {  // the largest size this kernel is ever launched with
+    e = cudaFuncSetAttribute(route_wres_kernel<GM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kWresMaxSmem);
+    if (e != cudaSuccess) return e;
+    configured = dev;
+  }
+  const int npairs = a.dm * GM / 4;
+  route_pairs_kernel<GM><<<(npairs + 255) / 256, 256, 0, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int ntiles = (a.T + kWresTok - 1) / kWresTok;
+  const int grid = ntiles < sms ? ntiles : sms;
+  route_wres_kernel<GM><<<grid, kWresThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+// The shared-memory-resident kernel when W_r fits and each K slice is a whole
+// number of 8-value groups; the streamed kernel otherwise.
+template <int GM>
+cudaError_t launch_route_any(const RouteArgs& a, cudaStream_t st) {
+  const bool fits = a.dm % (8 * WresShape<GM>::KS) == 0 &&
+                    static_cast<int64_t>(a.dm) * GM * 4 <= kWresMaxW &&
+                    WresLayout<GM>(a.dm).total <= static_cast<size_t>(kWresMaxSmem);
+  return fits ? launch_route_wres<GM>(a, st) : launch_route_gm<GM>(a, st);
+}
+
 }  // namespace
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   switch (a.G * a.M) {
-    case 4: return launch_route_gm<4>(a, st);
-    case 8: return launch_route_gm<8>(a, st);
-    case 16: return launch_route_gm<16>(a, st);
-    case 32: return launch_route_gm<32>(a, st);
+    case 4: return launch_route_any<4>(a, st);
+    case 8: return launch_route_any<8>(a, st);
+    case 16: return launch_route_any<16>(a, st);
+    case 32: return launch_route_any<32>(a, st);
     default: return cudaErrorInvalidValue;
   }
 }
