@@ -331,6 +331,17 @@ void gqe_set_profile_events(void* begin, void* end);
  * each call; returns the previous value. */
 int64_t gqe_set_pair_threshold(int64_t kv_bytes);
 
+/* Router kernel choice (tuning; no counterpart on the pages).  gqe_route keeps
+ * W_r in shared memory (float32, one CTA of 16 warps per SM over 64-token
+ * tiles) when d_model * G * M <= 16384, d_model is a multiple of 128 (of 64
+ * when G*M = 32) and the call has at least 3 such tiles per SM; otherwise it
+ * streams W_r from a float32 copy.  Both take the same certified decisions
+ * (top-k identical; p and w within float32 rounding of each other).
+ * on = 1 takes the resident kernel whenever W_r fits, whatever the token
+ * count; 0 restores the default; a negative value only reads the setting.
+ * Process-wide, read at each call; returns the previous setting (0 or 1). */
+int32_t gqe_set_router_resident(int32_t on);
+
 /* ------------------------------------------------------------------------
  * Training: the forward call that also keeps each row's log-sum-exp, and the
  * backward pass of the path.

@@ -10,7 +10,7 @@ from ._lib import (  # noqa: F401
     gqe_attention_append, gqe_attention_decode, gqe_attention_prefill, gqe_decode_workspace_size,
     gqe_attention_prefill_static, gqe_bucket,
     gqe_dense_gqa_prefill, gqe_get_device_status, gqe_kv_cache_bytes, gqe_route,
-    gqe_selftest_bounded_wait, gqe_set_pair_threshold, gqe_set_profile_events, gqe_status_string,
+    gqe_selftest_bounded_wait, gqe_set_pair_threshold, gqe_set_profile_events, gqe_set_router_resident, gqe_status_string,
     gqe_workspace_size, gqe_static_device_status, gqe_linear, gqe_routed_q_project,
     gqe_layer_prefill, gqe_dense_layer_prefill, gqe_prefill_chunk_workspace_size,
     gqe_attention_prefill_chunk, gqe_attention_prefill_train, gqe_prefill_backward_workspace_size,

@@ -17,7 +17,7 @@ EXPORTS = (
     "gqe_workspace_size", "gqe_route", "gqe_bucket", "gqe_attention_prefill",
     "gqe_dense_gqa_prefill", "gqe_get_device_status", "gqe_kv_cache_bytes",
     "gqe_status_string", "gqe_selftest_bounded_wait", "gqe_set_profile_events",
-    "gqe_attention_prefill_static", "gqe_set_pair_threshold", "gqe_decode_workspace_size",
+    "gqe_attention_prefill_static", "gqe_set_pair_threshold", "gqe_set_router_resident", "gqe_decode_workspace_size",
     "gqe_attention_decode", "gqe_append_workspace_size", "gqe_attention_append",
     "gqe_static_device_status", "gqe_linear", "gqe_routed_q_project", "gqe_layer_prefill",
     "gqe_dense_layer_prefill", "gqe_prefill_chunk_workspace_size", "gqe_attention_prefill_chunk",
@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
         "gqe_set_profile_events": (None, [P, P]),
         "gqe_attention_prefill_static": (I32, [S, P, P, P, P, P, P, P, P, P, I64, P]),
         "gqe_set_pair_threshold": (I64, [I64]),
+        "gqe_set_router_resident": (I32, [I32]),
         "gqe_decode_workspace_size": (SZ, [S]),
         "gqe_attention_decode": (I32, [S, P, P, P, P, P, P, P, P, P, P, P, I64, P, SZ, P]),
         "gqe_append_workspace_size": (SZ, [S, I32]),
@@ -169,6 +170,12 @@ def gqe_set_pair_threshold(kv_bytes):
     """Working-set size (bytes) from which d = 64 attention uses the pair
     kernel (0: always, negative: never); returns the previous value."""
     return int(LIB.gqe_set_pair_threshold(int(kv_bytes)))
+
+
+def gqe_set_router_resident(on):
+    """1: the W_r-resident router whenever W_r fits; 0: by token count (the
+    default); negative: read only.  Returns the previous setting."""
+    return int(LIB.gqe_set_router_resident(int(on)))
 
 
 def gqe_attention_prefill_static(dm, Q, Qs, K, V, topk_idx, w, O_sel, o_bar, s_out,

@@ -265,6 +265,8 @@ gqe_status gqe_dense_gqa_prefill(const gqe_dims* dims, const void* Q, const void
 
 int64_t gqe_set_pair_threshold(int64_t kv_bytes) { return set_pair_threshold(kv_bytes); }
 
+int32_t gqe_set_router_resident(int32_t on) { return set_route_force_resident(on); }
+
 // ------------------------------------------------------------ backward
 
 namespace {

@@ -98,6 +98,9 @@ struct RouteArgs {
   int tok;              // tokens per route_kernel tile (set by the launcher)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
+// 1: the shared-memory-resident router whenever it fits; 0: by token count;
+// negative: no change.  Returns the previous setting.
+int set_route_force_resident(int on);
 
 // Chunked prefill over a cache: query row i of sequence b sits at absolute
 // position q_off[b] + i of a KV sequence of T slots, and sees slots

@@ -395,6 +395,9 @@ __global__ void __launch_bounds__(kRouteThreads, 3) route_kernel(const RouteArgs
 // D of the bound |l_hat - l| <= D u ||x|| ||w_c|| used to certify each
 // decision, as in route_kernel; the steps after the logits are
 // route_tile_epilogue's.
+// Tests set this to take the resident kernel at any token count.
+bool g_route_force_resident = false;
+
 constexpr int kWresWarps = 16;
 constexpr int kWresThreads = 32 * kWresWarps;
 constexpr int kWresTok = 64;                   // tokens per tile (two per lane)
@@ -976,17 +979,33 @@ cudaError_t launch_route_wres(const RouteArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// The shared-memory-resident kernel when W_r fits and each K slice is a whole
-// number of 8-value groups; the streamed kernel otherwise.
+// The shared-memory-resident kernel when W_r fits, each K slice is a whole
+// number of 8-value groups and there are at least kWresMinTiles tiles per SM
+// (its per-CTA start, loading all of W_r, costs about as much as a tile; with
+// fewer tokens the streamed kernel measured as fast or faster); the streamed
+// kernel otherwise.
+constexpr int kWresMinTiles = 3;
+
 template <int GM>
 cudaError_t launch_route_any(const RouteArgs& a, cudaStream_t st) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const bool fits = a.dm % (8 * WresShape<GM>::KS) == 0 &&
                     static_cast<int64_t>(a.dm) * GM * 4 <= kWresMaxW &&
                     WresLayout<GM>(a.dm).total <= static_cast<size_t>(kWresMaxSmem);
-  return fits ? launch_route_wres<GM>(a, st) : launch_route_gm<GM>(a, st);
+  const bool many = static_cast<int64_t>(a.T) >= static_cast<int64_t>(kWresMinTiles) * sms * kWresTok;
+  return fits && (many || g_route_force_resident) ? launch_route_wres<GM>(a, st)
+                                                  : launch_route_gm<GM>(a, st);
 }
 
 }  // namespace
+
+int set_route_force_resident(int on) {
+  const int prev = g_route_force_resident ? 1 : 0;
+  if (on >= 0) g_route_force_resident = on != 0;
+  return prev;
+}
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
   switch (a.G * a.M) {

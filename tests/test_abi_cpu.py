@@ -111,6 +111,21 @@ def test_pair_threshold_is_a_host_setting():
     assert prev == 96 << 20  # the default: 96 MiB of K/V
 
 
+def test_router_resident_is_a_host_setting():
+    """The router kernel choice: default 0 (by token count), set, read back
+    through the previous-value return (a negative value only reads),
+    restored.  No device is touched."""
+    prev = gqe.gqe_set_router_resident(-1)
+    assert prev == 0
+    try:
+        assert gqe.gqe_set_router_resident(1) == 0
+        assert gqe.gqe_set_router_resident(-1) == 1
+        assert gqe.gqe_set_router_resident(0) == 1
+    finally:
+        gqe.gqe_set_router_resident(prev)
+    assert gqe.gqe_set_router_resident(-1) == 0
+
+
 
 def test_decode_rejects_bad_arguments():
     """gqe_attention_decode validates before launching (dims.S is the cache

@@ -1,12 +1,16 @@
 """The router at every (d_model, G*M) shape class its kernels take: top-k
 indices bit-exact against the oracle, p and w within float32 rounding.
 
-The router keeps W_r in shared memory when d_model is a multiple of 128 and
-W_r (float32) plus two tiles of x fit, and streams it from a float32 copy
-otherwise; these shapes reach both, with every column-group split of the
-first (G*M = 4, 8, 16, 32), with Gaussian data (certified decisions), with a
-value set that makes many logits tie exactly (the exact fix-up), and with
-products spread over many binary orders (the wide fixed-point accumulator).
+The router keeps W_r in shared memory when W_r (float32) fits and d_model
+splits into whole 8-value groups per K slice, and streams it from a float32
+copy otherwise; by default the resident kernel also needs 3 tiles of 64
+tokens per SM, so every test here runs twice: with the resident kernel forced
+wherever it fits, and with the default choice (the streamed kernel at these
+token counts).  The shapes reach every column-group split of the resident
+kernel (G*M = 4, 8, 16, 32) and the streamed fallbacks, with Gaussian data
+(certified decisions), with a value set that makes many logits tie exactly
+(the exact fix-up), and with products spread over many binary orders (the
+wide fixed-point accumulator).
 """
 import numpy as np
 import pytest
@@ -21,18 +25,26 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
 
+import moe_routed_grouped_b200 as gqe  # noqa: E402
 from moe_routed_grouped_b200.layer import GqePrefill  # noqa: E402
+
+
+@pytest.fixture(params=[1, 0], ids=["resident", "default"])
+def resident(request):
+    prev = gqe.gqe_set_router_resident(request.param)
+    yield request.param
+    gqe.gqe_set_router_resident(prev)
 
 # (G, M, k, d_model)
 SHAPES = [
-    (8, 2, 1, 128),    # G*M = 16 (two column groups, 16-token tiles), 4 row pairs a slice
+    (8, 2, 1, 128),    # G*M = 16: 16 K slices of 8 values
     (8, 2, 1, 256),
     (8, 2, 1, 512),
     (8, 2, 1, 1024),   # the 250M-layer and long-context shapes
-    (2, 2, 1, 256),    # G*M = 4: 32-token tiles
+    (2, 2, 1, 256),    # G*M = 4
     (4, 2, 2, 1024),   # G*M = 8, k = M
-    (8, 4, 2, 512),    # G*M = 32: four column groups, 8-token tiles
-    (4, 2, 2, 2048),   # streamed: two x tiles do not fit
+    (8, 4, 2, 512),    # G*M = 32: two column groups, 8 K slices
+    (4, 2, 2, 2048),   # G*M = 8 with 64 KB of W_r
     (8, 4, 2, 4096),   # streamed: W_r does not fit (the wide-grouping shape)
     (8, 2, 1, 64),     # streamed: d_model not a multiple of 128
 ]
@@ -48,7 +60,7 @@ def _route(x, Wb, bias, G, M, k, dm):
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
-def test_router_gaussian(shape):
+def test_router_gaussian(shape, resident):
     G, M, k, dm = shape
     rng = np.random.default_rng(31000 + G * 1000 + dm)
     S = 1000  # ragged against every tile size
@@ -63,7 +75,7 @@ def test_router_gaussian(shape):
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
-def test_router_exact_ties(shape):
+def test_router_exact_ties(shape, resident):
     """Duplicated columns tie exactly everywhere (the lower index must win);
     x and W_r from a small value set tie many other logits too."""
     G, M, k, dm = shape
@@ -86,7 +98,7 @@ def test_router_exact_ties(shape):
 
 @pytest.mark.parametrize("shape", [SHAPES[1], SHAPES[3], SHAPES[6], SHAPES[9]],
                          ids=lambda s: "x".join(map(str, s)))
-def test_router_wide_exponent_range(shape):
+def test_router_wide_exponent_range(shape, resident):
     G, M, k, dm = shape
     rng = np.random.default_rng(33000 + dm)
     S = 200
