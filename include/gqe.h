@@ -448,6 +448,13 @@ gqe_status gqe_routed_q_project(const gqe_dims* dims, const void* x, const void*
  *  topk_idx, p, w as for gqe_route;  Q bf16 [B, S, N, d] (selected rows);
  *  Qs bf16 [B, S, d];  K, V bf16 [B, S, G, d];
  *  concat    bf16 [B*S, (G*k + G + 1)*d];  y float32 [B, S, d_model]
+ * K, V and Qs do not depend on the routing, so they are computed on a second
+ * stream the library keeps per device (created on first use), ordered after
+ * the work already in `stream` and joined back into `stream` before the
+ * attention call by events; everything the call writes is complete when
+ * `stream` reaches the end of the call, as with the other entry points.
+ * Several host threads calling this on one device share that stream (their
+ * projections then run in turn).
  */
 gqe_status gqe_layer_prefill(const gqe_dims* dims, const void* x, const void* W_Q,
                              const void* W_K, const void* W_V, const void* W_s, const void* W_r,

@@ -468,15 +468,36 @@ gqe_status gqe_layer_prefill(const gqe_dims* dims, const void* x, const void* W_
   const int32_t T = dims->B * dims->S, dm = dims->d_model, d = dims->d, G = dims->G;
   const int64_t row = static_cast<int64_t>(G * dims->k + G + 1) * d;
   if (!aligned16(concat) || !aligned16(y)) return GQE_ERR_INVALID_ARG;
+  // K, V and Qs do not depend on the routing: they run on the side stream
+  // while this stream routes and projects the selected query heads; the
+  // attention call waits for both.
+  cudaStream_t s = static_cast<cudaStream_t>(stream), side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if (side_stream(&side) != cudaSuccess ||
+      cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+    if (fork) cudaEventDestroy(fork);
+    return GQE_ERR_CUDA;
+  }
+  // destroying an event whose record is still pending is allowed
+  struct Events {
+    cudaEvent_t a, b;
+    ~Events() {
+      cudaEventDestroy(a);
+      cudaEventDestroy(b);
+    }
+  } guard{fork, join};
+  if (cudaEventRecord(fork, s) != cudaSuccess || cudaStreamWaitEvent(side, fork, 0) != cudaSuccess)
+    return GQE_ERR_CUDA;
+  if ((st = gqe_linear(T, dm, G, d, x, dm, W_K, K, int64_t(G) * d, 0, side)) != GQE_OK) return st;
+  if ((st = gqe_linear(T, dm, G, d, x, dm, W_V, V, int64_t(G) * d, 0, side)) != GQE_OK) return st;
+  if ((st = gqe_linear(T, dm, 1, d, x, dm, W_s, Qs, d, 0, side)) != GQE_OK) return st;
+  if (cudaEventRecord(join, side) != cudaSuccess) return GQE_ERR_CUDA;
   if ((st = gqe_route(&db, x, W_r, bias, topk_idx, p, w, ws, ws_bytes, stream)) != GQE_OK)
     return st;
-  if ((st = gqe_linear(T, dm, G, d, x, dm, W_K, K, int64_t(G) * d, 0, stream)) != GQE_OK)
-    return st;
-  if ((st = gqe_linear(T, dm, G, d, x, dm, W_V, V, int64_t(G) * d, 0, stream)) != GQE_OK)
-    return st;
-  if ((st = gqe_linear(T, dm, 1, d, x, dm, W_s, Qs, d, 0, stream)) != GQE_OK) return st;
   if ((st = gqe_routed_q_project(&db, x, W_Q, topk_idx, Q, ws, ws_bytes, stream)) != GQE_OK)
     return st;
+  if (cudaStreamWaitEvent(s, join, 0) != cudaSuccess) return GQE_ERR_CUDA;
   uint16_t* cb = static_cast<uint16_t*>(concat);
   const int64_t a = int64_t(G) * dims->k * d;
   if ((st = gqe_attention_prefill(&db, Q, Qs, K, V, topk_idx, w, cb, cb + a, cb + a + G * d, row,

@@ -100,6 +100,22 @@ bool map_bsd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, in
   return encode_map(m, dt, 3, base, dims, strides, box);
 }
 
+cudaError_t side_stream(cudaStream_t* out) {
+  static std::mutex mu;
+  static cudaStream_t streams[kMaxSideDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return e;
+  }
+  *out = streams[dev];
+  return cudaSuccess;
+}
+
 void set_profile_events(cudaEvent_t begin, cudaEvent_t end) {
   std::lock_guard<std::mutex> lock(g_prof_mu);
   g_prof_begin = begin;

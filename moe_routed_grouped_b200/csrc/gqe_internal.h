@@ -292,5 +292,10 @@ bool map_bsd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int B, in
 // The attention launch, bracketed by the profiling events when they are set.
 void set_profile_events(cudaEvent_t begin, cudaEvent_t end);
 cudaError_t timed_attention(const AttnArgs& a, int64_t n_list, cudaStream_t s);
+// A non-blocking stream per device, created on first use and kept for the
+// process: work that does not depend on the caller's stream runs there,
+// ordered against it by events.
+constexpr int kMaxSideDevices = 64;
+cudaError_t side_stream(cudaStream_t* out);
 
 }  // namespace gqe
