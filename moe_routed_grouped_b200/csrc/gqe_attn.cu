@@ -346,8 +346,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
     nrows = min(kTileM, S - row0);
     nkv = qt + 1;
   } else {
-    if (static_cast<int>(blockIdx.x) >= *a.tile_count) return;
+    // the list holds at least gridDim.x entries: read the entry and the count
+    // together rather than one after the other
+    const int count = *a.tile_count;
     const TileDesc td = a.tiles[blockIdx.x];
+    if (static_cast<int>(blockIdx.x) >= count) return;
     if (td.nkv == 0) return;  // empty second half of a pair
     kind = td.code >> 24;
     const int id = td.code & 0xFFFFFF;
@@ -502,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
     const int r = warp * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int rv = min(r, nrows - 1);
-    int pos, pos_first;
+    int pos, pos_first, slot = 0;
     if (kind == kRouted) {
       pos = a.bucket_tok[bstart + row0 + rv];
       pos_first = a.bucket_tok[bstart + row0];
@@ -511,6 +514,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
                                 r < nrows);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarQFull]);
+      // the row's output slot (rank of expert m among its selections), read
+      // now so the epilogue does not wait for it
+      const int32_t* sel = a.topk_idx + ((static_cast<int64_t>(b) * S + pos) * G + g) * a.k;
+      for (int q = 0; q < a.k; ++q)
+        if (sel[q] == m) slot = q;
     } else {
       pos = row0 + rv;
       pos_first = row0;
@@ -543,10 +551,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
       } else if (kind == kShared) {
         dst = static_cast<uint8_t*>(a.s_out) + (tokrow * a.out_row_stride) * esz;
       } else {
-        const int32_t* sel = a.topk_idx + (tokrow * G + g) * a.k;
-        int slot = 0;
-        for (int q = 0; q < a.k; ++q)
-          if (sel[q] == m) slot = q;
         dst = static_cast<uint8_t*>(a.O_sel) +
               (tokrow * a.out_row_stride + static_cast<int64_t>(g * a.k + slot) * D) * esz;
         if (a.k == 1)
