@@ -690,7 +690,7 @@ def e2e_measure(torch, w, L, dev, steps):
 # capture one launch (inputs from torch's generator; a few hundred MB on the
 # device at most, more than the 126 MB L2).
 NCU_CASES = ("attn_d64_32k", "attn_d128_32k", "pair_d64_32k", "layer250m", "bwd_d64_8k",
-             "decode_32k")
+             "decode_32k", "route_32k")
 
 
 def run_ncu_case(torch, name, device, reps=2):
@@ -713,6 +713,15 @@ def run_ncu_case(torch, name, device, reps=2):
         L = GqeLayer(B, S, N, G, k, d, dm, device=device)
         for _ in range(reps):
             L.forward(x, *W, None, Wo)
+    elif name == "route_32k":  # the router alone on the 32k biased shape (W_r-resident kernel)
+        B, S, N, G, k, d, dm = 1, 32768, 16, 8, 1, 64, 1024
+        M = N // G
+        bias = torch.zeros(G, M, dtype=torch.float32, device=device)
+        bias[:, 0] = 1.5
+        x, Wr = rn(B, S, dm), rn(G, dm, M, std=dm ** -0.5)
+        L = GqePrefill(B, S, N, G, k, d, dm, device=device)
+        for _ in range(reps):
+            L.route(x, Wr, bias)
     elif name == "decode_32k":
         B, T, N, G, k, d, dm = 1, 32768, 16, 8, 1, 64, 1024
         L = GqeDecode(B, T, N, G, k, d, dm, device=device)
