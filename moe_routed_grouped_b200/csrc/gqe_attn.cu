@@ -323,6 +323,7 @@ __device__ __noinline__ void store_rows_coalesced(float* stage, uint32_t taddr_o
 template <int D>
 __global__ void __launch_bounds__(kThreads, Cfg<D>::kMinBlocks)
     attn_kernel(const __grid_constant__ AttnArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -660,6 +661,7 @@ __device__ __forceinline__ Slot decode_tile(const TileDesc& td, const AttnArgs& 
 
 __global__ void __launch_bounds__(kPairThreads, 1)
     attn_pair_kernel(const __grid_constant__ AttnArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   using C = PairCfg;
   constexpr int D = C::D;
   extern __shared__ uint8_t smem_raw[];
@@ -921,8 +923,8 @@ cudaError_t launch_d(const AttnArgs& a, int64_t grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  attn_kernel<D><<<static_cast<unsigned>(grid), kThreads, Cfg<D>::kSmemBytes, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(attn_kernel<D>, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
+                    Cfg<D>::kSmemBytes, st, a);
 }
 
 // K/V working set (bytes) from which the d = 64 calls use the pair kernel:
@@ -941,8 +943,8 @@ cudaError_t launch_pair(const AttnArgs& a, int64_t grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  attn_pair_kernel<<<static_cast<unsigned>(grid), kPairThreads, PairCfg::kSmemBytes, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(attn_pair_kernel, dim3(static_cast<unsigned>(grid)), dim3(kPairThreads),
+                    PairCfg::kSmemBytes, st, a);
 }
 
 }  // namespace

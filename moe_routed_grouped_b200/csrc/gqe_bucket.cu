@@ -262,6 +262,7 @@ __device__ void convert_v_body(const ConvertArgs& a, int block, int nblocks) {
 // finishes last (fenced counter) sorts the work list.
 __global__ void __launch_bounds__(kBucketThreads)
     prep_kernel(const BucketArgs a, const ConvertArgs cv, int with_schedule) {
+  grid_dep_wait();  // launched with launch_pdl
   extern __shared__ int hist[];
   __shared__ int is_last;
   const int nbucket = a.B * a.G;
@@ -285,6 +286,7 @@ __global__ void convert_v_kernel(const ConvertArgs a) { convert_v_body(a, blockI
 // o_bar[t, g] = sum_j w[t, g, j] * O_sel[t, g, j] in slot order
 // (review §二 三个关键部件, the renormalised weighted-sum slot); k > 1 only.
 __global__ void combine_kernel(const CombineArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   const int lanes_per_row = a.d / 4;  // 4 elements per thread
   const int64_t rows = static_cast<int64_t>(a.T) * a.G;
   const int64_t tid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
@@ -352,8 +354,8 @@ cudaError_t launch_prep(const BucketArgs& a, const ConvertArgs* cv, bool with_sc
     if (nconv > cap) nconv = cap;
     if (nconv < 1) nconv = 1;
   }
-  prep_kernel<<<a.B * a.G + nconv, kBucketThreads, smem, st>>>(a, c, with_schedule ? 1 : 0);
-  return cudaGetLastError();
+  return launch_pdl(prep_kernel, dim3(a.B * a.G + nconv), dim3(kBucketThreads), smem, st, a, c,
+                    with_schedule ? 1 : 0);
 }
 
 cudaError_t launch_convert_v(const ConvertArgs& a, cudaStream_t st) {
@@ -370,8 +372,7 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
   int64_t blocks = (work + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  combine_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, a);
 }
 
 }  // namespace gqe

@@ -22,6 +22,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Programmatic dependent launch: a kernel launched with launch_pdl may start
+// while the previous kernel in its stream finishes; this waits until that
+// kernel has completed and its memory is visible.  Every such kernel calls it
+// before its first global-memory access (a no-op without a prerequisite).
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Latch the first device-side error into the workspace status word.
 __device__ __forceinline__ void latch_status(int* status, int code) {
   atomicCAS(status, 0, code);

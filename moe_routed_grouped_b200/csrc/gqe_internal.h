@@ -1,6 +1,8 @@
 // Internal declarations shared by the GQE kernels and the C-ABI layer.
 #pragma once
 
+#include <utility>
+
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
@@ -97,6 +99,25 @@ struct RouteArgs {
   int T, dm, G, M, k;
   int tok;              // tokens per route_kernel tile (set by the launcher)
 };
+// Launch with programmatic stream serialization: the kernel's CTAs may start
+// as the previous kernel's CTAs retire; the kernel must call grid_dep_wait()
+// before it touches global memory.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st);
 // 1: the shared-memory-resident router whenever it fits; 0: by token count;
 // negative: no change.  Returns the previous setting.

@@ -244,6 +244,7 @@ __device__ __forceinline__ void route_tile_epilogue(const RouteArgs& a, const fl
 // of the bound |l_hat - l| <= D u ||x|| ||w_c||, u = 2^-24.
 template <int GM>
 __global__ void __launch_bounds__(kRouteThreads, 3) route_kernel(const RouteArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   using Sh = RouteShape<GM>;
   constexpr int TPL = Sh::kTPL;
   const int TOK = a.tok;
@@ -446,6 +447,7 @@ struct WresLayout {
 // of columns c, c+1 (p = d / (GM/2), c = 2 (d % (GM/2))).
 template <int GM>
 __global__ void __launch_bounds__(256) route_pairs_kernel(const RouteArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   const int d = blockIdx.x * 256 + threadIdx.x;
   if (d >= a.dm * GM / 4) return;
   const int dm = a.dm, M = a.M;
@@ -460,6 +462,7 @@ __global__ void __launch_bounds__(256) route_pairs_kernel(const RouteArgs a) {
 
 template <int GM>
 __global__ void __launch_bounds__(kWresThreads, 1) route_wres_kernel(const RouteArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   using Sh = WresShape<GM>;
   constexpr int CPW = Sh::CPW, CGW = Sh::CGW, KS = Sh::KS;
   extern __shared__ __align__(128) uint8_t wres_smem_raw[];
@@ -951,8 +954,7 @@ cudaError_t launch_route_gm(const RouteArgs& a, cudaStream_t st) {
   b.tok = static_cast<int>(want < 1 ? 1 : (want > RouteShape<GM>::kTok ? RouteShape<GM>::kTok : want));
   const int ntiles = (a.T + b.tok - 1) / b.tok;
   const int grid = ntiles < 4 * sms ? ntiles : 4 * sms;
-  route_kernel<GM><<<grid, kRouteThreads, smem, st>>>(b);
-  return cudaGetLastError();
+  return launch_pdl(route_kernel<GM>, dim3(grid), dim3(kRouteThreads), smem, st, b);
 }
 
 template <int GM>
@@ -970,13 +972,11 @@ cudaError_t launch_route_wres(const RouteArgs& a, cudaStream_t st) {
     configured = dev;
   }
   const int npairs = a.dm * GM / 4;
-  route_pairs_kernel<GM><<<(npairs + 255) / 256, 256, 0, st>>>(a);
-  e = cudaGetLastError();
+  e = launch_pdl(route_pairs_kernel<GM>, dim3((npairs + 255) / 256), dim3(256), 0, st, a);
   if (e != cudaSuccess) return e;
   const int ntiles = (a.T + kWresTok - 1) / kWresTok;
   const int grid = ntiles < sms ? ntiles : sms;
-  route_wres_kernel<GM><<<grid, kWresThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(route_wres_kernel<GM>, dim3(grid), dim3(kWresThreads), smem, st, a);
 }
 
 // The shared-memory-resident kernel when W_r fits, each K slice is a whole
