@@ -281,7 +281,10 @@ __global__ void __launch_bounds__(kBucketThreads)
   if (threadIdx.x == 0) *a.done = 0;  // ready for the next call
 }
 
-__global__ void convert_v_kernel(const ConvertArgs a) { convert_v_body(a, blockIdx.x, gridDim.x); }
+__global__ void convert_v_kernel(const ConvertArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
+  convert_v_body(a, blockIdx.x, gridDim.x);
+}
 
 // o_bar[t, g] = sum_j w[t, g, j] * O_sel[t, g, j] in slot order
 // (review §二 三个关键部件, the renormalised weighted-sum slot); k > 1 only.
@@ -363,8 +366,7 @@ cudaError_t launch_convert_v(const ConvertArgs& a, cudaStream_t st) {
   int64_t blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  convert_v_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(convert_v_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, a);
 }
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {

@@ -132,6 +132,7 @@ __device__ __forceinline__ void gather_row(uint8_t* dst, int r, const uint16_t* 
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const __grid_constant__ BwdArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -450,6 +451,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const __grid_consta
 // One warp per row: routed slot (token, group, slot) or shared-head token.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   const int lane = threadIdx.x & 31;
   const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t T = static_cast<int64_t>(a.B) * a.S;
@@ -514,19 +516,23 @@ cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(a.B) * a.G * nq);
   cudaError_t e;
   if (a.d == 64) {
-    bwd_prep_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(bwd_prep_kernel<64>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+                        a)) != cudaSuccess)
+      return e;
     if ((e = cudaFuncSetAttribute(bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BwdCfg<64>::kSmemBytes)) != cudaSuccess)
       return e;
-    bwd_kernel<64><<<grid, kBwdThreads, BwdCfg<64>::kSmemBytes, st>>>(a);
+    e = launch_pdl(bwd_kernel<64>, dim3(grid), dim3(kBwdThreads), BwdCfg<64>::kSmemBytes, st, a);
+    if (e != cudaSuccess) return e;
   } else if (a.d == 128) {
-    bwd_prep_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(bwd_prep_kernel<128>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+                        a)) != cudaSuccess)
+      return e;
     if ((e = cudaFuncSetAttribute(bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   BwdCfg<128>::kSmemBytes)) != cudaSuccess)
       return e;
-    bwd_kernel<128><<<grid, kBwdThreads, BwdCfg<128>::kSmemBytes, st>>>(a);
+    e = launch_pdl(bwd_kernel<128>, dim3(grid), dim3(kBwdThreads), BwdCfg<128>::kSmemBytes, st, a);
+    if (e != cudaSuccess) return e;
   } else {
     return cudaErrorInvalidValue;
   }

@@ -58,6 +58,7 @@ __device__ __forceinline__ void store_out(void* base, int64_t off, float v, int 
 // end of the chunk.
 template <int D, int HB, bool MULTI>
 __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const DecodeArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   constexpr int L = D / 8;
   constexpr int SPW = 32 / L;
   constexpr int NS = (kDecThreads / 32) * SPW;
@@ -239,6 +240,7 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const De
 // shared head for g = 0.  One thread per output element.
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   // one CTA per (new token row, g); row tr = b * n_new + r
   const int g = static_cast<int>(blockIdx.x % a.G);
   const int64_t tr = blockIdx.x / a.G;
@@ -289,12 +291,11 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
 template <int D, int HB, bool MULTI>
 cudaError_t launch_decode_dh(const DecodeArgs& a, cudaStream_t st) {
   const int64_t ctas = static_cast<int64_t>(a.B) * a.G * a.passes * a.nchunks;
-  decode_partial_kernel<D, HB, MULTI><<<static_cast<unsigned>(ctas), kDecThreads, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(decode_partial_kernel<D, HB, MULTI>, dim3(static_cast<unsigned>(ctas)),
+                             dim3(kDecThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(a.B) * a.n_new * a.G;
-  decode_merge_kernel<D><<<static_cast<unsigned>(rows), D, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(decode_merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(D), 0, st, a);
 }
 
 }  // namespace

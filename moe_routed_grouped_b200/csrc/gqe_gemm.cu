@@ -131,6 +131,7 @@ __device__ __forceinline__ void store_tile_rows(float* stage, uint32_t taddr, ui
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BN>::kMinBlocks)
     gemm_dense_kernel(const __grid_constant__ GemmArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -244,6 +245,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BN>::kMinBlocks)
 template <int D>
 __global__ void __launch_bounds__(kGemmThreads, GemmCfg<D>::kMinBlocks)
     gemm_routed_kernel(const __grid_constant__ GemmArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   using C = GemmCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -399,16 +401,16 @@ cudaError_t launch_gemm_dense(const GemmArgs& a, int bn, cudaStream_t st) {
   switch (bn) {
     case 64:
       if ((e = set_smem(gemm_dense_kernel<64>, GemmCfg<64>::kSmemBytes)) != cudaSuccess) return e;
-      gemm_dense_kernel<64><<<dim3(gm, a.n_total / 64), kGemmThreads, GemmCfg<64>::kSmemBytes, st>>>(a);
-      break;
+      return launch_pdl(gemm_dense_kernel<64>, dim3(gm, a.n_total / 64), dim3(kGemmThreads),
+                        GemmCfg<64>::kSmemBytes, st, a);
     case 128:
       if ((e = set_smem(gemm_dense_kernel<128>, GemmCfg<128>::kSmemBytes)) != cudaSuccess) return e;
-      gemm_dense_kernel<128><<<dim3(gm, a.n_total / 128), kGemmThreads, GemmCfg<128>::kSmemBytes, st>>>(a);
-      break;
+      return launch_pdl(gemm_dense_kernel<128>, dim3(gm, a.n_total / 128), dim3(kGemmThreads),
+                        GemmCfg<128>::kSmemBytes, st, a);
     case 256:
       if ((e = set_smem(gemm_dense_kernel<256>, GemmCfg<256>::kSmemBytes)) != cudaSuccess) return e;
-      gemm_dense_kernel<256><<<dim3(gm, a.n_total / 256), kGemmThreads, GemmCfg<256>::kSmemBytes, st>>>(a);
-      break;
+      return launch_pdl(gemm_dense_kernel<256>, dim3(gm, a.n_total / 256), dim3(kGemmThreads),
+                        GemmCfg<256>::kSmemBytes, st, a);
     default:
       return cudaErrorInvalidValue;
   }
@@ -420,10 +422,12 @@ cudaError_t launch_gemm_routed(const GemmArgs& a, int64_t n_list, cudaStream_t s
   cudaError_t e;
   if (a.d == 64) {
     if ((e = set_smem(gemm_routed_kernel<64>, GemmCfg<64>::kSmemBytes)) != cudaSuccess) return e;
-    gemm_routed_kernel<64><<<static_cast<unsigned>(n_list), kGemmThreads, GemmCfg<64>::kSmemBytes, st>>>(a);
+    return launch_pdl(gemm_routed_kernel<64>, dim3(static_cast<unsigned>(n_list)), dim3(kGemmThreads),
+                      GemmCfg<64>::kSmemBytes, st, a);
   } else if (a.d == 128) {
     if ((e = set_smem(gemm_routed_kernel<128>, GemmCfg<128>::kSmemBytes)) != cudaSuccess) return e;
-    gemm_routed_kernel<128><<<static_cast<unsigned>(n_list), kGemmThreads, GemmCfg<128>::kSmemBytes, st>>>(a);
+    return launch_pdl(gemm_routed_kernel<128>, dim3(static_cast<unsigned>(n_list)), dim3(kGemmThreads),
+                      GemmCfg<128>::kSmemBytes, st, a);
   } else {
     return cudaErrorInvalidValue;
   }

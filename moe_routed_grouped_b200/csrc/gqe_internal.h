@@ -49,7 +49,7 @@ struct WsLayout {
                       // [1] tile count, [2] prep-kernel completion counter
   size_t fix_list;    // int32[B*S*G]: (token*G + g) pairs needing exact routing
   size_t wt;          // float32 [d_model][G*M]: W_r transposed for the router
-  size_t wsq;         // float32 [G*M]: column sums of squares of W_r
+  size_t wsq;         // float32 [ceil(d_model/32)][G*M]: partial column sums of squares of W_r
   size_t v16;         // fp16 [B,S,G,d]: V converted for the P.V product
   size_t bucket_off;  // int32[B*G*M + 1]
   size_t bucket_tok;  // int32[B*G*S*k]
@@ -73,7 +73,7 @@ inline WsLayout make_ws_layout(const gqe_dims& d, int64_t T = -1) {
   L.counters = off;   off += 256;
   L.fix_list = off;   off = align_up(off + sizeof(int32_t) * B * S * G, 256);
   L.wt = off;         off = align_up(off + sizeof(float) * d.d_model * G * M, 256);
-  L.wsq = off;        off = align_up(off + sizeof(float) * G * M, 256);
+  L.wsq = off;        off = align_up(off + sizeof(float) * ((d.d_model + 31) / 32) * G * M, 256);
   L.v16 = off;        off = align_up(off + sizeof(uint16_t) * B * T * G * hd, 256);
   L.bucket_off = off; off = align_up(off + sizeof(int32_t) * (B * G * M + 1), 256);
   L.bucket_tok = off; off = align_up(off + sizeof(int32_t) * B * G * S * k, 256);
@@ -88,7 +88,7 @@ struct RouteArgs {
   const uint16_t* x;    // bf16 [T, dm]
   const uint16_t* Wr;   // bf16 [G, dm, M]
   float* wt;            // float32 [dm][G*M] (written by the prep kernel)
-  float* wsq;           // float32 [G*M]
+  float* wsq;           // float32 [ceil(dm/32)][G*M] (partial sums by route_prep_kernel)
   const float* bias;    // [G*M] or null
   int32_t* topk_idx;    // [T, G, k]
   float* p;             // [T, G, M]

@@ -30,10 +30,12 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
 
 __device__ void exact_rank_pair(const RouteArgs& a, int t, int g, int* sel_smem);
 
-// W_r [G][dm][M] (bf16) -> wt [dm][G*M] (float32) and the column sums of
-// squares wsq[G*M].  Block b covers rows 32b .. 32b+31; thread (j, col).
+// W_r [G][dm][M] (bf16) -> wt [dm][G*M] (float32) and partial column sums of
+// squares wsq[b][G*M] over rows 32b .. 32b+31 (block b; thread (j, col)),
+// added by route_kernel in block order.
 template <int GM>
 __global__ void __launch_bounds__(32 * GM) route_prep_kernel(const RouteArgs a) {
+  grid_dep_wait();  // launched with launch_pdl
   const int col = threadIdx.x % GM, jj = threadIdx.x / GM;
   const int j = blockIdx.x * 32 + jj;
   const int g = col / a.M, m = col % a.M;
@@ -48,7 +50,7 @@ __global__ void __launch_bounds__(32 * GM) route_prep_kernel(const RouteArgs a) 
   if (threadIdx.x < GM) {
     float s2 = 0.f;
     for (int r = 0; r < 32; ++r) s2 += part[r][threadIdx.x];
-    atomicAdd(&a.wsq[threadIdx.x], s2);
+    a.wsq[blockIdx.x * GM + threadIdx.x] = s2;
   }
 }
 
@@ -259,7 +261,9 @@ __global__ void __launch_bounds__(kRouteThreads, 3) route_kernel(const RouteArgs
       1.01f;
 
   for (int c = tid; c < GM; c += kRouteThreads) {
-    sm.wnorm[c] = sqrtf(a.wsq[c]);
+    float s2 = 0.f;
+    for (int b = 0; b < (dm + 31) / 32; ++b) s2 += a.wsq[b * GM + c];
+    sm.wnorm[c] = sqrtf(s2);
     sm.bias[c] = a.bias ? a.bias[c] : 0.f;
   }
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -942,10 +946,7 @@ cudaError_t launch_route_gm(const RouteArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured = dev;
   }
-  e = cudaMemsetAsync(a.wsq, 0, sizeof(float) * GM, st);
-  if (e != cudaSuccess) return e;
-  route_prep_kernel<GM><<<(a.dm + 31) / 32, 32 * GM, 0, st>>>(a);
-  e = cudaGetLastError();
+  e = launch_pdl(route_prep_kernel<GM>, dim3((a.dm + 31) / 32), dim3(32 * GM), 0, st, a);
   if (e != cudaSuccess) return e;
   // tokens per tile: about two tiles per SM when the tokens allow it, at most
   // kTok (two per lane)
