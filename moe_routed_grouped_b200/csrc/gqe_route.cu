@@ -12,6 +12,8 @@
 // more than the two bounds; otherwise the same CTA recomputes that (token,
 // group) pair with an exact fixed-point (Kulisch-style) accumulation of the
 // products.
+#include <atomic>
+
 #include <cuda_bf16.h>
 
 #include "gqe_device.cuh"
@@ -400,8 +402,9 @@ __global__ void __launch_bounds__(kRouteThreads, 3) route_kernel(const RouteArgs
 // D of the bound |l_hat - l| <= D u ||x|| ||w_c|| used to certify each
 // decision, as in route_kernel; the steps after the logits are
 // route_tile_epilogue's.
-// Tests set this to take the resident kernel at any token count.
-bool g_route_force_resident = false;
+// Tests set this to take the resident kernel at any token count (a host
+// setting read at each call; atomic, as calls may come from several threads).
+std::atomic<int> g_route_force_resident{0};
 
 constexpr int kWresWarps = 16;
 constexpr int kWresThreads = 32 * kWresWarps;
@@ -996,16 +999,14 @@ cudaError_t launch_route_any(const RouteArgs& a, cudaStream_t st) {
                     static_cast<int64_t>(a.dm) * GM * 4 <= kWresMaxW &&
                     WresLayout<GM>(a.dm).total <= static_cast<size_t>(kWresMaxSmem);
   const bool many = static_cast<int64_t>(a.T) >= static_cast<int64_t>(kWresMinTiles) * sms * kWresTok;
-  return fits && (many || g_route_force_resident) ? launch_route_wres<GM>(a, st)
+  return fits && (many || g_route_force_resident.load() != 0) ? launch_route_wres<GM>(a, st)
                                                   : launch_route_gm<GM>(a, st);
 }
 
 }  // namespace
 
 int set_route_force_resident(int on) {
-  const int prev = g_route_force_resident ? 1 : 0;
-  if (on >= 0) g_route_force_resident = on != 0;
-  return prev;
+  return on < 0 ? g_route_force_resident.load() : g_route_force_resident.exchange(on != 0 ? 1 : 0);
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t st) {
