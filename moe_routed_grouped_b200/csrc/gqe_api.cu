@@ -123,7 +123,7 @@ gqe_status attention_prefill_impl(const gqe_dims* dims, int32_t T, const void* Q
                                   const float* w, void* O_sel, void* o_bar, void* s_out,
                                   int64_t out_row_stride, void* ws, size_t ws_bytes,
                                   void* stream, float* lse_sel = nullptr,
-                                  float* lse_s = nullptr) {
+                                  float* lse_s = nullptr, bool list_built = false) {
   gqe_status st = check_dims(dims, false);
   if (st != GQE_OK) return st;
   if (T < dims->S) return GQE_ERR_INVALID_ARG;
@@ -153,7 +153,10 @@ gqe_status attention_prefill_impl(const gqe_dims* dims, int32_t T, const void* Q
   ba.q_off = q_off;
   ba.kv_start = kv_start;
   ba.T = T;
-  cudaError_t e = launch_prep(ba, &cv, true, s);
+  // list_built: the buckets and the one-tile work list for these top-k are
+  // already in the workspace (the layer's routed Q projection built them):
+  // only V is converted
+  cudaError_t e = list_built && !pair ? launch_convert_v(cv, s) : launch_prep(ba, &cv, true, s);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
 
   AttnArgs a = attn_common(dims, wb, L);
@@ -500,8 +503,10 @@ gqe_status gqe_layer_prefill(const gqe_dims* dims, const void* x, const void* W_
   if (cudaStreamWaitEvent(s, join, 0) != cudaSuccess) return GQE_ERR_CUDA;
   uint16_t* cb = static_cast<uint16_t*>(concat);
   const int64_t a = int64_t(G) * dims->k * d;
-  if ((st = gqe_attention_prefill(&db, Q, Qs, K, V, topk_idx, w, cb, cb + a, cb + a + G * d, row,
-                                  ws, ws_bytes, stream)) != GQE_OK)
+  // the routed Q projection left this call's buckets and work list in ws
+  if ((st = attention_prefill_impl(&db, db.S, Q, Qs, K, V, nullptr, nullptr, topk_idx, w, cb,
+                                   cb + a, cb + a + G * d, row, ws, ws_bytes, stream, nullptr,
+                                   nullptr, true)) != GQE_OK)
     return st;
   return gqe_linear(T, static_cast<int32_t>(row), 1, dm, concat, row, W_O, y, dm, 1, stream);
 }
