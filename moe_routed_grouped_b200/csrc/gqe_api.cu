@@ -123,7 +123,8 @@ gqe_status attention_prefill_impl(const gqe_dims* dims, int32_t T, const void* Q
                                   const float* w, void* O_sel, void* o_bar, void* s_out,
                                   int64_t out_row_stride, void* ws, size_t ws_bytes,
                                   void* stream, float* lse_sel = nullptr,
-                                  float* lse_s = nullptr, bool list_built = false) {
+                                  float* lse_s = nullptr, bool list_built = false,
+                                  bool v16_built = false) {
   gqe_status st = check_dims(dims, false);
   if (st != GQE_OK) return st;
   if (T < dims->S) return GQE_ERR_INVALID_ARG;
@@ -154,9 +155,14 @@ gqe_status attention_prefill_impl(const gqe_dims* dims, int32_t T, const void* Q
   ba.kv_start = kv_start;
   ba.T = T;
   // list_built: the buckets and the one-tile work list for these top-k are
-  // already in the workspace (the layer's routed Q projection built them):
-  // only V is converted
-  cudaError_t e = list_built && !pair ? launch_convert_v(cv, s) : launch_prep(ba, &cv, true, s);
+  // already in the workspace (the layer's routed Q projection built them);
+  // v16_built: so is the fp16 copy of V (the layer converts it on its side
+  // stream); what is left of the preparation runs here
+  cudaError_t e = cudaSuccess;
+  if (!(list_built && !pair))
+    e = launch_prep(ba, &cv, true, s);
+  else if (!v16_built)
+    e = launch_convert_v(cv, s);
   if (e != cudaSuccess) return GQE_ERR_CUDA;
 
   AttnArgs a = attn_common(dims, wb, L);
@@ -494,6 +500,14 @@ gqe_status gqe_layer_prefill(const gqe_dims* dims, const void* x, const void* W_
     return GQE_ERR_CUDA;
   if ((st = gqe_linear(T, dm, G, d, x, dm, W_K, K, int64_t(G) * d, 0, side)) != GQE_OK) return st;
   if ((st = gqe_linear(T, dm, G, d, x, dm, W_V, V, int64_t(G) * d, 0, side)) != GQE_OK) return st;
+  // V to fp16 for the attention's P.V (into the workspace), off the critical path
+  const bool pair = pair_kernel_for(db);
+  const WsLayout L = make_ws_layout(db);
+  if (!aligned16(ws) || ws_bytes < L.total) return GQE_ERR_WORKSPACE;
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  ConvertArgs cv{static_cast<const uint16_t*>(V), reinterpret_cast<uint16_t*>(wb + L.v16),
+                 int64_t(T) * G * d, reinterpret_cast<int*>(wb + L.status)};
+  if (!pair && launch_convert_v(cv, side) != cudaSuccess) return GQE_ERR_CUDA;
   if ((st = gqe_linear(T, dm, 1, d, x, dm, W_s, Qs, d, 0, side)) != GQE_OK) return st;
   if (cudaEventRecord(join, side) != cudaSuccess) return GQE_ERR_CUDA;
   if ((st = gqe_route(&db, x, W_r, bias, topk_idx, p, w, ws, ws_bytes, stream)) != GQE_OK)
@@ -503,10 +517,11 @@ gqe_status gqe_layer_prefill(const gqe_dims* dims, const void* x, const void* W_
   if (cudaStreamWaitEvent(s, join, 0) != cudaSuccess) return GQE_ERR_CUDA;
   uint16_t* cb = static_cast<uint16_t*>(concat);
   const int64_t a = int64_t(G) * dims->k * d;
-  // the routed Q projection left this call's buckets and work list in ws
+  // the routed Q projection left this call's buckets and work list in ws, the
+  // side stream its fp16 V
   if ((st = attention_prefill_impl(&db, db.S, Q, Qs, K, V, nullptr, nullptr, topk_idx, w, cb,
                                    cb + a, cb + a + G * d, row, ws, ws_bytes, stream, nullptr,
-                                   nullptr, true)) != GQE_OK)
+                                   nullptr, true, true)) != GQE_OK)
     return st;
   return gqe_linear(T, static_cast<int32_t>(row), 1, dm, concat, row, W_O, y, dm, 1, stream);
 }
