@@ -694,7 +694,7 @@ def e2e_measure(torch, w, L, dev, steps, warmup):
 # capture one launch (inputs from torch's generator; a few hundred MB on the
 # device at most, more than the 126 MB L2).
 NCU_CASES = ("attn_d64_32k", "attn_d128_32k", "pair_d64_32k", "layer250m", "bwd_d64_8k",
-             "decode_32k", "route_32k")
+             "decode_32k", "decode_b8_2k", "route_32k")
 
 
 def run_ncu_case(torch, name, device, reps=2):
@@ -726,8 +726,9 @@ def run_ncu_case(torch, name, device, reps=2):
         L = GqePrefill(B, S, N, G, k, d, dm, device=device)
         for _ in range(reps):
             L.route(x, Wr, bias)
-    elif name == "decode_32k":
-        B, T, N, G, k, d, dm = 1, 32768, 16, 8, 1, 64, 1024
+    elif name.startswith("decode"):  # one sequence over 32k cached tokens, or the bench's B = 8, T = 2k
+        B, T = (1, 32768) if name == "decode_32k" else (8, 2048)
+        N, G, k, d, dm = 16, 8, 1, 64, 1024
         L = GqeDecode(B, T, N, G, k, d, dm, device=device)
         args = (rn(B, dm), rn(G, dm, N // G, std=dm ** -0.5), None, rn(B, N, d), rn(B, d),
                 rn(B, T, G, d), rn(B, T, G, d),

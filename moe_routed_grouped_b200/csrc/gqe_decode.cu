@@ -237,10 +237,16 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const De
 // token, rescale every chunk that holds keys it sees (the partial kernel
 // wrote those) to the common maximum, add, normalise; then
 // o_bar = sum_j w_j * O_j in slot order (review §二 三个关键部件) and the
-// shared head for g = 0.  One thread per output element.
+// shared head for g = 0.  One thread per output element.  A head's chunk
+// maxima and sums are first staged in shared memory by all threads at once,
+// and the chunk loop is unrolled, so the partial outputs' loads are issued
+// in batches instead of one dependent load per chunk; the adds keep chunk
+// order.
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
   grid_dep_wait();  // launched with launch_pdl
+  __shared__ float sm_m[kDecMaxChunks];
+  __shared__ float sm_l[kDecMaxChunks];
   // one CTA per (new token row, g); row tr = b * n_new + r
   const int g = static_cast<int>(blockIdx.x % a.G);
   const int64_t tr = blockIdx.x / a.G;
@@ -266,15 +272,24 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
       ok = ok && m >= 0 && m < a.M;
     }
     float out = nan;  // a rejected position or expert index yields NaN
+    const int64_t p0 = (bg * a.heads + static_cast<int64_t>(r) * (a.k + 1) + j) * a.nchunks;
+    if (j > 0) __syncthreads();  // the previous head's staged values are read
+    if (ok)
+      for (int c = c_lo + e; c < nc; c += D) {
+        sm_m[c] = a.part_m[p0 + c];
+        sm_l[c] = a.part_l[p0 + c];
+      }
+    __syncthreads();
     if (ok) {
-      const int64_t p0 = (bg * a.heads + static_cast<int64_t>(r) * (a.k + 1) + j) * a.nchunks;
       float mx = kNoKeyMax;
-      for (int c = c_lo; c < nc; ++c) mx = fmaxf(mx, a.part_m[p0 + c]);
+      for (int c = c_lo; c < nc; ++c) mx = fmaxf(mx, sm_m[c]);
       float acc = 0.f, lsum = 0.f;
+      const float* po = a.part_o + p0 * D + e;
+#pragma unroll 8
       for (int c = c_lo; c < nc; ++c) {
-        const float sc = exp2f(a.part_m[p0 + c] - mx);
-        acc = fmaf(a.part_o[(p0 + c) * D + e], sc, acc);
-        lsum = fmaf(a.part_l[p0 + c], sc, lsum);
+        const float sc = exp2f(sm_m[c] - mx);
+        acc = fmaf(po[static_cast<int64_t>(c) * D], sc, acc);
+        lsum = fmaf(sm_l[c], sc, lsum);
       }
       out = acc / lsum;
     }
@@ -301,6 +316,7 @@ cudaError_t launch_decode_dh(const DecodeArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
+  if (a.nchunks < 1 || a.nchunks > kDecMaxChunks) return cudaErrorInvalidValue;
   if (a.n_new > 1) {  // several new tokens: per-slot causal bounds
     if (a.d == 64) return launch_decode_dh<64, kDecHeads, true>(a, st);
     if (a.d == 128) return launch_decode_dh<128, kDecHeads, true>(a, st);

@@ -17,6 +17,9 @@ constexpr int kDecHeads = 4;         // head slots per CTA (registers bound it)
 constexpr int kDecUnroll = 4;        // keys in flight per key slot
 constexpr int64_t kDecTargetCtas = 4 * 148;
 constexpr int64_t kDecMinChunk = 256;
+// Chunks per (b, g) never exceed the CTA target: chunk >= ceil(T / want) with
+// want <= kDecTargetCtas, so nchunks = ceil(T / chunk) <= want.
+constexpr int kDecMaxChunks = static_cast<int>(kDecTargetCtas);
 constexpr int kMaxAppend = 64;       // new tokens per sequence in one append call
 
 struct DecodePlan {
@@ -37,7 +40,7 @@ inline DecodePlan make_decode_plan(const gqe_dims& d, int64_t n_new = 1) {
   int64_t chunk = (T + want - 1) / want;
   chunk = (chunk + 63) / 64 * 64;
   P.chunk = chunk < kDecMinChunk ? kDecMinChunk : chunk;
-  P.nchunks = (T + P.chunk - 1) / P.chunk;
+  P.nchunks = (T + P.chunk - 1) / P.chunk;  // <= kDecMaxChunks (the merge stages that many)
   const int64_t parts = B * G * P.heads * P.nchunks;
   size_t off = 0;
   P.status = off;  off += 512;  // status word; bytes 256..511 stay the router's counters
