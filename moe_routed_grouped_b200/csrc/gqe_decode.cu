@@ -237,16 +237,22 @@ __global__ void __launch_bounds__(kDecThreads, 3) decode_partial_kernel(const De
 // token, rescale every chunk that holds keys it sees (the partial kernel
 // wrote those) to the common maximum, add, normalise; then
 // o_bar = sum_j w_j * O_j in slot order (review §二 三个关键部件) and the
-// shared head for g = 0.  One thread per output element.  A head's chunk
-// maxima and sums are first staged in shared memory by all threads at once,
-// and the chunk loop is unrolled, so the partial outputs' loads are issued
-// in batches instead of one dependent load per chunk; the adds keep chunk
-// order.
+// shared head for g = 0.
+//
+// kMergeSplit groups of D threads (thread e of a group: output element e)
+// take the chunks c = c_lo + q, c_lo + q + kMergeSplit, ... of a head, so the
+// partial outputs are loaded by several groups at once; the groups' sums are
+// then added in group order.  A head's chunk maxima and sums are first staged
+// in shared memory by all threads.
+constexpr int kMergeSplit = 4;
+
 template <int D>
-__global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(D * kMergeSplit) decode_merge_kernel(const DecodeArgs a) {
   grid_dep_wait();  // launched with launch_pdl
   __shared__ float sm_m[kDecMaxChunks];
   __shared__ float sm_l[kDecMaxChunks];
+  __shared__ float sm_acc[kMergeSplit][D];
+  __shared__ float sm_lsum[kMergeSplit];
   // one CTA per (new token row, g); row tr = b * n_new + r
   const int g = static_cast<int>(blockIdx.x % a.G);
   const int64_t tr = blockIdx.x / a.G;
@@ -254,7 +260,8 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
   const int r = static_cast<int>(tr % a.n_new);
   const int64_t bg = static_cast<int64_t>(b) * a.G + g;  // partials are per (b, g)
   const int64_t rg = tr * a.G + g;                       // router outputs per (row, g)
-  const int e = threadIdx.x;
+  const int e = static_cast<int>(threadIdx.x) % D;
+  const int q = static_cast<int>(threadIdx.x) / D;
   const int pos = a.pos[b];
   const int lo = a.kv_start ? a.kv_start[b] : 0;
   const bool pos_ok = pos >= 0 && static_cast<int64_t>(pos) + a.n_new - 1 < a.T && lo >= 0 &&
@@ -271,36 +278,49 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
       const int m = a.topk_idx[rg * a.k + j];
       ok = ok && m >= 0 && m < a.M;
     }
-    float out = nan;  // a rejected position or expert index yields NaN
     const int64_t p0 = (bg * a.heads + static_cast<int64_t>(r) * (a.k + 1) + j) * a.nchunks;
     if (j > 0) __syncthreads();  // the previous head's staged values are read
     if (ok)
-      for (int c = c_lo + e; c < nc; c += D) {
+      for (int c = c_lo + static_cast<int>(threadIdx.x); c < nc; c += D * kMergeSplit) {
         sm_m[c] = a.part_m[p0 + c];
         sm_l[c] = a.part_l[p0 + c];
       }
     __syncthreads();
+    float acc = 0.f, lsum = 0.f;
     if (ok) {
       float mx = kNoKeyMax;
       for (int c = c_lo; c < nc; ++c) mx = fmaxf(mx, sm_m[c]);
-      float acc = 0.f, lsum = 0.f;
       const float* po = a.part_o + p0 * D + e;
-#pragma unroll 8
-      for (int c = c_lo; c < nc; ++c) {
+#pragma unroll 4
+      for (int c = c_lo + q; c < nc; c += kMergeSplit) {
         const float sc = exp2f(sm_m[c] - mx);
         acc = fmaf(po[static_cast<int64_t>(c) * D], sc, acc);
         lsum = fmaf(sm_l[c], sc, lsum);
       }
-      out = acc / lsum;
     }
-    if (j < a.k) {
-      store_out(a.O_sel, row + (static_cast<int64_t>(g) * a.k + j) * D + e, out, a.out_fp32);
-      obar = fmaf(a.w[rg * a.k + j], out, obar);
-    } else {
-      store_out(a.s_out, row + e, out, a.out_fp32);
+    sm_acc[q][e] = acc;
+    if (e == 0) sm_lsum[q] = lsum;
+    __syncthreads();
+    if (q == 0) {
+      float out = nan;  // a rejected position or expert index yields NaN
+      if (ok) {
+        float at = 0.f, lt = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMergeSplit; ++i) {
+          at += sm_acc[i][e];
+          lt += sm_lsum[i];
+        }
+        out = at / lt;
+      }
+      if (j < a.k) {
+        store_out(a.O_sel, row + (static_cast<int64_t>(g) * a.k + j) * D + e, out, a.out_fp32);
+        obar = fmaf(a.w[rg * a.k + j], out, obar);
+      } else {
+        store_out(a.s_out, row + e, out, a.out_fp32);
+      }
     }
   }
-  store_out(a.o_bar, row + static_cast<int64_t>(g) * D + e, obar, a.out_fp32);
+  if (q == 0) store_out(a.o_bar, row + static_cast<int64_t>(g) * D + e, obar, a.out_fp32);
 }
 
 template <int D, int HB, bool MULTI>
@@ -310,7 +330,8 @@ cudaError_t launch_decode_dh(const DecodeArgs& a, cudaStream_t st) {
                              dim3(kDecThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(a.B) * a.n_new * a.G;
-  return launch_pdl(decode_merge_kernel<D>, dim3(static_cast<unsigned>(rows)), dim3(D), 0, st, a);
+  return launch_pdl(decode_merge_kernel<D>, dim3(static_cast<unsigned>(rows)),
+                    dim3(D * kMergeSplit), 0, st, a);
 }
 
 }  // namespace
