@@ -163,6 +163,47 @@ def test_decode_workspace_scales_with_the_split():
     assert _lib.gqe_decode_workspace_size(_lib.dims(1, 1 << 20, 16, 8, 1, 64)) <= 2 * long
 
 
+def _decode_chunks(B, T, N, G, k, d, n_new):
+    """Chunks per (b, g) of the decode plan, read back from the workspace
+    size: 512 header bytes, then per-(slot, chunk) maxima, sums and d
+    outputs in float32, each block 256-byte aligned."""
+    dm = _lib.dims(B, T, N, G, k, d)
+    total = (_lib.gqe_decode_workspace_size(dm) if n_new == 1
+             else _lib.gqe_append_workspace_size(dm, n_new))
+    if total == 0:  # a shape the library refuses (size limits): never launched
+        return None
+    up = lambda x: (x + 255) // 256 * 256
+    per = B * G * (k + 1) * n_new
+    for nc in range(1, 4097):
+        parts = per * nc
+        if 512 + 2 * up(4 * parts) + up(4 * parts * d) == total:
+            return nc
+    raise AssertionError(f"no chunk count gives {total} bytes")
+
+
+def test_decode_chunks_stay_within_the_merge_staging():
+    """The merge kernel stages a head's chunk maxima and sums in a fixed
+    shared-memory array of 592 entries (the plan's CTA target), so no shape
+    may split a (b, g) into more chunks than that."""
+    worst, refused = 0, 0
+    for B in (1, 2, 3, 8, 64):
+        for T in (1, 255, 256, 257, 4096, 32768, 100003, 1 << 20, 1 << 22):
+            for (N, G, k) in ((16, 8, 1), (32, 8, 2), (4, 1, 2)):
+                for d in (64, 128):
+                    for n_new in (1, 7, 64):
+                        if n_new > T:
+                            continue
+                        nc = _decode_chunks(B, T, N, G, k, d, n_new)
+                        if nc is None:
+                            refused += 1
+                            continue
+                        assert 1 <= nc <= 592, (B, T, N, G, k, d, n_new, nc)
+                        assert nc == 1 or T > 256 * (nc - 1)  # chunks hold at least 256 keys
+                        worst = max(worst, nc)
+    assert worst > 256  # the sweep reaches the long-chunk regime
+    assert refused < 30   # only the largest caches are refused
+
+
 def test_append_rejects_bad_token_counts():
     dm = _lib.dims(2, 100, 16, 8, 1, 64)
     L = _lib.LIB
